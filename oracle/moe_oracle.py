@@ -1,0 +1,328 @@
+"""CPU oracle for the skew-aware MoE forward layer.
+
+TEST INFRASTRUCTURE ONLY. This is the plain, slow, obviously correct statement of what the
+layer computes, used to check the CUDA library. It shares no code with the library and
+imports nothing from it. Only the tests, the package smoke check and the benchmark's CPU
+baseline leg may import or run it; the product path never does.
+
+Sources (cited by page title and section; the pages print no code and no worked example):
+  [MF]  "MegaFlux" summary (picx.dev/p/e4jAzZ):
+          - "Routing Skew Problem": the skew measure kappa and its uniform case kappa = 1;
+          - Methodology 1, "Problem Formulation": token blocks of at most beta rows,
+            b_e = ceil(c_e / beta), the planner objective min_q max_r l_r with
+            l_r = sum_e q_er, the constraints sum_r q_er = b_e and
+            sum_{e: h(e) != r} 1[q_er > 0] <= s;
+          - Methodology 1, "Bounded Greedy Search": four greedy searches from the
+            no-replica assignment toward tau = ceil(sum_e b_e / P), donor priority
+            (total overload | largest remaining home-expert load) x fan-out (one new copy
+            per expert per round | several);
+          - Methodology 2, expert-computation equation: Z_e = X_e W1_e, Z_e = [G_e, U_e],
+            A_e = SiLU(G_e) * U_e, O_e = A_e W2_e, y_t = sum_{e in S_t} p_{t,e} O_e[t];
+          - Summary and "Theoretical Contributions" 1: router outputs, token counts,
+            expert selections and routing weights are preserved.
+  [UE]  "UltraEP: Exact Load Balancing for Rack-Scale MoE" reading notes, section 4,
+        Algorithm 1: the receiver of a shifted quota is the rank with the most slack that
+        does not already host the expert (used here as the receiver rule).
+  [TE]  TopoEP abstract: plans are deterministic and bitwise identical.
+
+Readings where the pages leave a step open (each is also listed in the design notes):
+  R1  top-k order is by descending logit, ties to the lower expert id; gates are the
+      softmax over the k chosen logits (= full softmax renormalised over the top-k),
+      evaluated in fp64 and rounded to fp32.
+  R2  kappa = E * S / N^2 with S = sum_e c_e^2 and N = sum_e c_e, exact integers, one
+      fp64 rounding; kappa = 0.0 when N = 0 (no routed rows).
+  R3  owner map h(e) = floor(e * P / E) (contiguous equal ranges of experts per slot).
+  R4  the bounded greedy rule of `plan_variant` (donor order, expert order, receiver
+      choice, move size, rounds, stop rule) and the best-variant choice of `plan`.
+  R5  dispatch is a stable counting sort of the (t, j) pairs by expert, token-ascending
+      inside an expert; expert e's i-th row goes to padded row beta*block_off[e] + i.
+  R6  the FFN is evaluated in fp32 from the exact bf16 input values; A is kept in fp32.
+  R7  the combine sums j = 0..k-1 in ascending order in fp32.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+VARIANT_NAMES = ("over/one", "over/multi", "hot/one", "hot/multi")
+
+
+# --------------------------------------------------------------------------- routing
+def route_topk(logits: np.ndarray, k: int) -> tuple[np.ndarray, np.ndarray]:
+    """S_t and p_{t,e} per token: the k largest logits and their renormalised softmax.
+
+    [MF] Summary (router outputs are fixed inputs); reading R1.
+    Returns ids int32 [T, k] (descending logit, ties to the lower id) and gates fp32 [T, k].
+    """
+    logits = np.asarray(logits, dtype=np.float32)
+    if not np.all(np.isfinite(logits)):
+        raise ValueError("router logits must be finite")
+    T, E = logits.shape
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    # a stable ascending sort of -logit keeps equal logits in expert-id order
+    ids = np.argsort(-logits, axis=1, kind="stable")[:, :k].astype(np.int32)
+    sel = np.take_along_axis(logits, ids, axis=1).astype(np.float64)
+    w = np.exp(sel - sel[:, :1])          # sel[:, 0] is the row's largest chosen logit
+    gates = (w / w.sum(axis=1, keepdims=True)).astype(np.float32)
+    return ids, gates
+
+
+def expert_counts(ids: np.ndarray, E: int) -> np.ndarray:
+    """c_e: number of routed (t, j) pairs with ids[t, j] = e.  [MF] Routing Skew Problem."""
+    ids = np.asarray(ids).ravel()
+    if ids.size and (ids.min() < 0 or ids.max() >= E):
+        raise ValueError("expert id out of range")
+    return np.bincount(ids, minlength=E).astype(np.int64)
+
+
+def skew_kappa(counts) -> tuple[int, float]:
+    """(S, kappa): S = sum_e c_e^2 and kappa = E * sum_e (c_e / sum_j c_j)^2.
+
+    [MF] "Routing Skew Problem" equation; reading R2. Written as E*S/N^2 over exact
+    integers, so the single rounding is Python's correctly rounded int/int division.
+    """
+    c = [int(v) for v in counts]
+    E = len(c)
+    S = sum(v * v for v in c)
+    N = sum(c)
+    if N == 0:
+        return 0, 0.0
+    return S, (E * S) / (N * N)
+
+
+# --------------------------------------------------------------------------- blocks
+def block_counts(counts, beta: int) -> list[int]:
+    """b_e = ceil(c_e / beta) (0 for an idle expert).  [MF] Problem Formulation."""
+    return [-(-int(c) // beta) for c in counts]
+
+
+def block_offsets(b) -> list[int]:
+    """Exclusive prefix sum of b_e, E+1 entries; block_off[E] = B = sum_e b_e."""
+    off = [0]
+    for v in b:
+        off.append(off[-1] + int(v))
+    return off
+
+
+def owner(e: int, E: int, P: int) -> int:
+    """h(e), the home slot of expert e.  Reading R3: contiguous equal ranges."""
+    return e * P // E
+
+
+# --------------------------------------------------------------------------- planner
+def plan_variant(b, P: int, s: int, v: int) -> dict:
+    """One bounded greedy search of [MF] "Bounded Greedy Search"; reading R4.
+
+    Variant v = 2*D + F with donor priority D (0: decreasing total overload l_r,
+    1: largest remaining home-expert load max_{h(e)=r} q_er) and fan-out F (0: at most
+    one new copy of an expert per round, 1: several copies per round).
+
+    Start: the no-replica assignment q[e][h(e)] = b_e.  Target: tau = ceil(B / P).
+    A round visits the donors (slots with l_r > tau) in priority order (ties to the
+    lower slot); a donor offers its home experts in order of q[e][r] descending (ties to
+    the lower id); a home expert keeps moving blocks while its donor is above tau:
+      receivers = slots t != r with l_t < tau that either already hold a copy of e
+                  (q[e][t] > 0) or may open one (rep_t < s, and under fan-out "one" e has
+                  not been copied yet in this round);
+      receiver  = the one with the most slack, i.e. least l_t, ties to the lower slot
+                  ([UE] Algorithm 1's receiver rule);
+      move      = min(l_r - tau, tau - l_t, q[e][r]) blocks, the largest that keeps both
+                  ends on their side of tau.
+    The search stops when max_r l_r <= tau or a round moves nothing (bounded: every move
+    lowers the total overload by at least one block).
+    """
+    E = len(b)
+    b = [int(x) for x in b]
+    D, F = v >> 1, v & 1
+    h = [owner(e, E, P) for e in range(E)]
+    q = [[0] * P for _ in range(E)]
+    for e in range(E):
+        q[e][h[e]] = b[e]
+    load = [0] * P
+    for e in range(E):
+        load[h[e]] += b[e]
+    rep = [0] * P
+    B = sum(b)
+    tau = -(-B // P)
+    rounds = 0
+    while max(load) > tau:
+        rounds += 1
+        newcopies = [0] * E
+        progress = False
+        donors = [r for r in range(P) if load[r] > tau]
+        if D == 0:
+            donors.sort(key=lambda r: (-load[r], r))
+        else:
+            donors.sort(key=lambda r: (-max([q[e][r] for e in range(E) if h[e] == r],
+                                              default=0), r))
+        for r in donors:
+            home = sorted((e for e in range(E) if h[e] == r), key=lambda e: (-q[e][r], e))
+            for e in home:
+                while load[r] > tau and q[e][r] > 0:
+                    cand = [t for t in range(P)
+                            if t != r and load[t] < tau
+                            and (q[e][t] > 0
+                                 or (rep[t] < s and (F == 1 or newcopies[e] == 0)))]
+                    if not cand:
+                        break
+                    t = min(cand, key=lambda t: (load[t], t))
+                    delta = min(load[r] - tau, tau - load[t], q[e][r])
+                    if q[e][t] == 0:
+                        rep[t] += 1
+                        newcopies[e] += 1
+                    q[e][r] -= delta
+                    q[e][t] += delta
+                    load[r] -= delta
+                    load[t] += delta
+                    progress = True
+        if not progress:
+            break
+    return {"q": np.array(q, dtype=np.int32).reshape(E, P), "load": load,
+            "makespan": max(load) if P else 0, "replicas": sum(rep), "tau": tau,
+            "B": B, "variant": v, "rounds": rounds}
+
+
+def fixed_makespan(b, P: int) -> int:
+    """Largest slot load of the no-replica (fixed placement) assignment."""
+    E = len(b)
+    load = [0] * P
+    for e in range(E):
+        load[owner(e, E, P)] += int(b[e])
+    return max(load)
+
+
+def plan(b, P: int, s: int, variant_mask: int = 0xF) -> dict:
+    """Run the enabled variants and keep the best.  Reading R4: the best is the
+    lexicographic minimum of (makespan, total replicas, variant index)."""
+    mask = variant_mask & 0xF or 0xF
+    results = [plan_variant(b, P, s, v) for v in range(4) if mask >> v & 1]
+    best = min(results, key=lambda r: (r["makespan"], r["replicas"], r["variant"]))
+    out = dict(best)
+    out["all"] = {r["variant"]: r for r in results}
+    out["fixed_makespan"] = fixed_makespan(b, P)
+    return out
+
+
+def block_list(q: np.ndarray) -> tuple[list[tuple[int, int]], list[int]]:
+    """Expand q into the per-slot block list and its slot offsets.
+
+    Slot r lists its experts in ascending order; expert e's slot-r share is the run of
+    block indices j in [sum_{r' < r} q[e][r'], + q[e][r]).
+    Returns (blocks [(e, j)], slot_off [P+1]).
+    """
+    q = np.asarray(q)
+    E, P = q.shape
+    blocks: list[tuple[int, int]] = []
+    slot_off = [0]
+    for r in range(P):
+        for e in range(E):
+            j0 = int(q[e, :r].sum())
+            for j in range(j0, j0 + int(q[e, r])):
+                blocks.append((e, j))
+        slot_off.append(len(blocks))
+    return blocks, slot_off
+
+
+# --------------------------------------------------------------------------- dispatch
+def dispatch(ids: np.ndarray, gates: np.ndarray, block_off, beta: int):
+    """Tile-aligned dispatch; reading R5.
+
+    Visits the (t, j) pairs in t-major order; the next free row of expert e (starting at
+    beta * block_off[e]) receives the pair.  Returns row_token int32 [R] (-1 on padding
+    rows), row_gate fp32 [R] (0 on padding rows) and tok_row int32 [T, k], with
+    R = beta * block_off[E].
+    """
+    ids = np.asarray(ids)
+    T, k = ids.shape
+    E = len(block_off) - 1
+    R = beta * int(block_off[E])
+    row_token = np.full(R, -1, dtype=np.int32)
+    row_gate = np.zeros(R, dtype=np.float32)
+    tok_row = np.empty((T, k), dtype=np.int32)
+    nxt = [beta * int(block_off[e]) for e in range(E)]
+    for t in range(T):
+        for j in range(k):
+            e = int(ids[t, j])
+            r = nxt[e]
+            nxt[e] += 1
+            if r >= beta * int(block_off[e + 1]):
+                raise ValueError("expert overflows its blocks")
+            row_token[r] = t
+            row_gate[r] = gates[t, j]
+            tok_row[t, j] = r
+    return row_token, row_gate, tok_row
+
+
+def gather_rows(x: np.ndarray, row_token: np.ndarray) -> np.ndarray:
+    """Xp: x[row_token[r]] on valid rows, zeros on padding rows."""
+    xp = np.zeros((len(row_token), x.shape[1]), dtype=x.dtype)
+    valid = row_token >= 0
+    xp[valid] = x[row_token[valid]]
+    return xp
+
+
+# --------------------------------------------------------------------------- FFN
+def silu(g: np.ndarray) -> np.ndarray:
+    """SiLU(g) = g / (1 + exp(-g))."""
+    with np.errstate(over="ignore"):
+        return g / (np.float32(1.0) + np.exp(-g))
+
+
+def expert_ffn(x_rows: np.ndarray, w1: np.ndarray, w2: np.ndarray) -> np.ndarray:
+    """O_e = (SiLU(G_e) * U_e) W2_e for rows of one expert; [MF] expert-computation
+    equation; reading R6.  Shapes: x_rows [n, d], w1 [2f, d] (rows: G then U),
+    w2 [d, f]; all fp32.  Returns O [n, d] fp32."""
+    x_rows = np.asarray(x_rows, dtype=np.float32)
+    f = w1.shape[0] // 2
+    Z = x_rows @ np.asarray(w1, dtype=np.float32).T
+    G, U = Z[:, :f], Z[:, f:]
+    A = silu(G) * U
+    return A @ np.asarray(w2, dtype=np.float32).T
+
+
+def combine(O_rows: np.ndarray, tok_row: np.ndarray, gates: np.ndarray) -> np.ndarray:
+    """y_t = sum_j p_{t,j} O[tok_row[t, j]], j ascending in fp32; reading R7."""
+    T, k = tok_row.shape
+    y = np.zeros((T, O_rows.shape[1]), dtype=np.float32)
+    for j in range(k):
+        y += gates[:, j:j + 1].astype(np.float32) * O_rows[tok_row[:, j]]
+    return y
+
+
+def moe_forward(logits, x, get_expert, k: int, beta: int, P: int, s: int,
+                variant_mask: int = 0xF) -> dict:
+    """The whole forward layer: route, histogram + kappa, blocks, plan, dispatch,
+    per-expert FFN, combine.  `x` is [T, d] fp32 holding bf16 values; `get_expert(e)`
+    returns (w1 [2f, d], w2 [d, f]) as fp32 arrays holding bf16 values."""
+    logits = np.asarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    ids, gates = route_topk(logits, k)
+    counts = expert_counts(ids, E)
+    S, kappa = skew_kappa(counts)
+    b = block_counts(counts, beta)
+    boff = block_offsets(b)
+    pl = plan(b, P, s, variant_mask)
+    row_token, row_gate, tok_row = dispatch(ids, gates, boff, beta)
+    d = x.shape[1]
+    O = np.zeros((len(row_token), d), dtype=np.float32)
+    for e in range(E):
+        if counts[e] == 0:
+            continue
+        r0 = beta * boff[e]
+        rows = slice(r0, r0 + int(counts[e]))
+        w1, w2 = get_expert(e)
+        O[rows] = expert_ffn(x[row_token[rows]], w1, w2)
+    y = combine(O, tok_row, gates)
+    return {"ids": ids, "gates": gates, "counts": counts, "sumsq": S, "kappa": kappa,
+            "b": b, "block_off": boff, "plan": pl, "row_token": row_token,
+            "row_gate": row_gate, "tok_row": tok_row, "O": O, "y": y}
+
+
+def token_output(x_t: np.ndarray, experts, gates_t, get_expert) -> np.ndarray:
+    """y_t for one token from its chosen experts and gates (rows of the FFN are
+    independent, so any single token can be checked on its own at full size)."""
+    y = np.zeros(x_t.shape[-1], dtype=np.float32)
+    for e, g in zip(experts, gates_t):
+        w1, w2 = get_expert(int(e))
+        y += np.float32(g) * expert_ffn(x_t[None, :], w1, w2)[0]
+    return y
