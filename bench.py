@@ -1,0 +1,386 @@
+"""Benchmark of the skew-aware MoE forward layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole layer (route + histogram + kappa, block plan, dispatch,
+grouped SwiGLU FFN with the fused combine) over one batch of seeded synthetic inputs that
+are resident in HBM.  Prints one JSON line (rank 0).  `--impl reference` times the CPU
+oracle instead, on the host cores, on a bounded sample of the same workload.
+
+With N > 1 (torchrun) every rank runs an independent replica of the layer on its own GPU:
+the layer has no exchange step on one GPU, so there is no data-path collective; the
+process group only carries the barrier and the max over ranks of the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from skew_aware_token_b200 import native as N  # noqa: E402
+from skew_aware_token_b200 import synth  # noqa: E402
+
+METRIC = "MoE-layer fwd routed tokens/s and TFLOP/s on 1 B200; % of roofline vs kappa"
+DEFAULT_WORKLOAD = "olmoe_a1"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LAUNCHES_PER_STEP = 7  # route, kappa, plan, rank, gather, fc1, fc2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "of measured"
+    return dict(FALLBACK_PEAKS), "of fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as exc:  # NVML missing: report that instead of clocks
+            self.nv = None
+            self.error = repr(exc)
+
+    _REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self._REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.error}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if args.impl == "ours":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif args.impl == "ours":
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def workload_config(wl, extra=None):
+    cfg = {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "f": wl.f,
+           "beta": wl.beta, "P": wl.P, "s": wl.s, "alpha": wl.alpha, "hot_p": wl.hot_p,
+           "hot_mode": wl.hot_mode, "seed": wl.seed, "parallelism": "replicas"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def oracle_sample(wl, logits, x, get_expert, n_tokens):
+    """One oracle forward over the first n_tokens tokens of the workload."""
+    from oracle import moe_oracle as O
+    return O.moe_forward(logits[:n_tokens], x[:n_tokens], get_expert, k=wl.k, beta=wl.beta,
+                         P=wl.P, s=wl.s)
+
+
+def host_expert_getter(w1, w2):
+    """Expert weights for the oracle, copied to the host one expert at a time."""
+    cache = {}
+
+    def get(e):
+        if e not in cache:
+            if len(cache) > 64:
+                cache.clear()
+            cache[e] = (w1[e].float().cpu().numpy(), w2[e].float().cpu().numpy())
+        return cache[e]
+    return get
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def time_oracle(wl, logits_np, x_np, get_expert, budget_s):
+    """Times the oracle on a token sample sized to about budget_s seconds of CPU work."""
+    n = min(wl.T, 64)
+    t0 = time.perf_counter()
+    oracle_sample(wl, logits_np, x_np, get_expert, n)
+    per_tok = (time.perf_counter() - t0) / n
+    n = int(max(1, min(wl.T, budget_s / max(per_tok, 1e-9))))
+    t0 = time.perf_counter()
+    oracle_sample(wl, logits_np, x_np, get_expert, n)
+    dt = time.perf_counter() - t0
+    return n, dt
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, wl, world, rank, local):
+    from skew_aware_token_b200.layer import MoeLayer
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    logits_h = synth.make_logits(wl)
+    x_h = synth.make_x(wl)
+    w1, w2 = synth.make_weights(wl, dev)
+    logits = logits_h.to(dev)
+    x = x_h.to(dev)
+    layer = MoeLayer(wl, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(record=None):
+        if record is None:
+            layer(logits, x, w1, w2)
+            return
+        record[0].record(stream)
+        layer.route(logits)
+        record[1].record(stream)
+        layer.plan(0)
+        record[2].record(stream)
+        layer.dispatch(x)
+        record[3].record(stream)
+        layer.ffn(w1, w2)
+        record[4].record(stream)
+
+    layer.clear_status()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    status = layer.read_status()
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {N.moe_status_string(status)}")
+
+    # per-stage events on the launching stream over the whole timed region
+    recs = [[ev() for _ in range(5)] for _ in range(args.steps)]
+    start, stop = ev(), ev()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            step(recs[i])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    elapsed = start.elapsed_time(stop) / 1e3
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed = float(t.item())
+    stage_ms = {name: statistics.mean(r[i].elapsed_time(r[i + 1]) for r in recs)
+                for i, name in enumerate(["route", "plan", "dispatch", "ffn"])}
+    status = layer.read_status()
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {N.moe_status_string(status)}")
+
+    kappa = float(layer.kappa[0].item())
+    pi = layer.plan_info.cpu().tolist()
+    tokens = wl.T * wl.k * args.steps * world
+    value = tokens / elapsed
+    tflops = wl.flops * args.steps * world / elapsed / 1e12
+    ffn_s = stage_ms["ffn"] / 1e3
+    ffn_tflops = wl.flops / ffn_s / 1e12
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    weight_bytes = 6 * wl.d * wl.f * sum(1 for c in layer.view("counts").cpu().tolist() if c)
+    roofline = {"bound": "tensor", "kernel": "expert FFN (FC1+SwiGLU, FC2+combine)",
+                "achieved": round(ffn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(ffn_tflops / peak, 4), "peak_source": f"bf16 burst {peak_src}",
+                "traffic": None, "flops_per_launch": wl.flops,
+                "ms_per_launch": round(stage_ms["ffn"], 4),
+                "frac_of_sustained": round(ffn_tflops / peaks.get(
+                    "bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]), 4)}
+    traffic_path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(traffic_path):
+        with open(traffic_path) as fh:
+            tr = json.load(fh).get(wl.name)
+        if tr:
+            roofline["traffic"] = tr
+
+    # end to end through the public API: pinned host inputs in, y out, every step
+    logits_p = logits_h.pin_memory()
+    x_p = x_h.pin_memory()
+    y_p = torch.empty(wl.T, wl.d, dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 200))
+    for _ in range(2):
+        layer.forward_host(logits_p, x_p, w1, w2, y_p, logits, x)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        layer.forward_host(logits_p, x_p, w1, w2, y_p, logits, x)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_t = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        t = torch.tensor([e2e_t], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_t = float(t.item())
+    h2d = logits_h.numel() * 4 + x_h.numel() * 2
+    d2h = wl.T * wl.d * 4
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, dt = time_oracle(wl, logits_h.numpy(), x_h.float().numpy(),
+                            host_expert_getter(w1, w2), args.cpu_budget)
+        cpu = {"value": n * wl.k / dt, "unit": "tokens/s", "cores": cpu_cores(),
+               "kind": "oracle",
+               "sample": f"first {n} of {wl.T} tokens of {wl.name}, whole layer, one run "
+                         f"({dt:.1f} s, numpy fp32 + OpenBLAS)"}
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(elapsed / args.steps * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; router logits N(0,1) + Zipf bias, x N(0,1), "
+                "weights N(0, 1/sqrt(fan_in)), random-init)",
+        "config": workload_config(wl, {"kappa": kappa, "l2": "inputs larger than L2 "
+                                       f"(expert weights {weight_bytes / 1e9:.2f} GB > 126 MB)",
+                                       "B": pi[0], "tau": pi[1], "makespan": pi[2],
+                                       "fixed_makespan": pi[5], "variant": pi[3]}),
+        "tflops": round(tflops, 2), "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+        "roofline": roofline, "cpu_baseline": cpu,
+        "e2e": {"value": round(wl.T * wl.k * e2e_steps * world / e2e_t, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks.summary(),
+        "impl": "ours",
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return
+    logits_h = synth.make_logits(wl)
+    x_h = synth.make_x(wl)
+    # the oracle reads host weights; draw them on the host with the same recipe
+    cache = {}
+
+    def get_expert(e):
+        if e not in cache:
+            if len(cache) > 64:
+                cache.clear()
+            w1, w2 = synth.expert_weights(wl, e, "cpu")
+            cache[e] = (w1.float().numpy(), w2.float().numpy())
+        return cache[e]
+
+    logits_np, x_np = logits_h.numpy(), x_h.float().numpy()
+    total = args.warmup + args.steps
+    n, dt = time_oracle(wl, logits_np, x_np, get_expert, max(0.05, args.ref_budget / total))
+    for _ in range(args.warmup):
+        oracle_sample(wl, logits_np, x_np, get_expert, n)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample(wl, logits_np, x_np, get_expert, n)
+    elapsed = time.perf_counter() - t0
+    value = n * wl.k * args.steps / elapsed
+    sample = (f"first {n} of {wl.T} tokens of {wl.name} per step, whole layer "
+              f"(numpy fp32 + OpenBLAS)")
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(elapsed / args.steps * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded)", "config": workload_config(wl),
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "kind": "oracle",
+                         "cores": cpu_cores(), "sample": sample},
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of CPU work for the oracle baseline sample")
+    ap.add_argument("--ref-budget", type=float, default=120.0,
+                    help="seconds of CPU work for the whole reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    wl = synth.WORKLOADS[args.workload]
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, wl, world, rank)
+        else:
+            from skew_aware_token_b200 import build as B
+            if not os.path.exists(N.LIB_PATH):
+                B.build()
+            run_ours(args, wl, world, rank, local)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,196 @@
+/*
+ * moeskew.h - C ABI of the skew-aware MoE forward layer on one NVIDIA B200 (sm_100a).
+ *
+ * The layer follows the "MegaFlux" summary (picx.dev): routing skew kappa ("Routing Skew
+ * Problem"), tile-aligned token blocks and the replica-budgeted block planner
+ * (Methodology 1, "Problem Formulation" and "Bounded Greedy Search"), and the SwiGLU
+ * expert computation with the gate-weighted combine (Methodology 2, expert-computation
+ * equation).  On one GPU the P "GPUs" of the planner are P virtual execution slots.
+ *
+ * Conventions shared by every entry point
+ *   - Every array argument is a DEVICE pointer owned by the caller; the library never
+ *     allocates, frees or keeps a pointer after the call returns.  Arrays must be 16-byte
+ *     aligned.  bf16 data is passed as uint16_t bit patterns.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t / CUstream handle; NULL is
+ *     the legacy default stream) and never synchronises the host.  Inputs are const and
+ *     never modified.
+ *   - The return value is MOE_OK or a negative host-detected error; on error nothing has
+ *     been enqueued.  Problems only the device can see (an expert id out of range, more
+ *     rows than the blocks hold, a non-finite logit, a bounded wait that ran out) are
+ *     OR-ed into the caller's int32 `status` word in device memory as MOE_STATUS_* bits;
+ *     the caller clears it before and reads it after its own synchronisation.  When a bit
+ *     is set the outputs of that call are unspecified (but every write stayed inside the
+ *     caller's buffers).
+ *   - There is no mutable global state: calls on different streams with different
+ *     buffers may run concurrently.
+ *
+ * Sizes: N = T*k routed rows; b_e = ceil(c_e/beta) blocks of expert e; B = sum_e b_e;
+ * B_max = floor((N + min(E,N)*(beta-1)) / beta) bounds B for every routing; R_max =
+ * beta*B_max bounds the padded rows.  moe_workspace_size() returns both.
+ */
+#ifndef MOESKEW_H
+#define MOESKEW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* moe_stream_t;   /* == cudaStream_t */
+
+/* Layer configuration, validated by every call.
+ *   T tokens; d model width; E experts (1..256); k experts per token (1..min(E,8));
+ *   f expert FFN width (FC1 has 2f outputs: f gate columns G then f up columns U);
+ *   beta rows per token block (64 or 128); P virtual slots (1..8); s replica budget
+ *   per slot (>= 0).  N = T*k must not exceed 2^22.
+ *   The FFN needs d % 256 == 0 and f % 128 == 0; dispatch and combine need d % 8 == 0. */
+typedef struct moe_cfg {
+  int32_t T, d, E, k, f, beta, P, s;
+} moe_cfg;
+
+/* host-detected errors (return values) */
+enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1, /* NULL pointer, k > E, k > 8, beta not 64/128, P > 8, ... */
+  MOE_ERR_UNSUPPORTED = -2, /* shape outside what the kernels take, misaligned pointer */
+  MOE_ERR_CUDA = -3         /* a launch or a CUDA call failed */
+};
+
+/* device-detected problems (bits OR-ed into *status) */
+enum {
+  MOE_STATUS_BAD_ID = 1,     /* an expert id outside [0, E) */
+  MOE_STATUS_OVERFLOW = 2,   /* an expert has more rows than its blocks hold */
+  MOE_STATUS_NONFINITE = 4,  /* a router logit is NaN or infinite */
+  MOE_STATUS_TIMEOUT = 8,    /* a bounded wait inside a kernel ran out */
+  MOE_STATUS_PLAN = 16       /* the block plan does not fit B_max (inconsistent counts) */
+};
+
+/* moe_workspace_size(which) */
+enum { MOE_WS_ROWS = 0, MOE_WS_BLOCKS = 1 };
+
+/* plan_info layout (int32[MOE_PI_LEN]) written by moe_plan_blocks */
+enum {
+  MOE_PI_B = 0,              /* B = sum_e b_e */
+  MOE_PI_TAU = 1,            /* tau = ceil(B / P) */
+  MOE_PI_MAKESPAN = 2,       /* max_r l_r of the chosen plan */
+  MOE_PI_VARIANT = 3,        /* chosen greedy variant (0..3) */
+  MOE_PI_NTILES = 4,         /* number of 128-row execution tiles */
+  MOE_PI_FIXED_MAKESPAN = 5, /* max_r l_r of the no-replica (fixed placement) plan */
+  MOE_PI_REPLICAS = 6,       /* total replicas of the chosen plan */
+  MOE_PI_ROUNDS = 7,         /* greedy rounds of the chosen plan */
+  MOE_PI_SLOT_TILE_OFF = 8,  /* P+1 entries: first tile of each slot */
+  MOE_PI_VAR_MAKESPAN = 17,  /* 4 entries: makespan per variant, -1 when disabled */
+  MOE_PI_VAR_REPLICAS = 21,  /* 4 entries */
+  MOE_PI_VAR_ROUNDS = 25,    /* 4 entries */
+  MOE_PI_LEN = 32
+};
+
+/* moe_expert_ffn modes */
+enum {
+  MOE_FFN_FUSED_COMBINE = 0, /* out = y fp32 [T, d]; the call zeroes y, then FC2's
+                                epilogue adds row_gate * O into y[row_token] */
+  MOE_FFN_WRITE_O = 1,       /* out = O bf16 [R_max, d]; moe_combine reduces it */
+  MOE_FFN_STRICT_SLOTS = 2   /* flag: CTA c only runs slot (c mod P)'s tiles, so the
+                                layer time follows the plan's makespan (one GPU standing
+                                in for P); without it every CTA takes tiles of any slot */
+};
+
+/* Upper bounds: which = MOE_WS_ROWS -> R_max rows (Xp, A, O, row_token, row_gate);
+ * MOE_WS_BLOCKS -> B_max entries (blocks, tiles).  Returns 0 for an invalid cfg. */
+MOE_API size_t moe_workspace_size(const moe_cfg* cfg, int which);
+
+/* Router top-k, expert histogram and skew ("Routing Skew Problem"; router outputs of the
+ * expert-computation equation).
+ *   logits     fp32 [T, E] row-major, read only.
+ *   topk_ids   int32 [T, k]: the k largest logits of each row, descending, ties to the
+ *              lower expert id.
+ *   topk_gates fp32 [T, k]: softmax over the k chosen logits (= the full softmax
+ *              renormalised over the top-k).
+ *   counts     int32 [E]: c_e = #{(t, j) : topk_ids[t, j] = e}.
+ *   sumsq      int64 [1]: S = sum_e c_e^2.
+ *   kappa      fp64 [1]: E * S / N^2 (one rounding, exact integers); 0 when N = 0.
+ * A non-finite logit sets MOE_STATUS_NONFINITE. */
+MOE_API int moe_route_hist(const moe_cfg* cfg, const float* logits, int32_t* topk_ids,
+                   float* topk_gates, int32_t* counts, int64_t* sumsq, double* kappa,
+                   int32_t* status, moe_stream_t stream);
+
+/* Token blocks and the block planner ("Problem Formulation", "Bounded Greedy Search").
+ *   counts       int32 [E] (from moe_route_hist).
+ *   variant_mask bits 0..3 enable greedy variants v = 2*D + F (D donor priority:
+ *                0 total overload, 1 largest home-expert load; F fan-out: 0 one new copy
+ *                per expert per round, 1 several); 0 means all four.
+ *   block_off    int32 [E+1]: exclusive prefix sum of b_e = ceil(c_e / beta).
+ *   q            int32 [E, P] row-major: blocks of expert e run by slot r, of the best
+ *                enabled variant (least makespan, then fewest replicas, then lowest v).
+ *   slot_load    int32 [P]: l_r = sum_e q[e, r].
+ *   slot_off     int32 [P+1]: exclusive prefix sum of slot_load.
+ *   blocks       int32 [B_max, 2]: (e, j) pairs; slot r's run is
+ *                [slot_off[r], slot_off[r+1]), experts ascending, expert e's share being
+ *                block indices j in [sum_{r'<r} q[e, r'], + q[e, r]).
+ *   tiles        int32 [B_max, 4]: 128-row execution tiles (e, first padded row, rows in
+ *                the tile (64 or 128), slot) in the same slot/expert order; with beta = 64
+ *                two consecutive blocks of one expert's run share a tile.
+ *   plan_info    int32 [MOE_PI_LEN]: see MOE_PI_*.
+ * The owner of expert e is slot h(e) = floor(e * P / E).  The plan is deterministic and
+ * bit-identical across calls.  Runs on one CTA. */
+MOE_API int moe_plan_blocks(const moe_cfg* cfg, const int32_t* counts, uint32_t variant_mask,
+                    int32_t* block_off, int32_t* q, int32_t* slot_load, int32_t* slot_off,
+                    int32_t* blocks, int32_t* tiles, int32_t* plan_info, int32_t* status,
+                    moe_stream_t stream);
+
+/* Tile-aligned dispatch: a stable counting sort of the (t, j) pairs by expert.
+ *   x          bf16 [T, d]; topk_ids, topk_gates [T, k]; block_off [E+1].
+ *   xp         bf16 [R_max, d]: row beta*block_off[e] + i holds x[t] of expert e's i-th
+ *              pair in token order; padding rows of each expert's blocks are zero; rows at
+ *              or beyond beta*B are not written.
+ *   row_token  int32 [R_max]: t on valid rows, -1 on padding rows.
+ *   row_gate   fp32 [R_max]: topk_gates[t, j] on valid rows, 0 on padding rows.
+ *   tok_row    int32 [T, k]: the padded row of pair (t, j).
+ * Ids outside [0, E) set MOE_STATUS_BAD_ID; rows beyond an expert's blocks set
+ * MOE_STATUS_OVERFLOW and are dropped. */
+MOE_API int moe_dispatch_permute(const moe_cfg* cfg, const uint16_t* x, const int32_t* topk_ids,
+                         const float* topk_gates, const int32_t* block_off, uint16_t* xp,
+                         int32_t* row_token, float* row_gate, int32_t* tok_row,
+                         int32_t* status, moe_stream_t stream);
+
+/* Grouped SwiGLU expert FFN over the planner's tiles (expert-computation equation):
+ * for each tile of expert e, Z = Xp[rows] W1_e^T (fp32 accumulate on the tensor cores),
+ * A = SiLU(G) * U rounded to bf16 into a_scratch, then O = A W2_e^T.
+ *   w1         bf16 [E, 2f, d] (rows 0..f-1 = G, f..2f-1 = U; K-major).
+ *   w2         bf16 [E, d, f] (K-major).
+ *   tiles, plan_info from moe_plan_blocks; row_token, row_gate from moe_dispatch_permute.
+ *   a_scratch  bf16 [R_max, f], caller-owned scratch.
+ *   out        MOE_FFN_FUSED_COMBINE: y fp32 [T, d], zeroed by the call, then
+ *              y[row_token[r]] += row_gate[r] * O[r] for every valid row (fp32 atomic
+ *              adds: the summation order, and so the last bits, may vary run to run).
+ *              MOE_FFN_WRITE_O: O bf16 [R_max, d] (rows of the plan's tiles).
+ *   mode       MOE_FFN_FUSED_COMBINE or MOE_FFN_WRITE_O, optionally | MOE_FFN_STRICT_SLOTS.
+ * Two persistent kernels (FC1+SwiGLU, then FC2) of one CTA per SM; every wait inside them
+ * is bounded and sets MOE_STATUS_TIMEOUT instead of hanging. */
+MOE_API int moe_expert_ffn(const moe_cfg* cfg, const uint16_t* xp, const uint16_t* w1,
+                   const uint16_t* w2, const int32_t* tiles, const int32_t* plan_info,
+                   const int32_t* row_token, const float* row_gate, int mode,
+                   uint16_t* a_scratch, void* out, int32_t* status, moe_stream_t stream);
+
+/* Deterministic gate-weighted combine (expert-computation equation):
+ * y[t] = sum_{j=0..k-1} topk_gates[t, j] * O[tok_row[t, j]], in that order, fp32.
+ *   o bf16 [R_max, d]; tok_row, topk_gates [T, k]; y fp32 [T, d] (overwritten). */
+MOE_API int moe_combine(const moe_cfg* cfg, const uint16_t* o, const int32_t* tok_row,
+                const float* topk_gates, float* y, int32_t* status, moe_stream_t stream);
+
+/* Static text for a return code (negative) or a status bit mask (positive). */
+MOE_API const char* moe_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOESKEW_H */

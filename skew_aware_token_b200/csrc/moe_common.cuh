@@ -1,0 +1,50 @@
+// Shared definitions of the moeskew CUDA library (sm_100a).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "moeskew.h"
+
+namespace moe {
+
+constexpr int kMaxE = 256;
+constexpr int kMaxK = 8;
+constexpr int kMaxP = 8;
+constexpr long long kMaxN = 1LL << 22;
+
+// Bound on the number of token blocks over every routing of N rows into E experts:
+// sum_e ceil(c_e / beta) <= (N + min(E, N) * (beta - 1)) / beta.
+inline long long max_blocks(const moe_cfg& c) {
+  const long long N = (long long)c.T * c.k;
+  const long long nz = N < c.E ? N : c.E;
+  return (N + nz * (c.beta - 1)) / c.beta;
+}
+inline long long max_rows(const moe_cfg& c) { return max_blocks(c) * c.beta; }
+
+__device__ __forceinline__ void set_status(int32_t* status, int bits) {
+  atomicOr(status, bits);
+}
+
+// ---- launchers (one per kernel family), called by the C ABI after validation ----
+cudaError_t launch_route_hist(const moe_cfg& c, const float* logits, int32_t* ids,
+                              float* gates, int32_t* counts, int64_t* sumsq, double* kappa,
+                              int32_t* status, cudaStream_t st);
+cudaError_t launch_plan(const moe_cfg& c, const int32_t* counts, uint32_t mask,
+                        int32_t* block_off, int32_t* q, int32_t* slot_load,
+                        int32_t* slot_off, int32_t* blocks, int32_t* tiles,
+                        int32_t* plan_info, int32_t* status, cudaStream_t st);
+cudaError_t launch_dispatch(const moe_cfg& c, const uint16_t* x, const int32_t* ids,
+                            const float* gates, const int32_t* block_off, uint16_t* xp,
+                            int32_t* row_token, float* row_gate, int32_t* tok_row,
+                            int32_t* status, cudaStream_t st);
+cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
+                       const uint16_t* w2, const int32_t* tiles, const int32_t* plan_info,
+                       const int32_t* row_token, const float* row_gate, int mode,
+                       uint16_t* a_scratch, void* out, int32_t* status, cudaStream_t st);
+cudaError_t launch_combine(const moe_cfg& c, const uint16_t* o, const int32_t* tok_row,
+                           const float* gates, float* y, int32_t* status, cudaStream_t st);
+
+int num_sms();
+
+}  // namespace moe

@@ -1,0 +1,372 @@
+// Token blocks and the replica-budgeted block planner, on one CTA.
+//
+// "MegaFlux" summary, Methodology 1: "Problem Formulation" (b_e = ceil(c_e / beta); find
+// q in Z^{E x P} minimising max_r sum_e q_er with sum_r q_er = b_e and at most s remote
+// experts per slot) and "Bounded Greedy Search" (four searches from the no-replica
+// assignment toward tau = ceil(B / P): donor priority x fan-out).  The receiver of a move
+// is the slot with the most slack, as in the quota solver of the UltraEP notes
+// (section 4, Algorithm 1); that solver is also a one-SM kernel with its load matrix in
+// shared memory.  Plans are deterministic (TopoEP: bitwise-identical plans).
+//
+// The greedy rule (shared word for word with the CPU statement of the method):
+//   start  q[e][h(e)] = b_e, h(e) = floor(e P / E); loads l_r; replicas rep_r = 0.
+//   round  while max_r l_r > tau: donors = {r : l_r > tau} ordered by (key desc, r asc)
+//          with key = l_r (variant D = 0) or max_{h(e)=r} q[e][r] (D = 1), taken at the
+//          start of the round; a donor's home experts in order (q[e][r] desc, e asc);
+//          while the donor is above tau and the expert still has home blocks:
+//            receivers t != r with l_t < tau and (q[e][t] > 0 or (rep_t < s and
+//            (F = 1 or no copy of e was opened this round)));
+//            t = the receiver of least (l_t, t); move min(l_r - tau, tau - l_t, q[e][r]).
+//          A round that moves nothing ends the search.
+//   best   least (makespan, total replicas, variant index) among enabled variants.
+//
+// One warp runs one variant: slot-parallel work (candidate test, arg-min, maxima) uses
+// lanes 0..P-1 and warp shuffles; expert-parallel work strides the lanes over experts.
+// Lane 0 applies each move; __syncwarp() orders it against the next read.
+#include <climits>
+
+#include "moe_common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kPlanThreads = 128;  // 4 warps = 4 greedy variants
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ int home_lo(int r, int E, int P) { return (r * E + P - 1) / P; }
+
+__device__ __forceinline__ int warp_max(int v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = max(v, __shfl_xor_sync(kFull, v, off));
+  return v;
+}
+__device__ __forceinline__ int warp_min(int v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = min(v, __shfl_xor_sync(kFull, v, off));
+  return v;
+}
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+  return v;
+}
+// exclusive prefix sum over lanes
+__device__ __forceinline__ int warp_excl_scan(int v, int lane) {
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(kFull, incl, off);
+    if (lane >= off) incl += y;
+  }
+  return incl - v;
+}
+
+struct VariantState {
+  int* q;      // [E * P]
+  int* load;   // [P]
+  int* rep;    // [P]
+  int* newc;   // [E]
+  int* order;  // [E]
+  int* donors; // [P]
+};
+
+// Runs greedy variant v on the calling warp; returns (makespan, replicas, rounds) in lane 0.
+__device__ void greedy_variant(int v, int E, int P, int s, int tau, const int* b,
+                               VariantState st, int* out_makespan, int* out_replicas,
+                               int* out_rounds) {
+  const int lane = threadIdx.x & 31;
+  const int D = v >> 1, F = v & 1;
+  int* q = st.q;
+  int* load = st.load;
+  int* rep = st.rep;
+
+  for (int i = lane; i < E * P; i += 32) q[i] = 0;
+  __syncwarp();
+  for (int e = lane; e < E; e += 32) q[e * P + e * P / E] = b[e];
+  if (lane < P) {
+    int sum = 0;
+    for (int e = home_lo(lane, E, P); e < home_lo(lane + 1, E, P); ++e) sum += b[e];
+    load[lane] = sum;
+    rep[lane] = 0;
+  }
+  __syncwarp();
+
+  int rounds = 0;
+  while (true) {
+    const int maxload = warp_max(lane < P ? load[lane] : INT_MIN);
+    if (maxload <= tau) break;
+    ++rounds;
+    for (int e = lane; e < E; e += 32) st.newc[e] = 0;
+
+    // donor order, keys taken at the start of the round
+    const bool is_donor = lane < P && load[lane] > tau;
+    int key = 0;
+    if (lane < P) {
+      if (D == 0) {
+        key = load[lane];
+      } else {
+        for (int e = home_lo(lane, E, P); e < home_lo(lane + 1, E, P); ++e)
+          key = max(key, q[e * P + lane]);
+      }
+    }
+    const unsigned dmask = __ballot_sync(kFull, is_donor);
+    const int ndon = __popc(dmask);
+    int rank = 0;
+    for (int r2 = 0; r2 < P; ++r2) {
+      const int k2 = __shfl_sync(kFull, key, r2);
+      if (is_donor && (dmask >> r2 & 1u) && (k2 > key || (k2 == key && r2 < lane))) ++rank;
+    }
+    if (is_donor) st.donors[rank] = lane;
+    __syncwarp();
+
+    bool progress = false;
+    for (int di = 0; di < ndon; ++di) {
+      const int r = st.donors[di];
+      const int lo = home_lo(r, E, P), n = home_lo(r + 1, E, P) - lo;
+      // home experts by (q[e][r] desc, e asc)
+      for (int i = lane; i < n; i += 32) {
+        const int e = lo + i, qe = q[e * P + r];
+        int rk = 0;
+        for (int i2 = 0; i2 < n; ++i2) {
+          const int q2 = q[(lo + i2) * P + r];
+          rk += (q2 > qe) || (q2 == qe && i2 < i);
+        }
+        st.order[rk] = e;
+      }
+      __syncwarp();
+      for (int oi = 0; oi < n; ++oi) {
+        const int e = st.order[oi];
+        while (true) {
+          const int lr = load[r], qer = q[e * P + r];
+          if (!(lr > tau && qer > 0)) break;
+          int ck = INT_MAX;
+          if (lane < P && lane != r) {
+            const int lt = load[lane];
+            if (lt < tau && (q[e * P + lane] > 0 || (rep[lane] < s && (F || st.newc[e] == 0))))
+              ck = (lt << 4) | lane;
+          }
+          ck = warp_min(ck);
+          if (ck == INT_MAX) break;
+          const int t = ck & 15, lt = ck >> 4;
+          const int delta = min(min(lr - tau, tau - lt), qer);
+          __syncwarp();
+          if (lane == 0) {
+            if (q[e * P + t] == 0) {
+              rep[t] += 1;
+              st.newc[e] += 1;
+            }
+            q[e * P + r] -= delta;
+            q[e * P + t] += delta;
+            load[r] -= delta;
+            load[t] += delta;
+          }
+          __syncwarp();
+          progress = true;
+        }
+      }
+      __syncwarp();
+    }
+    if (!progress) break;
+  }
+  const int mk = warp_max(lane < P ? load[lane] : 0);
+  const int reps = warp_sum(lane < P ? rep[lane] : 0);
+  if (lane == 0) {
+    *out_makespan = mk;
+    *out_replicas = reps;
+    *out_rounds = rounds;
+  }
+}
+
+__global__ void __launch_bounds__(kPlanThreads, 1)
+plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
+            unsigned mask, int b_max, int32_t* __restrict__ block_off, int32_t* __restrict__ q_out,
+            int32_t* __restrict__ slot_load, int32_t* __restrict__ slot_off,
+            int32_t* __restrict__ blocks, int32_t* __restrict__ tiles,
+            int32_t* __restrict__ plan_info, int32_t* __restrict__ status) {
+  extern __shared__ int sm[];
+  int* b = sm;                          // E
+  int* boff = b + E;                    // E + 1
+  int* qv = boff + E + 1;               // 4 * E * P
+  int* loadv = qv + 4 * E * P;          // 4 * 8
+  int* repv = loadv + 4 * kMaxP;        // 4 * 8
+  int* newc = repv + 4 * kMaxP;         // 4 * E
+  int* order = newc + 4 * E;            // 4 * E
+  int* donors = order + 4 * E;          // 4 * 8
+  int* res = donors + 4 * kMaxP;        // 12: makespan[4], replicas[4], rounds[4]
+  int* misc = res + 12;                 // [0] B, [1] tau, [2] best, [3..3+P] slot tile offsets
+                                        // [12..12+P] slot_off, [24..] fixed loads (P)
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // ---- b_e and the exclusive scan block_off (warp 0; lane owns a chunk of experts)
+  if (warp == 0) {
+    const int C = (E + 31) / 32;
+    const int e0 = min(lane * C, E), e1 = min(e0 + C, E);
+    int local = 0;
+    for (int e = e0; e < e1; ++e) {
+      const int c = max(counts[e], 0);
+      const int be = (c + beta - 1) / beta;
+      b[e] = be;
+      local += be;
+    }
+    int run = warp_excl_scan(local, lane);
+    for (int e = e0; e < e1; ++e) {
+      boff[e] = run;
+      block_off[e] = run;
+      run += b[e];
+    }
+    const int B = __shfl_sync(kFull, run, 31);
+    if (lane == 31) {
+      boff[E] = B;
+      block_off[E] = B;
+      misc[0] = B;
+      misc[1] = (B + P - 1) / P;
+    }
+  }
+  __syncthreads();
+  const int B = misc[0], tau = misc[1];
+
+  // ---- four greedy variants, one per warp
+  {
+    VariantState st;
+    st.q = qv + warp * E * P;
+    st.load = loadv + warp * kMaxP;
+    st.rep = repv + warp * kMaxP;
+    st.newc = newc + warp * E;
+    st.order = order + warp * E;
+    st.donors = donors + warp * kMaxP;
+    if (mask >> warp & 1u) {
+      greedy_variant(warp, E, P, s, tau, b, st, &res[warp], &res[4 + warp], &res[8 + warp]);
+    } else if (lane == 0) {
+      res[warp] = INT_MAX;
+      res[4 + warp] = INT_MAX;
+      res[8 + warp] = 0;
+    }
+  }
+  __syncthreads();
+
+  // ---- best variant: least (makespan, replicas, v)
+  if (tid == 0) {
+    int best = -1;
+    for (int v = 0; v < 4; ++v) {
+      if (!(mask >> v & 1u)) continue;
+      if (best < 0 || res[v] < res[best] || (res[v] == res[best] && res[4 + v] < res[4 + best]))
+        best = v;
+    }
+    misc[2] = best;
+  }
+  __syncthreads();
+  const int best = misc[2];
+  const int* qb = qv + best * E * P;
+  const int* lb = loadv + best * kMaxP;
+
+  for (int i = tid; i < E * P; i += blockDim.x) q_out[i] = qb[i];
+
+  // ---- per-slot tile counts, slot offsets (thread 0; P <= 8)
+  if (tid < P) {
+    const int r = tid;
+    int nt = 0;
+    for (int e = 0; e < E; ++e) {
+      const int qer = qb[e * P + r];
+      nt += beta == 128 ? qer : (qer + 1) / 2;
+    }
+    misc[3 + r] = nt;  // temporarily the count
+    int fixed = 0;
+    for (int e = home_lo(r, E, P); e < home_lo(r + 1, E, P); ++e) fixed += b[e];
+    misc[24 + r] = fixed;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0, tacc = 0, fixed_max = 0;
+    for (int r = 0; r < P; ++r) {
+      slot_load[r] = lb[r];
+      slot_off[r] = acc;
+      misc[12 + r] = acc;
+      acc += lb[r];
+      const int nt = misc[3 + r];
+      misc[3 + r] = tacc;
+      tacc += nt;
+      fixed_max = max(fixed_max, misc[24 + r]);
+    }
+    slot_off[P] = acc;
+    misc[12 + P] = acc;
+    misc[3 + P] = tacc;
+    if (B > b_max) set_status(status, MOE_STATUS_PLAN);
+    plan_info[MOE_PI_B] = B;
+    plan_info[MOE_PI_TAU] = tau;
+    plan_info[MOE_PI_MAKESPAN] = res[best];
+    plan_info[MOE_PI_VARIANT] = best;
+    plan_info[MOE_PI_NTILES] = min(tacc, b_max);
+    plan_info[MOE_PI_FIXED_MAKESPAN] = fixed_max;
+    plan_info[MOE_PI_REPLICAS] = res[4 + best];
+    plan_info[MOE_PI_ROUNDS] = res[8 + best];
+    for (int r = 0; r <= kMaxP; ++r)
+      plan_info[MOE_PI_SLOT_TILE_OFF + r] = r <= P ? min(misc[3 + r], b_max) : min(tacc, b_max);
+    for (int v = 0; v < 4; ++v) {
+      const bool on = mask >> v & 1u;
+      plan_info[MOE_PI_VAR_MAKESPAN + v] = on ? res[v] : -1;
+      plan_info[MOE_PI_VAR_REPLICAS + v] = on ? res[4 + v] : -1;
+      plan_info[MOE_PI_VAR_ROUNDS + v] = on ? res[8 + v] : -1;
+    }
+    for (int i = MOE_PI_VAR_ROUNDS + 4; i < MOE_PI_LEN; ++i) plan_info[i] = 0;
+  }
+  __syncthreads();
+
+  // ---- block list and tile list: warp w expands slots w, w+4
+  for (int r = warp; r < P; r += 4) {
+    const int C = (E + 31) / 32;
+    const int e0 = min(lane * C, E), e1 = min(e0 + C, E);
+    int nb = 0, nt = 0;
+    for (int e = e0; e < e1; ++e) {
+      const int qer = qb[e * P + r];
+      nb += qer;
+      nt += beta == 128 ? qer : (qer + 1) / 2;
+    }
+    int pb = misc[12 + r] + warp_excl_scan(nb, lane);
+    int pt = misc[3 + r] + warp_excl_scan(nt, lane);
+    for (int e = e0; e < e1; ++e) {
+      const int qer = qb[e * P + r];
+      int j0 = 0;
+      for (int r2 = 0; r2 < r; ++r2) j0 += qb[e * P + r2];
+      for (int i = 0; i < qer; ++i, ++pb) {
+        if (pb < b_max) {
+          blocks[2 * pb] = e;
+          blocks[2 * pb + 1] = j0 + i;
+        }
+      }
+      const int per = beta == 128 ? 1 : 2;
+      for (int i = 0; i < qer; i += per, ++pt) {
+        if (pt < b_max) {
+          tiles[4 * pt + 0] = e;
+          tiles[4 * pt + 1] = beta * (boff[e] + j0 + i);
+          tiles[4 * pt + 2] = (i + per <= qer) ? 128 : beta;
+          tiles[4 * pt + 3] = r;
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_plan(const moe_cfg& c, const int32_t* counts, uint32_t mask,
+                        int32_t* block_off, int32_t* q, int32_t* slot_load,
+                        int32_t* slot_off, int32_t* blocks, int32_t* tiles,
+                        int32_t* plan_info, int32_t* status, cudaStream_t st) {
+  const int E = c.E, P = c.P;
+  const size_t words = (size_t)E + (E + 1) + 4 * E * P + 4 * kMaxP + 4 * kMaxP + 4 * E +
+                       4 * E + 4 * kMaxP + 12 + 40;
+  const size_t bytes = words * sizeof(int);
+  if (bytes > 48 * 1024) {
+    cudaError_t err = cudaFuncSetAttribute(plan_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)bytes);
+    if (err != cudaSuccess) return err;
+  }
+  const unsigned m = (mask & 0xFu) ? (mask & 0xFu) : 0xFu;
+  plan_kernel<<<1, kPlanThreads, bytes, st>>>(counts, E, P, c.s, c.beta, m,
+                                              (int)max_blocks(c), block_off, q, slot_load,
+                                              slot_off, blocks, tiles, plan_info, status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

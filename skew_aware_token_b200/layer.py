@@ -1,0 +1,128 @@
+"""The forward MoE layer as one call: owns the device buffers of one configuration and
+strings the five C-ABI calls together on the current CUDA stream.
+
+    layer = MoeLayer(workload, device="cuda")
+    y = layer(logits, x, w1, w2)          # device tensors in, y fp32 [T, d] out
+    y_host = layer.forward_host(...)      # pinned host tensors in and out (end to end)
+"""
+from __future__ import annotations
+
+import torch
+
+from . import native as N
+
+
+class MoeLayer:
+    def __init__(self, wl, device="cuda", write_o: bool = False, guard: int = 0):
+        """`guard` adds that many spare elements after every buffer (canary checks)."""
+        self.cfg = N.MoeCfg.of(wl)
+        self.wl = wl
+        dev = torch.device(device)
+        T, d, E, k, f, P = wl.T, wl.d, wl.E, wl.k, wl.f, wl.P
+        R = N.moe_workspace_size(self.cfg, N.MOE_WS_ROWS)
+        Bm = N.moe_workspace_size(self.cfg, N.MOE_WS_BLOCKS)
+        if R == 0 and T > 0:
+            raise ValueError("configuration rejected by moe_workspace_size")
+        self.R_max, self.B_max = R, Bm
+        i32, f32 = torch.int32, torch.float32
+        z = lambda n, dt=i32: torch.zeros(n + guard, dtype=dt, device=dev)
+        # at least one 16-byte granule per buffer so every pointer is valid and aligned
+        self.topk_ids = z(max(T * k, 4))
+        self.topk_gates = z(max(T * k, 4), dt=f32)
+        self.counts = z(max(E, 4))
+        self.sumsq = z(2, dt=torch.int64)
+        self.kappa = z(2, dt=torch.float64)
+        self.status = z(4)
+        self.block_off = z(E + 4)
+        self.q = z(max(E * P, 4))
+        self.slot_load = z(8)
+        self.slot_off = z(12)
+        self.blocks = z(max(2 * Bm, 4))
+        self.tiles = z(max(4 * Bm, 4))
+        self.plan_info = z(N.PI["LEN"])
+        self.xp = z(max(R * d, 8), dt=torch.bfloat16)
+        self.row_token = z(max(R, 4))
+        self.row_gate = z(max(R, 4), dt=f32)
+        self.tok_row = z(max(T * k, 4))
+        self.a_scratch = z(max(R * f, 8), dt=torch.bfloat16)
+        self.y = z(max(T * d, 4), dt=f32)
+        self.o = z(max(R * d, 8), dt=torch.bfloat16) if write_o else None
+        self.device = dev
+
+    # ------------------------------------------------------------------ stages
+    def route(self, logits, stream=None):
+        N.moe_route_hist(self.cfg, logits, self.topk_ids, self.topk_gates, self.counts,
+                         self.sumsq, self.kappa, self.status, stream)
+
+    def plan(self, variant_mask=0, stream=None):
+        N.moe_plan_blocks(self.cfg, self.counts, variant_mask, self.block_off, self.q,
+                          self.slot_load, self.slot_off, self.blocks, self.tiles,
+                          self.plan_info, self.status, stream)
+
+    def dispatch(self, x, stream=None):
+        N.moe_dispatch_permute(self.cfg, x, self.topk_ids, self.topk_gates, self.block_off,
+                               self.xp, self.row_token, self.row_gate, self.tok_row,
+                               self.status, stream)
+
+    def ffn(self, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, stream=None):
+        out = self.o if mode & N.MOE_FFN_WRITE_O else self.y
+        if out is None:
+            raise ValueError("layer built without an O buffer (write_o=False)")
+        N.moe_expert_ffn(self.cfg, self.xp, w1, w2, self.tiles, self.plan_info,
+                         self.row_token, self.row_gate, mode, self.a_scratch, out,
+                         self.status, stream)
+
+    def combine(self, stream=None):
+        N.moe_combine(self.cfg, self.o, self.tok_row, self.topk_gates, self.y, self.status,
+                      stream)
+
+    # ------------------------------------------------------------------ whole layer
+    def __call__(self, logits, x, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, variant_mask=0,
+                 stream=None):
+        """Route, plan, dispatch, FFN (+ combine): returns y fp32 [T, d] (a view of the
+        layer's buffer, valid until the next call)."""
+        self.route(logits, stream)
+        self.plan(variant_mask, stream)
+        self.dispatch(x, stream)
+        self.ffn(w1, w2, mode, stream)
+        if mode & N.MOE_FFN_WRITE_O:
+            self.combine(stream)
+        return self.y[: self.wl.T * self.wl.d].view(self.wl.T, self.wl.d)
+
+    def forward_host(self, logits_h, x_h, w1, w2, y_h, logits_d, x_d, mode=0, stream=None):
+        """End to end from pinned host buffers: copies logits and x in, runs the layer,
+        copies y out (all asynchronous on the current stream)."""
+        logits_d.copy_(logits_h, non_blocking=True)
+        x_d.copy_(x_h, non_blocking=True)
+        y = self(logits_d, x_d, w1, w2, mode=mode, stream=stream)
+        y_h.copy_(y, non_blocking=True)
+        return y_h
+
+    def clear_status(self):
+        self.status.zero_()
+
+    def read_status(self) -> int:
+        return int(self.status[0].item())
+
+    def view(self, name):
+        """Typed views of the layer's buffers (for tests and reports)."""
+        wl = self.wl
+        T, d, E, k, P = wl.T, wl.d, wl.E, wl.k, wl.P
+        R, Bm = self.R_max, self.B_max
+        shapes = {
+            "topk_ids": (self.topk_ids, (T, k)), "topk_gates": (self.topk_gates, (T, k)),
+            "counts": (self.counts, (E,)), "block_off": (self.block_off, (E + 1,)),
+            "q": (self.q, (E, P)), "slot_load": (self.slot_load, (P,)),
+            "slot_off": (self.slot_off, (P + 1,)), "blocks": (self.blocks, (Bm, 2)),
+            "tiles": (self.tiles, (Bm, 4)), "xp": (self.xp, (R, d)),
+            "row_token": (self.row_token, (R,)), "row_gate": (self.row_gate, (R,)),
+            "tok_row": (self.tok_row, (T, k)), "a_scratch": (self.a_scratch, (R, wl.f)),
+            "y": (self.y, (T, d)),
+        }
+        if self.o is not None:
+            shapes["o"] = (self.o, (R, d))
+        buf, shape = shapes[name]
+        n = 1
+        for s in shape:
+            n *= s
+        return buf[:n].view(*shape)

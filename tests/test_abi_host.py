@@ -1,0 +1,102 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point the header
+declares, sizes its workspaces by the stated bounds, and rejects bad arguments before
+launching anything.  No GPU: the argument checks run before any CUDA call."""
+import ctypes
+import subprocess
+
+import pytest
+import torch
+
+from skew_aware_token_b200 import build as B
+from skew_aware_token_b200 import native as N
+from skew_aware_token_b200.synth import WORKLOADS
+
+NO_GPU = not torch.cuda.is_available()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    B.build()
+    return N.lib()
+
+
+def test_exports_every_declared_symbol():
+    declared = N.declared_symbols()
+    assert set(declared) == {"moe_workspace_size", "moe_route_hist", "moe_plan_blocks",
+                             "moe_dispatch_permute", "moe_expert_ffn", "moe_combine",
+                             "moe_status_string"}
+    out = subprocess.run(["nm", "-D", "--defined-only", N.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in declared:
+        assert name in exported, name
+        assert hasattr(N.lib(), name)
+    # nothing but the declared API is exported
+    assert {s for s in exported if s.startswith("moe_")} == set(declared)
+
+
+def test_workspace_sizes_follow_the_block_bound():
+    for wl in WORKLOADS.values():
+        Nr = wl.T * wl.k
+        b_max = (Nr + min(wl.E, Nr) * (wl.beta - 1)) // wl.beta
+        assert N.moe_workspace_size(wl, N.MOE_WS_BLOCKS) == b_max
+        assert N.moe_workspace_size(wl, N.MOE_WS_ROWS) == b_max * wl.beta
+        # the bound holds for the worst routing: every expert one row past a block
+        worst = [wl.beta + 1] * wl.E
+        if sum(worst) <= Nr:
+            assert sum(-(-c // wl.beta) for c in worst) <= b_max
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("k", 9, N.MOE_ERR_INVALID_ARG), ("k", 0, N.MOE_ERR_INVALID_ARG),
+    ("beta", 96, N.MOE_ERR_INVALID_ARG), ("P", 9, N.MOE_ERR_INVALID_ARG),
+    ("P", 0, N.MOE_ERR_INVALID_ARG), ("s", -1, N.MOE_ERR_INVALID_ARG),
+    ("T", -1, N.MOE_ERR_INVALID_ARG), ("E", 300, N.MOE_ERR_UNSUPPORTED),
+    ("T", (1 << 21) + 1, N.MOE_ERR_UNSUPPORTED),
+])
+def test_bad_config_rejected_everywhere(field, value, code):
+    wl = WORKLOADS["tiny"].with_(**{field: value})
+    cfg = N.MoeCfg.of(wl)
+    fake = 1 << 20  # never dereferenced: the config check comes first
+    lib = N.lib()
+    p = ctypes.byref(cfg)
+    assert lib.moe_workspace_size(p, 0) == 0
+    assert lib.moe_route_hist(p, *[fake] * 7, None) == code
+    assert lib.moe_plan_blocks(p, fake, 0, *[fake] * 8, None) == code
+    assert lib.moe_dispatch_permute(p, *[fake] * 9, None) == code
+    assert lib.moe_expert_ffn(p, *[fake] * 7, 0, *[fake] * 3, None) == code
+    assert lib.moe_combine(p, *[fake] * 5, None) == code
+
+
+@pytest.mark.skipif(not NO_GPU, reason="fake pointers are only passed where no GPU exists")
+def test_null_and_misaligned_pointers_rejected():
+    cfg = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"]))
+    lib = N.lib()
+    ok = 1 << 20
+    for i in range(7):
+        args = [ok] * 7
+        args[i] = None
+        assert lib.moe_route_hist(cfg, *args, None) == N.MOE_ERR_INVALID_ARG
+        args[i] = ok + 4
+        assert lib.moe_route_hist(cfg, *args, None) == N.MOE_ERR_UNSUPPORTED
+    for i in range(10):
+        args = [ok] * 10
+        args[i] = ok + 8
+        assert lib.moe_expert_ffn(cfg, *args[:7], 0, *args[7:], None) == N.MOE_ERR_UNSUPPORTED
+    assert lib.moe_plan_blocks(cfg, ok, 16, *[ok] * 8, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_ffn(cfg, *[ok] * 7, 4, *[ok] * 3, None) == N.MOE_ERR_INVALID_ARG
+    bad_d = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(d=320)))
+    assert lib.moe_expert_ffn(bad_d, *[ok] * 7, 0, *[ok] * 3, None) == N.MOE_ERR_UNSUPPORTED
+    bad_f = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(f=192)))
+    assert lib.moe_expert_ffn(bad_f, *[ok] * 7, 0, *[ok] * 3, None) == N.MOE_ERR_UNSUPPORTED
+
+
+def test_status_strings():
+    assert N.moe_status_string(0) == "ok"
+    for code in (-1, -2, -3, 1, 2, 4, 8, 16):
+        assert N.moe_status_string(code) not in ("", "unknown code")
+
+
+def test_binding_refuses_host_tensors():
+    with pytest.raises(TypeError):
+        N.moe_route_hist(WORKLOADS["tiny"], torch.zeros(4), *[torch.zeros(4)] * 6)
