@@ -136,17 +136,28 @@ def oracle_sample(wl, logits, x, get_expert, n_tokens):
                          P=wl.P, s=wl.s)
 
 
-def host_expert_getter(w1, w2):
-    """Expert weights for the oracle, copied to the host one expert at a time."""
-    cache = {}
+class ExpertCache:
+    """fp32 host copies of expert weights for the oracle, loaded on first use and kept
+    while they fit in `max_bytes` (oldest dropped first)."""
 
-    def get(e):
-        if e not in cache:
-            if len(cache) > 64:
-                cache.clear()
-            cache[e] = (w1[e].float().cpu().numpy(), w2[e].float().cpu().numpy())
-        return cache[e]
-    return get
+    def __init__(self, load, max_bytes=6e9):
+        self.load, self.max_bytes, self.cache, self.bytes = load, max_bytes, {}, 0
+
+    def __call__(self, e):
+        if e not in self.cache:
+            w = self.load(e)
+            size = sum(a.nbytes for a in w)
+            while self.cache and self.bytes + size > self.max_bytes:
+                old = next(iter(self.cache))
+                self.bytes -= sum(a.nbytes for a in self.cache.pop(old))
+            self.cache[e] = w
+            self.bytes += size
+        return self.cache[e]
+
+
+def host_expert_getter(w1, w2):
+    """Expert weights for the oracle, copied from the device one expert at a time."""
+    return ExpertCache(lambda e: (w1[e].float().cpu().numpy(), w2[e].float().cpu().numpy()))
 
 
 def cpu_cores():
@@ -157,19 +168,51 @@ def cpu_cores():
 
 
 def time_oracle(wl, logits_np, x_np, get_expert, budget_s):
-    """Times the oracle on a token sample sized to about budget_s seconds of CPU work."""
-    n = min(wl.T, 64)
-    t0 = time.perf_counter()
-    oracle_sample(wl, logits_np, x_np, get_expert, n)
-    per_tok = (time.perf_counter() - t0) / n
-    n = int(max(1, min(wl.T, budget_s / max(per_tok, 1e-9))))
-    t0 = time.perf_counter()
-    oracle_sample(wl, logits_np, x_np, get_expert, n)
-    dt = time.perf_counter() - t0
-    return n, dt
+    """Times the oracle on the first n tokens, n grown until one run takes about budget_s
+    seconds of CPU work (or covers the whole workload).  Returns (n, seconds)."""
+    n = min(wl.T, 16)
+    oracle_sample(wl, logits_np, x_np, get_expert, n)  # untimed: loads the first experts
+    while True:
+        t0 = time.perf_counter()
+        oracle_sample(wl, logits_np, x_np, get_expert, n)
+        dt = time.perf_counter() - t0
+        if n >= wl.T or dt >= 0.5 * budget_s:
+            return n, dt
+        grow = budget_s / max(dt, 1e-6)
+        n = int(min(wl.T, max(n + 1, n * min(grow, 8.0))))
 
 
 # ------------------------------------------------------------------ our arm
+def run_e2e(layer, logits_h, x_h, logits, x, w1, w2, mode, wl, args, world, dev):
+    """The same layer end to end through the public API: every step copies that step's
+    inputs (logits, x) from pinned host memory and reads y back to pinned host memory."""
+    stream = torch.cuda.current_stream(dev)
+    logits_p = logits_h.pin_memory()
+    x_p = x_h.pin_memory()
+    y_p = torch.empty(wl.T, wl.d, dtype=torch.float32).pin_memory()
+    steps = max(1, min(args.steps, 200))
+    for _ in range(2):
+        layer.forward_host(logits_p, x_p, w1, w2, y_p, logits, x, mode=mode)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        layer.forward_host(logits_p, x_p, w1, w2, y_p, logits, x, mode=mode)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        tt = torch.tensor([t], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        t = float(tt.item())
+    return {"value": round(wl.T * wl.k * steps * world / t, 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": logits_h.numel() * 4 + x_h.numel() * 2,
+            "d2h_bytes_per_step": wl.T * wl.d * 4, "steps": steps}
+
+
 def run_ours(args, wl, world, rank, local):
     from skew_aware_token_b200.layer import MoeLayer
     dev = torch.device("cuda", local)
@@ -181,21 +224,23 @@ def run_ours(args, wl, world, rank, local):
     x = x_h.to(dev)
     layer = MoeLayer(wl, dev)
     stream = torch.cuda.current_stream(dev)
+    mode = N.MOE_FFN_STRICT_SLOTS if args.strict else 0
+    vmask = 0
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
     def step(record=None):
         if record is None:
-            layer(logits, x, w1, w2)
+            layer(logits, x, w1, w2, mode=mode, variant_mask=vmask)
             return
         record[0].record(stream)
         layer.route(logits)
         record[1].record(stream)
-        layer.plan(0)
+        layer.plan(vmask)
         record[2].record(stream)
         layer.dispatch(x)
         record[3].record(stream)
-        layer.ffn(w1, w2)
+        layer.ffn(w1, w2, mode)
         record[4].record(stream)
 
     layer.clear_status()
@@ -252,30 +297,11 @@ def run_ours(args, wl, world, rank, local):
         if tr:
             roofline["traffic"] = tr
 
-    # end to end through the public API: pinned host inputs in, y out, every step
-    logits_p = logits_h.pin_memory()
-    x_p = x_h.pin_memory()
-    y_p = torch.empty(wl.T, wl.d, dtype=torch.float32).pin_memory()
-    e2e_steps = max(1, min(args.steps, 200))
-    for _ in range(2):
-        layer.forward_host(logits_p, x_p, w1, w2, y_p, logits, x)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
-    e0, e1 = ev(), ev()
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        layer.forward_host(logits_p, x_p, w1, w2, y_p, logits, x)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_t = e0.elapsed_time(e1) / 1e3
-    if world > 1:
-        t = torch.tensor([e2e_t], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_t = float(t.item())
-    h2d = logits_h.numel() * 4 + x_h.numel() * 2
-    d2h = wl.T * wl.d * 4
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(layer, logits_h, x_h, logits, x, w1, w2, mode, wl, args, world, dev)
 
+    cpu = None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n, dt = time_oracle(wl, logits_h.numpy(), x_h.float().numpy(),
@@ -292,14 +318,14 @@ def run_ours(args, wl, world, rank, local):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; router logits N(0,1) + Zipf bias, x N(0,1), "
                 "weights N(0, 1/sqrt(fan_in)), random-init)",
-        "config": workload_config(wl, {"kappa": kappa, "l2": "inputs larger than L2 "
+        "config": workload_config(wl, {"kappa": kappa, "strict_slots": bool(args.strict),
+                                       "l2": "inputs larger than L2 "
                                        f"(expert weights {weight_bytes / 1e9:.2f} GB > 126 MB)",
                                        "B": pi[0], "tau": pi[1], "makespan": pi[2],
                                        "fixed_makespan": pi[5], "variant": pi[3]}),
         "tflops": round(tflops, 2), "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roofline, "cpu_baseline": cpu,
-        "e2e": {"value": round(wl.T * wl.k * e2e_steps * world / e2e_t, 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clocks.summary(),
         "impl": "ours",
@@ -314,16 +340,13 @@ def run_reference(args, wl, world, rank):
         return
     logits_h = synth.make_logits(wl)
     x_h = synth.make_x(wl)
-    # the oracle reads host weights; draw them on the host with the same recipe
-    cache = {}
-
-    def get_expert(e):
-        if e not in cache:
-            if len(cache) > 64:
-                cache.clear()
-            w1, w2 = synth.expert_weights(wl, e, "cpu")
-            cache[e] = (w1.float().numpy(), w2.float().numpy())
-        return cache[e]
+    # the oracle reads host weights: drawn on the host with the same recipe (the host
+    # generator's values differ from the device's; the work is the same)
+    get_expert = ExpertCache(lambda e: tuple(w.float().numpy()
+                                             for w in synth.expert_weights(wl, e, "cpu")))
+    if wl.E * 3 * wl.d * wl.f * 4 <= get_expert.max_bytes:
+        for e in range(wl.E):
+            get_expert(e)
 
     logits_np, x_np = logits_h.numpy(), x_h.float().numpy()
     total = args.warmup + args.steps
@@ -364,10 +387,17 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=120.0,
                     help="seconds of CPU work for the whole reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--strict", action="store_true",
+                    help="strict slots: CTA c only runs slot c mod P (one GPU standing in for P)")
+    ap.add_argument("--fixed-placement", action="store_true",
+                    help="plan with replica budget s = 0 (the no-replica baseline)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     wl = synth.WORKLOADS[args.workload]
+    if args.fixed_placement:
+        wl = wl.with_(s=0)
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
