@@ -62,7 +62,8 @@ enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = -1, /* NULL pointer, k > E, k > 8, beta not 64/128, P > 8, ... */
   MOE_ERR_UNSUPPORTED = -2, /* shape outside what the kernels take, misaligned pointer */
-  MOE_ERR_CUDA = -3         /* a launch or a CUDA call failed */
+  MOE_ERR_CUDA = -3,        /* a launch or a CUDA call failed */
+  MOE_ERR_TOO_LARGE = -4    /* moe_expert_ffn_noalloc: A would not fit its fixed array */
 };
 
 /* device-detected problems (bits OR-ed into *status) */
@@ -186,6 +187,29 @@ MOE_API int moe_expert_ffn(const moe_cfg* cfg, const uint16_t* xp, const uint16_
  *   o bf16 [R_max, d]; tok_row, topk_gates [T, k]; y fp32 [T, d] (overwritten). */
 MOE_API int moe_combine(const moe_cfg* cfg, const uint16_t* o, const int32_t* tok_row,
                 const float* topk_gates, float* y, int32_t* status, moe_stream_t stream);
+
+/* Size of the library's fixed FC1-output array used by moe_expert_ffn_noalloc. */
+#define MOE_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* moe_expert_ffn without the caller's scratch buffer, for callers that cannot allocate
+ * device memory (a plugin or custom operator that its host framework hands only inputs
+ * and outputs, or a deployment that forbids cudaMalloc after start-up).  The pages have no
+ * counterpart: this is a deployment variant of the FFN entry point above.
+ *   Arguments, modes, outputs and device status are those of moe_expert_ffn, without
+ *   a_scratch: A (bf16 [R_max, f]) lives in a library-owned array of
+ *   MOE_NOALLOC_SCRATCH_BYTES, so R_max * f * 2 must not exceed it, else the call returns
+ *   MOE_ERR_TOO_LARGE and enqueues nothing.
+ *   The call allocates nothing.  The array is reserved on every GPU where the library's
+ *   device code is loaded, until the process exits.  The first call on a device looks up
+ *   the array's device address (cudaGetSymbolAddress, with that device current) and caches
+ *   it, so make that first call before any stream capture.
+ *   All calls share the array and it keeps the last call's contents; calls whose kernels
+ *   overlap on the GPU (e.g. on two streams) race on it and must be serialised. */
+MOE_API int moe_expert_ffn_noalloc(const moe_cfg* cfg, const uint16_t* xp, const uint16_t* w1,
+                                   const uint16_t* w2, const int32_t* tiles,
+                                   const int32_t* plan_info, const int32_t* row_token,
+                                   const float* row_gate, int mode, void* out,
+                                   int32_t* status, moe_stream_t stream);
 
 /* Static text for a return code (negative) or a status bit mask (positive). */
 MOE_API const char* moe_status_string(int code);

@@ -119,6 +119,7 @@ const char* moe_status_string(int code) {
     case MOE_ERR_INVALID_ARG: return "invalid argument";
     case MOE_ERR_UNSUPPORTED: return "unsupported shape or misaligned pointer";
     case MOE_ERR_CUDA: return "CUDA launch or call failed";
+    case MOE_ERR_TOO_LARGE: return "problem too large for the fixed scratch of moe_expert_ffn_noalloc";
     case MOE_STATUS_BAD_ID: return "expert id out of range";
     case MOE_STATUS_OVERFLOW: return "expert rows exceed their blocks";
     case MOE_STATUS_NONFINITE: return "non-finite router logit";

@@ -17,6 +17,8 @@ HEADER_PATH = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__fil
                            "include", "moeskew.h")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA = 0, -1, -2, -3
+MOE_ERR_TOO_LARGE = -4
+MOE_NOALLOC_SCRATCH_BYTES = 64 << 20
 MOE_STATUS_BAD_ID, MOE_STATUS_OVERFLOW, MOE_STATUS_NONFINITE = 1, 2, 4
 MOE_STATUS_TIMEOUT, MOE_STATUS_PLAN = 8, 16
 MOE_WS_ROWS, MOE_WS_BLOCKS = 0, 1
@@ -48,6 +50,8 @@ _SIGNATURES = {
     "moe_expert_ffn": (ctypes.c_int, [ctypes.POINTER(MoeCfg)] + [_VP] * 7 + [ctypes.c_int] +
                        [_VP] * 4),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(MoeCfg)] + [_VP] * 6),
+    "moe_expert_ffn_noalloc": (ctypes.c_int, [ctypes.POINTER(MoeCfg)] + [_VP] * 7 +
+                               [ctypes.c_int] + [_VP] * 3),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
@@ -155,3 +159,13 @@ def moe_combine(cfg, o, tok_row, topk_gates, y, status, stream=None) -> None:
     _check("moe_combine", lib().moe_combine(
         ctypes.byref(c), _dev(o, "o"), _dev(tok_row, "tok_row"), _dev(topk_gates, "topk_gates"),
         _dev(y, "y"), _dev(status, "status"), _stream(stream)))
+
+
+def moe_expert_ffn_noalloc(cfg, xp, w1, w2, tiles, plan_info, row_token, row_gate, mode, out,
+                           status, stream=None) -> None:
+    """moe_expert_ffn without a caller scratch buffer (the library's fixed array holds A)."""
+    c = _cfg(cfg)
+    _check("moe_expert_ffn_noalloc", lib().moe_expert_ffn_noalloc(
+        ctypes.byref(c), _dev(xp, "xp"), _dev(w1, "w1"), _dev(w2, "w2"), _dev(tiles, "tiles"),
+        _dev(plan_info, "plan_info"), _dev(row_token, "row_token"), _dev(row_gate, "row_gate"),
+        int(mode), _dev(out, "out"), _dev(status, "status"), _stream(stream)))

@@ -24,7 +24,7 @@ def test_exports_every_declared_symbol():
     declared = N.declared_symbols()
     assert set(declared) == {"moe_workspace_size", "moe_route_hist", "moe_plan_blocks",
                              "moe_dispatch_permute", "moe_expert_ffn", "moe_combine",
-                             "moe_status_string"}
+                             "moe_status_string", "moe_expert_ffn_noalloc"}
     out = subprocess.run(["nm", "-D", "--defined-only", N.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
@@ -93,7 +93,7 @@ def test_null_and_misaligned_pointers_rejected():
 
 def test_status_strings():
     assert N.moe_status_string(0) == "ok"
-    for code in (-1, -2, -3, 1, 2, 4, 8, 16):
+    for code in (-1, -2, -3, -4, 1, 2, 4, 8, 16):
         assert N.moe_status_string(code) not in ("", "unknown code")
 
 
