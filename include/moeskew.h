@@ -26,7 +26,8 @@
  *
  * Sizes: N = T*k routed rows; b_e = ceil(c_e/beta) blocks of expert e; B = sum_e b_e;
  * B_max = floor((N + min(E,N)*(beta-1)) / beta) bounds B for every routing; R_max =
- * beta*B_max bounds the padded rows.  moe_workspace_size() returns both.
+ * beta*B_max bounds the padded rows.  moe_workspace_size() returns both, and the byte size
+ * of the FFN's scratch buffer.
  */
 #ifndef MOESKEW_H
 #define MOESKEW_H
@@ -76,7 +77,7 @@ enum {
 };
 
 /* moe_workspace_size(which) */
-enum { MOE_WS_ROWS = 0, MOE_WS_BLOCKS = 1 };
+enum { MOE_WS_ROWS = 0, MOE_WS_BLOCKS = 1, MOE_WS_FFN_SCRATCH = 2 };
 
 /* plan_info layout (int32[MOE_PI_LEN]) written by moe_plan_blocks */
 enum {
@@ -106,7 +107,9 @@ enum {
 };
 
 /* Upper bounds: which = MOE_WS_ROWS -> R_max rows (Xp, A, O, row_token, row_gate);
- * MOE_WS_BLOCKS -> B_max entries (blocks, tiles).  Returns 0 for an invalid cfg. */
+ * MOE_WS_BLOCKS -> B_max entries (blocks, tiles); MOE_WS_FFN_SCRATCH -> bytes of the
+ * a_scratch buffer of moe_expert_ffn (A, bf16 [R_max, f], rounded up to 256 bytes, then
+ * 256 bytes of tile-scheduler counters).  Returns 0 for an invalid cfg. */
 MOE_API size_t moe_workspace_size(const moe_cfg* cfg, int which);
 
 /* Router top-k, expert histogram and skew ("Routing Skew Problem"; router outputs of the
@@ -169,7 +172,9 @@ MOE_API int moe_dispatch_permute(const moe_cfg* cfg, const uint16_t* x, const in
  *   w1         bf16 [E, 2f, d] (rows 0..f-1 = G, f..2f-1 = U; K-major).
  *   w2         bf16 [E, d, f] (K-major).
  *   tiles, plan_info from moe_plan_blocks; row_token, row_gate from moe_dispatch_permute.
- *   a_scratch  bf16 [R_max, f], caller-owned scratch.
+ *   a_scratch  caller-owned scratch of moe_workspace_size(cfg, MOE_WS_FFN_SCRATCH)
+ *              bytes: A (bf16 [R_max, f]) then the tile-scheduler counters, which the
+ *              call zeroes itself.
  *   out        MOE_FFN_FUSED_COMBINE: y fp32 [T, d], zeroed by the call, then
  *              y[row_token[r]] += row_gate[r] * O[r] for every valid row (fp32 atomic
  *              adds: the summation order, and so the last bits, may vary run to run).
@@ -196,8 +201,9 @@ MOE_API int moe_combine(const moe_cfg* cfg, const uint16_t* o, const int32_t* to
  * and outputs, or a deployment that forbids cudaMalloc after start-up).  The pages have no
  * counterpart: this is a deployment variant of the FFN entry point above.
  *   Arguments, modes, outputs and device status are those of moe_expert_ffn, without
- *   a_scratch: A (bf16 [R_max, f]) lives in a library-owned array of
- *   MOE_NOALLOC_SCRATCH_BYTES, so R_max * f * 2 must not exceed it, else the call returns
+ *   a_scratch: its contents (A and the tile-scheduler counters, together
+ *   moe_workspace_size(cfg, MOE_WS_FFN_SCRATCH) bytes) live in a library-owned array of
+ *   MOE_NOALLOC_SCRATCH_BYTES, which they must not exceed, else the call returns
  *   MOE_ERR_TOO_LARGE and enqueues nothing.
  *   The call allocates nothing.  The array is reserved on every GPU where the library's
  *   device code is loaded, until the process exits.  The first call on a device looks up

@@ -48,6 +48,7 @@ size_t moe_workspace_size(const moe_cfg* cfg, int which) {
   if (check_cfg(cfg) != MOE_OK) return 0;
   if (which == MOE_WS_ROWS) return (size_t)max_rows(*cfg);
   if (which == MOE_WS_BLOCKS) return (size_t)max_blocks(*cfg);
+  if (which == MOE_WS_FFN_SCRATCH) return (size_t)ffn_scratch_bytes(*cfg);
   return 0;
 }
 

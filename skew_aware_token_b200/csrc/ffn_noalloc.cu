@@ -15,8 +15,8 @@
 // cudaGetSymbolAddress and caches it; that first call should therefore come before any
 // stream capture.  All calls share the one array: its contents are whatever the last
 // call left, and calls whose kernels overlap on the GPU (for example on two streams)
-// race on it.  Nothing in it needs to start at zero: FC1 writes every row of A that FC2
-// reads for an output row.
+// race on it.  The only part that must start at zero, the tile-scheduler counters, is
+// zeroed by every call; FC1 writes every row of A that FC2 reads for an output row.
 #include <mutex>
 
 #include "moe_common.cuh"
@@ -72,9 +72,8 @@ extern "C" MOE_API int moe_expert_ffn_noalloc(const moe_cfg* cfg, const uint16_t
     if (!p) return MOE_ERR_INVALID_ARG;
     if (!aligned16(p)) return MOE_ERR_UNSUPPORTED;
   }
-  // A is bf16 [R_max, f]: it must fit the fixed array
-  if ((unsigned long long)max_rows(c) * (unsigned long long)c.f * 2ull >
-      (unsigned long long)MOE_NOALLOC_SCRATCH_BYTES)
+  // A (bf16 [R_max, f]) and the scheduler counters must fit the fixed array
+  if ((unsigned long long)ffn_scratch_bytes(c) > (unsigned long long)MOE_NOALLOC_SCRATCH_BYTES)
     return MOE_ERR_TOO_LARGE;
   void* scratch = nullptr;
   const int rc = scratch_on_current_device(&scratch);

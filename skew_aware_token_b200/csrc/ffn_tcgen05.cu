@@ -22,10 +22,13 @@
 //                      (fused combine), or O rounded to bf16 (unfused path).
 //   TMEM holds two 256-column accumulators (512 columns), so the epilogue of one work item
 //   overlaps the MMAs of the next.
-// Work items: item L -> m-tile L / n_n, n-tile L % n_n, dealt round-robin to the CTAs
-// (all n-tiles of a block are in flight together, and consecutive blocks belong to the
-// same expert, so each expert's weights stream from HBM about once).  With
-// MOE_FFN_STRICT_SLOTS, CTA c only deals slot (c mod P)'s tiles.
+// Work items: item L -> m-tile L / n_n, n-tile L % n_n, handed out in increasing L by a
+// global atomic counter (the producer thread draws the next item when it is ready for
+// it, so faster SMs take more items) and passed to the MMA and epilogue warps through a
+// small shared-memory ring.  All n-tiles of a block are in flight together, and
+// consecutive blocks belong to the same expert, so each expert's weights stream from HBM
+// about once.  With MOE_FFN_STRICT_SLOTS, CTA c draws from slot (c mod P)'s counter and
+// only runs that slot's tiles.
 // Every mbarrier wait is bounded (globaltimer); on expiry the kernel sets
 // MOE_STATUS_TIMEOUT, lets the other roles drop out, waits (bounded) for its own copies
 // and MMAs in flight, frees its TMEM and returns.
@@ -49,7 +52,8 @@ constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int RING = 8;   // work items in flight between the producer and the consumers
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512;  // + alignment slack, barriers
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per wait
 
 // kind::f16 instruction descriptor: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 = 1),
@@ -58,6 +62,7 @@ constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
                             ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
 struct FfnArgs {
+  int32_t* sched;           // this launch's counters: [0] or [slot] (strict), zeroed
   const int32_t* tiles;
   const int32_t* plan_info;
   const int32_t* row_token;
@@ -187,14 +192,12 @@ __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g));
 
 // ------------------------------------------------------------------ work schedule
 struct Sched {
-  long long total, first, stride;
+  int32_t* counter;   // global counter this CTA draws items from
+  long long total;    // items in its range
   int m_base, n_n;
-  __device__ bool get(int it, int& m, int& n) const {
-    const long long L = first + (long long)it * stride;
-    if (L >= total) return false;
-    m = m_base + (int)(L / n_n);
-    n = (int)(L % n_n);
-    return true;
+  __device__ void decode(int L, int& m, int& n) const {
+    m = m_base + L / n_n;
+    n = L % n_n;
   }
 };
 
@@ -203,16 +206,14 @@ __device__ Sched make_sched(const FfnArgs& a) {
   s.n_n = a.n_n;
   const int* pi = a.plan_info;
   if (!a.strict) {
+    s.counter = a.sched;
     s.total = (long long)max(pi[MOE_PI_NTILES], 0) * a.n_n;
-    s.first = blockIdx.x;
-    s.stride = gridDim.x;
     s.m_base = 0;
   } else {
     const int r = blockIdx.x % a.P;
     const int lo = pi[MOE_PI_SLOT_TILE_OFF + r], hi = pi[MOE_PI_SLOT_TILE_OFF + r + 1];
+    s.counter = a.sched + r;
     s.total = (long long)max(hi - lo, 0) * a.n_n;
-    s.first = blockIdx.x / a.P;
-    s.stride = (gridDim.x - r + a.P - 1) / a.P;
     s.m_base = lo;
   }
   return s;
@@ -241,9 +242,11 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  // bars: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  // bars: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain,
+  //       item_full[RING], item_empty[RING]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5 + 2 * RING);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [RING] items
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
@@ -251,6 +254,8 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
   auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 + b); };
   const uint32_t drain_bar = smem_u32(bars + 2 * STAGES + 4);
+  auto ifull_bar = [&](int i) { return smem_u32(bars + 2 * STAGES + 5 + i); };
+  auto iempty_bar = [&](int i) { return smem_u32(bars + 2 * STAGES + 5 + RING + i); };
   auto sA = [&](int s) { return smem_u32(smem + s * STAGE_BYTES); };
   auto sB = [&](int s) { return smem_u32(smem + s * STAGE_BYTES + A_BYTES); };
 
@@ -264,6 +269,10 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       mbar_init(tempty_bar(b), 4 * 32);
     }
     mbar_init(drain_bar, 1);
+    for (int i = 0; i < RING; ++i) {
+      mbar_init(ifull_bar(i), 1);
+      mbar_init(iempty_bar(i), 1 + 4);  // the MMA thread and the four epilogue warps
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -290,8 +299,16 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       uint32_t pending = 0, pend_parity = 0;
       bool bad_tile = false;
       for (int it = 0;; ++it) {
+        const int slot = it % RING;
+        const uint32_t ph = (uint32_t)(it / RING) & 1u;
+        if (!mbar_wait(iempty_bar(slot), ph ^ 1u, abort_flag, a.status, a.timeout_ns, true))
+          break;
+        const long long L = atomicAdd(sch.counter, 1);
+        ring[slot] = L < sch.total ? (int)L : -1;
+        mbar_arrive(ifull_bar(slot));
+        if (L >= sch.total) break;
         int m, n;
-        if (!sch.get(it, m, n)) break;
+        sch.decode((int)L, m, n);
         const TileInfo ti = read_tile(a, m);
         if (!ti.ok) {
           bad_tile = true;
@@ -338,8 +355,14 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       int acc_it = 0;
       bool issued = false;
       for (int it = 0;; ++it) {
+        const int slot = it % RING;
+        const uint32_t ph = (uint32_t)(it / RING) & 1u;
+        if (!mbar_wait(ifull_bar(slot), ph, abort_flag, a.status, a.timeout_ns, true)) break;
+        const int L = ring[slot];
+        mbar_arrive(iempty_bar(slot));
+        if (L < 0) break;
         int m, n;
-        if (!sch.get(it, m, n)) break;
+        sch.decode(L, m, n);
         const TileInfo ti = read_tile(a, m);
         if (!ti.ok) continue;
         const int buf = acc_it & 1;
@@ -383,8 +406,17 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     const int rit = quarter * 32 + lane;  // row inside the tile
     int acc_it = 0;
     for (int it = 0;; ++it) {
+      const int slot = it % RING;
+      const uint32_t ph = (uint32_t)(it / RING) & 1u;
+      const bool have =
+          mbar_wait(ifull_bar(slot), ph, abort_flag, a.status, a.timeout_ns, true);
+      if (!__all_sync(0xffffffffu, have)) break;
+      const int L = ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(iempty_bar(slot));
+      if (L < 0) break;
       int m, n;
-      if (!sch.get(it, m, n)) break;
+      sch.decode(L, m, n);
       const TileInfo ti = read_tile(a, m);
       if (!ti.ok) continue;
       const int buf = acc_it & 1;
@@ -521,6 +553,12 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   }
   if (r_max == 0) return cudaSuccess;
 
+  // scheduler counters after A in the scratch buffer: [0, 8) FC1, [8, 16) FC2
+  int32_t* sched = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(a_scratch) +
+                                              ffn_a_bytes(c));
+  err = cudaMemsetAsync(sched, 0, 16 * sizeof(int32_t), st);
+  if (err != cudaSuccess) return err;
+
   CUtensorMap tm_xp, tm_w1, tm_a, tm_w2;
   if (!encode_2d(&tm_xp, xp, c.d, r_max, BM) ||
       !encode_2d(&tm_w1, w1, c.d, (uint64_t)c.E * 2 * c.f, BN / 2) ||
@@ -552,6 +590,8 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   a1.timeout_ns = kTimeoutNs;
 
   FfnArgs a2 = a1;
+  a1.sched = sched;
+  a2.sched = sched + 8;
   a1.out = a_scratch;
   a1.n_k = c.d / BK;
   a1.n_n = c.f / (BN / 2);

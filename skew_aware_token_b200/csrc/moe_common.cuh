@@ -22,6 +22,14 @@ inline long long max_blocks(const moe_cfg& c) {
 }
 inline long long max_rows(const moe_cfg& c) { return max_blocks(c) * c.beta; }
 
+// FFN scratch: A (bf16 [R_max, f]) rounded up to 256 bytes, then the tile-scheduler
+// counters (kSchedBytes).
+constexpr long long kSchedBytes = 256;
+inline long long ffn_a_bytes(const moe_cfg& c) {
+  return (max_rows(c) * c.f * 2 + 255) / 256 * 256;
+}
+inline long long ffn_scratch_bytes(const moe_cfg& c) { return ffn_a_bytes(c) + kSchedBytes; }
+
 __device__ __forceinline__ void set_status(int32_t* status, int bits) {
   atomicOr(status, bits);
 }

@@ -44,7 +44,8 @@ class MoeLayer:
         self.row_token = z(max(R, 4))
         self.row_gate = z(max(R, 4), dt=f32)
         self.tok_row = z(max(T * k, 4))
-        self.a_scratch = z(max(R * f, 8), dt=torch.bfloat16)
+        ws = N.moe_workspace_size(self.cfg, N.MOE_WS_FFN_SCRATCH)
+        self.a_scratch = z(max(ws // 2, 8), dt=torch.bfloat16)
         self.y = z(max(T * d, 4), dt=f32)
         self.o = z(max(R * d, 8), dt=torch.bfloat16) if write_o else None
         self.device = dev

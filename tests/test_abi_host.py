@@ -41,6 +41,8 @@ def test_workspace_sizes_follow_the_block_bound():
         b_max = (Nr + min(wl.E, Nr) * (wl.beta - 1)) // wl.beta
         assert N.moe_workspace_size(wl, N.MOE_WS_BLOCKS) == b_max
         assert N.moe_workspace_size(wl, N.MOE_WS_ROWS) == b_max * wl.beta
+        a_bytes = (b_max * wl.beta * wl.f * 2 + 255) // 256 * 256
+        assert N.moe_workspace_size(wl, N.MOE_WS_FFN_SCRATCH) == a_bytes + 256
         # the bound holds for the worst routing: every expert one row past a block
         worst = [wl.beta + 1] * wl.E
         if sum(worst) <= Nr:

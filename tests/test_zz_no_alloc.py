@@ -32,7 +32,7 @@ def _within(got: torch.Tensor, ref: torch.Tensor) -> bool:
 @pytest.mark.parametrize("wl", CASES, ids=lambda w: w.name)
 @pytest.mark.parametrize("mode", [N.MOE_FFN_FUSED_COMBINE, N.MOE_FFN_WRITE_O])
 def test_noalloc_matches_scratch_entry_point_twice(wl, mode):
-    assert N.moe_workspace_size(wl, N.MOE_WS_ROWS) * wl.f * 2 <= N.MOE_NOALLOC_SCRATCH_BYTES
+    assert N.moe_workspace_size(wl, N.MOE_WS_FFN_SCRATCH) <= N.MOE_NOALLOC_SCRATCH_BYTES
     torch.manual_seed(0)
     logits, x = synth.make_logits(wl).cuda(), synth.make_x(wl).cuda()
     w1, w2 = synth.make_weights(wl, "cuda")
@@ -64,7 +64,7 @@ def test_noalloc_matches_scratch_entry_point_twice(wl, mode):
 
 def test_noalloc_refuses_a_problem_larger_than_its_array():
     wl = WORKLOADS["olmoe_a1"]
-    assert N.moe_workspace_size(wl, N.MOE_WS_ROWS) * wl.f * 2 > N.MOE_NOALLOC_SCRATCH_BYTES
+    assert N.moe_workspace_size(wl, N.MOE_WS_FFN_SCRATCH) > N.MOE_NOALLOC_SCRATCH_BYTES
     w1, w2 = synth.make_weights(wl, "cuda")
     layer = MoeLayer(wl, "cuda")
     cfg = N.MoeCfg.of(wl)
