@@ -222,9 +222,11 @@ def run_ours(args, wl, world, rank, local):
     w1, w2 = synth.make_weights(wl, dev)
     logits = logits_h.to(dev)
     x = x_h.to(dev)
-    layer = MoeLayer(wl, dev)
+    write_o = args.ffn == "write_o"
+    layer = MoeLayer(wl, dev, write_o=write_o)
     stream = torch.cuda.current_stream(dev)
-    mode = N.MOE_FFN_STRICT_SLOTS if args.strict else 0
+    mode = ((N.MOE_FFN_STRICT_SLOTS if args.strict else 0) |
+            (N.MOE_FFN_WRITE_O if write_o else 0) | (N.MOE_FFN_SM_PAIR if args.sm_pair else 0))
     vmask = 0
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
@@ -241,6 +243,8 @@ def run_ours(args, wl, world, rank, local):
         layer.dispatch(x)
         record[3].record(stream)
         layer.ffn(w1, w2, mode)
+        if write_o:
+            layer.combine()
         record[4].record(stream)
 
     layer.clear_status()
@@ -319,6 +323,7 @@ def run_ours(args, wl, world, rank, local):
         "data": "synthetic (seeded; router logits N(0,1) + Zipf bias, x N(0,1), "
                 "weights N(0, 1/sqrt(fan_in)), random-init)",
         "config": workload_config(wl, {"kappa": kappa, "strict_slots": bool(args.strict),
+                                       "ffn": args.ffn, "sm_pair": bool(args.sm_pair),
                                        "l2": "inputs larger than L2 "
                                        f"(expert weights {weight_bytes / 1e9:.2f} GB > 126 MB)",
                                        "B": pi[0], "tau": pi[1], "makespan": pi[2],
@@ -326,7 +331,7 @@ def run_ours(args, wl, world, rank, local):
         "tflops": round(tflops, 2), "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roofline, "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": (LAUNCHES_PER_STEP + (1 if write_o else 0)) * args.steps,
         "clocks": clocks.summary(),
         "impl": "ours",
     }
@@ -388,6 +393,10 @@ def main():
                     help="seconds of CPU work for the whole reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ffn", default="fused", choices=["fused", "write_o"],
+                    help="fused: FC2 adds gate*O into y; write_o: FC2 stores O, then moe_combine")
+    ap.add_argument("--sm-pair", action="store_true",
+                    help="run the FFN on SM pairs (tcgen05 cta_group::2) instead of single SMs")
     ap.add_argument("--strict", action="store_true",
                     help="strict slots: CTA c only runs slot c mod P (one GPU standing in for P)")
     ap.add_argument("--fixed-placement", action="store_true",

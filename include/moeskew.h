@@ -85,7 +85,7 @@ enum {
   MOE_PI_TAU = 1,            /* tau = ceil(B / P) */
   MOE_PI_MAKESPAN = 2,       /* max_r l_r of the chosen plan */
   MOE_PI_VARIANT = 3,        /* chosen greedy variant (0..3) */
-  MOE_PI_NTILES = 4,         /* number of 128-row execution tiles */
+  MOE_PI_NTILES = 4,         /* number of execution tiles (up to 256 rows each) */
   MOE_PI_FIXED_MAKESPAN = 5, /* max_r l_r of the no-replica (fixed placement) plan */
   MOE_PI_REPLICAS = 6,       /* total replicas of the chosen plan */
   MOE_PI_ROUNDS = 7,         /* greedy rounds of the chosen plan */
@@ -101,9 +101,13 @@ enum {
   MOE_FFN_FUSED_COMBINE = 0, /* out = y fp32 [T, d]; the call zeroes y, then FC2's
                                 epilogue adds row_gate * O into y[row_token] */
   MOE_FFN_WRITE_O = 1,       /* out = O bf16 [R_max, d]; moe_combine reduces it */
-  MOE_FFN_STRICT_SLOTS = 2   /* flag: CTA c only runs slot (c mod P)'s tiles, so the
-                                layer time follows the plan's makespan (one GPU standing
-                                in for P); without it every CTA takes tiles of any slot */
+  MOE_FFN_STRICT_SLOTS = 2,  /* flag: execution unit u (an SM pair, or an SM) only runs
+                                slot (u mod P)'s tiles, so the layer time follows the
+                                plan's makespan (one GPU standing in for P); without it
+                                every unit takes tiles of any slot */
+  MOE_FFN_SM_PAIR = 4        /* flag: run each tile on a pair of SMs (a cluster of two
+                                CTAs, tcgen05 cta_group::2, M = 256) instead of each
+                                128-row half on one SM (cta_group::1, the default) */
 };
 
 /* Upper bounds: which = MOE_WS_ROWS -> R_max rows (Xp, A, O, row_token, row_gate);
@@ -140,9 +144,10 @@ MOE_API int moe_route_hist(const moe_cfg* cfg, const float* logits, int32_t* top
  *   blocks       int32 [B_max, 2]: (e, j) pairs; slot r's run is
  *                [slot_off[r], slot_off[r+1]), experts ascending, expert e's share being
  *                block indices j in [sum_{r'<r} q[e, r'], + q[e, r]).
- *   tiles        int32 [B_max, 4]: 128-row execution tiles (e, first padded row, rows in
- *                the tile (64 or 128), slot) in the same slot/expert order; with beta = 64
- *                two consecutive blocks of one expert's run share a tile.
+ *   tiles        int32 [B_max, 4]: execution tiles of the FFN (e, first padded row, rows
+ *                in the tile, slot): each slot's run of expert e (q[e, r] consecutive
+ *                blocks) cut into tiles of 256 rows (the last may be shorter), in the same
+ *                slot/expert order.
  *   plan_info    int32 [MOE_PI_LEN]: see MOE_PI_*.
  * The owner of expert e is slot h(e) = floor(e * P / E).  The plan is deterministic and
  * bit-identical across calls.  Runs on one CTA. */
@@ -179,9 +184,11 @@ MOE_API int moe_dispatch_permute(const moe_cfg* cfg, const uint16_t* x, const in
  *              y[row_token[r]] += row_gate[r] * O[r] for every valid row (fp32 atomic
  *              adds: the summation order, and so the last bits, may vary run to run).
  *              MOE_FFN_WRITE_O: O bf16 [R_max, d] (rows of the plan's tiles).
- *   mode       MOE_FFN_FUSED_COMBINE or MOE_FFN_WRITE_O, optionally | MOE_FFN_STRICT_SLOTS.
- * Two persistent kernels (FC1+SwiGLU, then FC2) of one CTA per SM; every wait inside them
- * is bounded and sets MOE_STATUS_TIMEOUT instead of hanging. */
+ *   mode       MOE_FFN_FUSED_COMBINE or MOE_FFN_WRITE_O, optionally | MOE_FFN_STRICT_SLOTS
+ *              and | MOE_FFN_SM_PAIR.
+ * Two persistent kernels (FC1+SwiGLU, then FC2) of one CTA per SM (in clusters of two
+ * CTAs with MOE_FFN_SM_PAIR); every wait inside them is bounded and sets
+ * MOE_STATUS_TIMEOUT instead of hanging. */
 MOE_API int moe_expert_ffn(const moe_cfg* cfg, const uint16_t* xp, const uint16_t* w1,
                    const uint16_t* w2, const int32_t* tiles, const int32_t* plan_info,
                    const int32_t* row_token, const float* row_gate, int mode,

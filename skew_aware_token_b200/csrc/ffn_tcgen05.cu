@@ -4,31 +4,45 @@
 //   Z_e = X_e W1_e,  Z_e = [G_e, U_e],  A_e = SiLU(G_e) * U_e,  O_e = A_e W2_e,
 //   y_t = sum_{e in S_t} p_{t,e} O_e[t].
 // The pages' forward megakernel runs FC1, then FC2 on each token block ("Executor:
-// Pipelined Expert Replication", Forward); here the blocks are the planner's 128-row tiles
-// and the two GEMMs are two persistent launches over the same tile list.
+// Pipelined Expert Replication", Forward); here the blocks are grouped into the planner's
+// execution tiles (up to 256 rows of one expert) and the two GEMMs are two persistent
+// launches over the same tile list.
 //
-// Kernel shape (one CTA per SM, 192 threads, persistent over (m-tile, n-tile) work items):
-//   warp 0      TMA producer: A tile [128 x 64] and B tile [256 x 64] bf16 per K step into
-//               a 4-stage shared-memory ring (128-byte swizzle), one mbarrier per stage.
-//   warp 1      MMA issuer: one thread issues tcgen05.mma.cta_group::1.kind::f16 (M=128,
-//               N=256, K=16 x 4 per stage) into a TMEM accumulator; tcgen05.commit frees
-//               the smem stage and, after the last K step, hands the accumulator over.
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (each warp reads its own 32
-//               TMEM lanes = 32 rows), then
-//                 FC1: A = SiLU(G) * U rounded to bf16 -> a_scratch (the B tile stacks
-//                      128 rows of W1_e's G half over the matching 128 rows of its U half,
-//                      so G and U of the same output column sit 128 TMEM columns apart);
-//                 FC2: y[row_token] += row_gate * O with 16-byte fp32 vector reductions
-//                      (fused combine), or O rounded to bf16 (unfused path).
-//   TMEM holds two 256-column accumulators (512 columns), so the epilogue of one work item
+// Two variants of one kernel template:
+//   single SM (default): one CTA runs one 128-row half of a tile with
+//     tcgen05.mma.cta_group::1 (M=128, N=256).
+//   SM pair (MOE_FFN_SM_PAIR): a cluster of two CTAs on two SMs runs one 256-row tile.  Each CTA
+//     loads its own 128 rows of the A tile and half of the B tile (128 of its 256 rows)
+//     into its shared memory; CTA 0 issues tcgen05.mma.cta_group::2 (M=256, N=256), whose
+//     accumulator lands in both CTAs' TMEM (each CTA: its 128 rows x 256 columns).  Each SM
+//     therefore moves 32 KB per K step instead of 48 KB, and six stages fit where four did;
+//     but a tile whose second half is empty still costs a full pair MMA.  On the MoE
+//     workloads measured here the single-SM variant is as fast or faster (the pair wins on
+//     long dense tiles), hence the default.
+// Roles in every CTA (192 threads, one CTA per SM, persistent):
+//   warp 0      TMA producer: A [128 x 64] and B [128 or 256 x 64] bf16 tiles per K step
+//               into a ring of shared-memory stages (128-byte swizzle).  In a pair, both
+//               CTAs' copies signal CTA 0's stage barrier.
+//   warp 1      MMA issuer (CTA 0 of a pair): one thread issues the MMAs of a stage into a
+//               TMEM accumulator; tcgen05.commit frees the stage (in both CTAs of a pair)
+//               and, after the last K step, hands the accumulator to the epilogue.
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (warp w reads TMEM lanes
+//               32*(w%4)..+31, i.e. 32 rows), then
+//                 FC1: A = SiLU(G) * U rounded to bf16 -> scratch (the B tile stacks 128 rows
+//                      of W1_e's G half over the matching 128 rows of its U half, so G and U
+//                      of an output column sit 128 accumulator columns apart);
+//                 FC2: y[row_token] += row_gate * O (fused combine): each 32 x 32 chunk is
+//                      transposed through shared memory so that one 16-byte vector reduction
+//                      instruction covers four whole 128-byte row segments; or O rounded to
+//                      bf16 (unfused path).
+//   TMEM holds two 256-column accumulators (512 columns): the epilogue of one work item
 //   overlaps the MMAs of the next.
-// Work items: item L -> m-tile L / n_n, n-tile L % n_n, handed out in increasing L by a
-// global atomic counter (the producer thread draws the next item when it is ready for
-// it, so faster SMs take more items) and passed to the MMA and epilogue warps through a
-// small shared-memory ring.  All n-tiles of a block are in flight together, and
-// consecutive blocks belong to the same expert, so each expert's weights stream from HBM
-// about once.  With MOE_FFN_STRICT_SLOTS, CTA c draws from slot (c mod P)'s counter and
-// only runs that slot's tiles.
+// Work items (tile, n-tile) are handed out in increasing order by a global atomic counter
+// (the producer draws the next item when it is ready for it, so fast SMs take more) and
+// passed to the other roles, and in a pair to the other CTA, through a small ring in
+// shared memory.  All n-tiles of a tile are in flight together and consecutive tiles
+// belong to the same expert, so each expert's weights stream from HBM about once.  With
+// MOE_FFN_STRICT_SLOTS, unit u (a CTA, or a pair) draws from slot (u mod P)'s counter.
 // Every mbarrier wait is bounded (globaltimer); on expiry the kernel sets
 // MOE_STATUS_TIMEOUT, lets the other roles drop out, waits (bounded) for its own copies
 // and MMAs in flight, frees its TMEM and returns.
@@ -43,26 +57,41 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;   // rows per tile (M)
+constexpr int BM = 128;   // A rows per CTA = TMEM lanes
 constexpr int BK = 64;    // K per stage: 64 bf16 = 128 bytes = one swizzle span
 constexpr int BN = 256;   // MMA N (FC1: 128 G + 128 U columns; FC2: 256 output columns)
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int RING = 8;   // work items in flight between the producer and the consumers
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512;  // + alignment slack, barriers
+constexpr int RING = 8;                 // work items in flight between roles
+constexpr int STG_STRIDE = 36;          // floats per staged row of the FC2 combine
+constexpr int STG_BYTES = 4 * 32 * STG_STRIDE * 4;
+constexpr int META_BYTES = 2048;        // barriers, ring, per-row tokens
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per wait
 
-// kind::f16 instruction descriptor: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 = 1),
-// B bf16 (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bit 17, M >> 4 at 24.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+template <int PHASE, bool PAIR>
+struct Geo {
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // B rows held by one CTA
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int TX_BYTES = PAIR ? 2 * STAGE_BYTES : STAGE_BYTES;  // per stage
+  static constexpr int M = PAIR ? 2 * BM : BM;
+  // kind::f16 instruction descriptor: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 = 1),
+  // B bf16 (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bit 17, M >> 4 at 24.
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
+                                    ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+  static constexpr int NBARS = 2 * STAGES + 5 + 2 * RING;
+  static constexpr int STG = PHASE == 2 ? STG_BYTES : 0;  // FC2 combine staging
+  static constexpr int SMEM = STAGES * STAGE_BYTES + STG + META_BYTES + 1024;
+};
+static_assert(Geo<1, true>::SMEM <= 227 * 1024 && Geo<2, true>::SMEM <= 227 * 1024 &&
+                  Geo<1, false>::SMEM <= 227 * 1024 && Geo<2, false>::SMEM <= 227 * 1024,
+              "smem");
+static_assert(Geo<1, true>::NBARS * 8 + 4 * (2 + RING) + 4 * 128 <= META_BYTES, "meta");
 
 struct FfnArgs {
-  int32_t* sched;           // this launch's counters: [0] or [slot] (strict), zeroed
+  int32_t* sched;           // this launch's counters: [0], or [slot] (strict); zeroed
   const int32_t* tiles;
   const int32_t* plan_info;
   const int32_t* row_token;
@@ -72,7 +101,7 @@ struct FfnArgs {
   long long r_max;
   int T, d, f, E, P;
   int n_k;       // K steps of 64
-  int n_n;       // n-tiles per m-tile
+  int n_n;       // n-tiles per tile
   int out_ld;    // output row length (elements)
   int write_o;   // FC2: store O (1) or fused combine (0)
   int strict;
@@ -82,6 +111,21 @@ struct FfnArgs {
 // ------------------------------------------------------------------ PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
@@ -93,10 +137,18 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// arrive on a barrier in another CTA of the cluster (cluster-mapped address)
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+__device__ __forceinline__ void st_remote_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; "
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; "
       "selp.u32 %0, 1, 0, p; }"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -134,6 +186,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(map), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+// Copy into this CTA's shared memory whose completion is counted on the barrier of the
+// pair's first CTA (cluster-mapped address `bar`).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -145,17 +207,72 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) |
          (1ull << 46) | (2ull << 61);
 }
+template <bool PAIR>
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                           uint32_t accumulate) {
-  asm volatile(
-      "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(kIdesc), "r"(accumulate));
+  if constexpr (PAIR) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(Geo<1, true>::IDESC), "r"(accumulate));
+  } else {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(Geo<1, false>::IDESC), "r"(accumulate));
+  }
 }
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-      : "memory");
+// Arrive on `bar` (same offset in both CTAs of a pair) once this thread's MMAs complete.
+template <bool PAIR>
+__device__ __forceinline__ void umma_commit_all(uint32_t bar) {
+  if constexpr (PAIR) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster"
+        ".b64 [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)3)
+        : "memory");
+  } else {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+  }
+}
+// Arrive on this CTA's `bar` once this thread's MMAs complete.
+template <bool PAIR>
+__device__ __forceinline__ void umma_commit_local(uint32_t bar) {
+  if constexpr (PAIR) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+  } else {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+  }
+}
+template <bool PAIR>
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_addr) {
+  if constexpr (PAIR) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     slot_addr),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  } else {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     slot_addr),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+}
+template <bool PAIR>
+__device__ __forceinline__ void tmem_dealloc(uint32_t base) {
+  if constexpr (PAIR) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(base),
+                 "r"(TMEM_COLS));
+  } else {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(base),
+                 "r"(TMEM_COLS));
+  }
 }
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -179,9 +296,9 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
+__device__ __forceinline__ void red_add_v4(float* addr, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w)
                : "memory");
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -191,87 +308,105 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
 
 // ------------------------------------------------------------------ work schedule
+// Item L of a unit's range -> tile m, n-tile n and (single SM) the tile half.
 struct Sched {
-  int32_t* counter;   // global counter this CTA draws items from
-  long long total;    // items in its range
-  int m_base, n_n;
-  __device__ void decode(int L, int& m, int& n) const {
-    m = m_base + L / n_n;
+  int32_t* counter;  // global counter this unit draws items from
+  long long total;   // items in its range
+  int m_base, n_n, halves;
+  __device__ void decode(int L, int& m, int& n, int& half) const {
     n = L % n_n;
+    const int t = L / n_n;
+    m = m_base + t / halves;
+    half = t % halves;
   }
 };
 
+template <bool PAIR>
 __device__ Sched make_sched(const FfnArgs& a) {
   Sched s;
   s.n_n = a.n_n;
+  s.halves = PAIR ? 1 : 2;
+  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int* pi = a.plan_info;
   if (!a.strict) {
     s.counter = a.sched;
-    s.total = (long long)max(pi[MOE_PI_NTILES], 0) * a.n_n;
+    s.total = (long long)max(pi[MOE_PI_NTILES], 0) * a.n_n * s.halves;
     s.m_base = 0;
   } else {
-    const int r = blockIdx.x % a.P;
+    const int r = unit % a.P;
     const int lo = pi[MOE_PI_SLOT_TILE_OFF + r], hi = pi[MOE_PI_SLOT_TILE_OFF + r + 1];
     s.counter = a.sched + r;
-    s.total = (long long)max(hi - lo, 0) * a.n_n;
+    s.total = (long long)max(hi - lo, 0) * a.n_n * s.halves;
     s.m_base = lo;
   }
   return s;
 }
 
 struct TileInfo {
-  int e, row0, nrows;
-  bool ok;
+  int e, row0, nrows;  // row0 / nrows of this CTA's 128-row half
+  int a_row;           // A rows this CTA loads (moved inside the buffer when empty)
+  bool ok;             // a well-formed tile (all roles of both CTAs agree)
+  bool run;            // this work item is executed (single SM: its half has rows)
 };
-__device__ __forceinline__ TileInfo read_tile(const FfnArgs& a, int m) {
+template <bool PAIR>
+__device__ __forceinline__ TileInfo read_tile(const FfnArgs& a, int m, int half) {
   TileInfo t;
   const int4 v = __ldg(reinterpret_cast<const int4*>(a.tiles) + m);
   t.e = v.x;
-  t.row0 = v.y;
-  t.nrows = v.z;
-  t.ok = v.x >= 0 && v.x < a.E && v.y >= 0 && (long long)v.y < a.r_max && v.z > 0 && v.z <= BM;
+  t.ok = v.x >= 0 && v.x < a.E && v.y >= 0 && (long long)v.y < a.r_max && v.z > 0 &&
+         v.z <= 2 * BM;
+  t.row0 = v.y + BM * half;
+  t.nrows = v.z - BM * half;
+  t.run = t.ok && (PAIR || t.nrows > 0);
+  t.a_row = t.nrows > 0 ? t.row0 : (int)max(a.r_max - BM, 0LL);
   return t;
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int PHASE>  // 1: FC1 + SwiGLU, 2: FC2 (+ combine)
+template <int PHASE, bool PAIR>  // PHASE 1: FC1 + SwiGLU, 2: FC2 (+ combine)
 __global__ void __launch_bounds__(THREADS, 1)
 ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const FfnArgs a) {
+  using G = Geo<PHASE, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  // bars: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain,
-  //       item_full[RING], item_empty[RING]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5 + 2 * RING);
+  float* stg = reinterpret_cast<float*>(smem + G::STAGES * G::STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G::STAGES * G::STAGE_BYTES + G::STG);
+  // bars: full[S], empty[S], tmem_full[2], tmem_empty[2], drain, item_full[R], item_empty[R]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + G::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [RING] items
+  int* s_tok = reinterpret_cast<int*>(tmem_slot + 2 + RING);           // [4][32] tokens
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool mma_cta = rank == 0;  // single SM: always; pair: CTA 0 issues the MMAs
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
-  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
-  auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + b); };
-  auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 + b); };
-  const uint32_t drain_bar = smem_u32(bars + 2 * STAGES + 4);
-  auto ifull_bar = [&](int i) { return smem_u32(bars + 2 * STAGES + 5 + i); };
-  auto iempty_bar = [&](int i) { return smem_u32(bars + 2 * STAGES + 5 + RING + i); };
-  auto sA = [&](int s) { return smem_u32(smem + s * STAGE_BYTES); };
-  auto sB = [&](int s) { return smem_u32(smem + s * STAGE_BYTES + A_BYTES); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + G::STAGES + s); };
+  auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * G::STAGES + b); };
+  auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * G::STAGES + 2 + b); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * G::STAGES + 4);
+  auto ifull_bar = [&](int i) { return smem_u32(bars + 2 * G::STAGES + 5 + i); };
+  auto iempty_bar = [&](int i) { return smem_u32(bars + 2 * G::STAGES + 5 + RING + i); };
+  auto sA = [&](int s) { return smem_u32(smem + s * G::STAGE_BYTES); };
+  auto sB = [&](int s) { return smem_u32(smem + s * G::STAGE_BYTES + A_BYTES); };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+    for (int s = 0; s < G::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);   // the MMA CTA's producer (expect_tx)
+      mbar_init(empty_bar(s), 1);  // the MMA thread's commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 4 * 32);
+      mbar_init(tempty_bar(b), PAIR ? 8 : 4);  // every epilogue warp (of both CTAs)
     }
     mbar_init(drain_bar, 1);
     for (int i = 0; i < RING; ++i) {
       mbar_init(ifull_bar(i), 1);
-      mbar_init(iempty_bar(i), 1 + 4);  // the MMA thread and the four epilogue warps
+      // consumers of an item: MMA thread + 4 epilogue warps (+ the other CTA's producer
+      // and 4 epilogue warps)
+      mbar_init(iempty_bar(i), PAIR ? 10 : 5);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -279,17 +414,12 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
+  if (warp == 1) tmem_alloc<PAIR>(smem_u32(tmem_slot));
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const Sched sch = make_sched(a);
+  const Sched sch = make_sched<PAIR>(a);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -301,47 +431,67 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       for (int it = 0;; ++it) {
         const int slot = it % RING;
         const uint32_t ph = (uint32_t)(it / RING) & 1u;
-        if (!mbar_wait(iempty_bar(slot), ph ^ 1u, abort_flag, a.status, a.timeout_ns, true))
-          break;
-        const long long L = atomicAdd(sch.counter, 1);
-        ring[slot] = L < sch.total ? (int)L : -1;
-        mbar_arrive(ifull_bar(slot));
-        if (L >= sch.total) break;
-        int m, n;
-        sch.decode((int)L, m, n);
-        const TileInfo ti = read_tile(a, m);
-        if (!ti.ok) {
-          bad_tile = true;
-          continue;
+        int L;
+        if (mma_cta) {
+          if (!mbar_wait(iempty_bar(slot), ph ^ 1u, abort_flag, a.status, a.timeout_ns, true))
+            break;
+          const long long v = atomicAdd(sch.counter, 1);
+          L = v < sch.total ? (int)v : -1;
+          ring[slot] = L;
+          if constexpr (PAIR) {
+            st_remote_u32(mapa(smem_u32((const void*)(ring + slot)), 1), (uint32_t)L);
+            mbar_arrive_remote(mapa(ifull_bar(slot), 1));
+          }
+          mbar_arrive(ifull_bar(slot));
+        } else {
+          if (!mbar_wait(ifull_bar(slot), ph, abort_flag, a.status, a.timeout_ns, true)) break;
+          L = ring[slot];
+          mbar_arrive_remote(mapa(iempty_bar(slot), 0));
         }
-        const int brow = PHASE == 1 ? ti.e * 2 * a.f + n * (BN / 2) : ti.e * a.d + n * BN;
+        if (L < 0) break;
+        int m, n, half;
+        sch.decode(L, m, n, half);
+        const TileInfo ti = read_tile<PAIR>(a, m, PAIR ? (int)rank : half);
+        if (!ti.ok) bad_tile = true;
+        if (!ti.run) continue;
+        int brow;
+        if (PHASE == 1) brow = ti.e * 2 * a.f + n * (BN / 2) + (PAIR ? (int)rank * a.f : 0);
+        else brow = ti.e * a.d + n * BN + (PAIR ? (int)rank * (BN / 2) : 0);
         bool stop = false;
         for (int kb = 0; kb < a.n_k; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status, a.timeout_ns, true)) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status, a.timeout_ns,
+                         true)) {
             stop = true;
             break;
           }
-          mbar_expect_tx(full_bar(stage), STAGE_BYTES);
-          tma_load_2d(sA(stage), &tmA, full_bar(stage), kb * BK, ti.row0);
-          if (PHASE == 1) {
-            tma_load_2d(sB(stage), &tmB, full_bar(stage), kb * BK, brow);
-            tma_load_2d(sB(stage) + B_BYTES / 2, &tmB, full_bar(stage), kb * BK, brow + a.f);
+          if (mma_cta) mbar_expect_tx(full_bar(stage), G::TX_BYTES);
+          if constexpr (PAIR) {
+            const uint32_t fb = mapa(full_bar(stage), 0);
+            tma_load_2d_pair(sA(stage), &tmA, fb, kb * BK, ti.a_row);
+            tma_load_2d_pair(sB(stage), &tmB, fb, kb * BK, brow);
           } else {
-            tma_load_2d(sB(stage), &tmB, full_bar(stage), kb * BK, brow);
+            tma_load_2d(sA(stage), &tmA, full_bar(stage), kb * BK, ti.a_row);
+            if (PHASE == 1) {
+              tma_load_2d(sB(stage), &tmB, full_bar(stage), kb * BK, brow);
+              tma_load_2d(sB(stage) + G::B_BYTES / 2, &tmB, full_bar(stage), kb * BK,
+                          brow + a.f);
+            } else {
+              tma_load_2d(sB(stage), &tmB, full_bar(stage), kb * BK, brow);
+            }
           }
           pending |= 1u << stage;
           pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == G::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (stop) break;
       }
-      if (bad_tile) set_status(a.status, MOE_STATUS_PLAN);
-      if (*abort_flag) {
-        // let the copies already issued land before the CTA's shared memory goes away
-        for (int s = 0; s < STAGES; ++s)
+      if (bad_tile && mma_cta) set_status(a.status, MOE_STATUS_PLAN);
+      if (*abort_flag && mma_cta) {
+        // let the copies already armed land before shared memory goes away
+        for (int s = 0; s < G::STAGES; ++s)
           if (pending >> s & 1u)
             mbar_wait(full_bar(s), pend_parity >> s & 1u, abort_flag, a.status, a.timeout_ns,
                       false);
@@ -349,7 +499,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && mma_cta) {
       int stage = 0;
       uint32_t phase = 0;
       int acc_it = 0;
@@ -361,13 +511,14 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         const int L = ring[slot];
         mbar_arrive(iempty_bar(slot));
         if (L < 0) break;
-        int m, n;
-        sch.decode(L, m, n);
-        const TileInfo ti = read_tile(a, m);
-        if (!ti.ok) continue;
+        int m, n, half;
+        sch.decode(L, m, n, half);
+        const TileInfo ti = read_tile<PAIR>(a, m, PAIR ? 0 : half);
+        if (!ti.run) continue;
         const int buf = acc_it & 1;
         const uint32_t use = (uint32_t)(acc_it >> 1) & 1u;
-        if (!mbar_wait(tempty_bar(buf), use ^ 1u, abort_flag, a.status, a.timeout_ns, true)) break;
+        if (!mbar_wait(tempty_bar(buf), use ^ 1u, abort_flag, a.status, a.timeout_ns, true))
+          break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
         bool stop = false;
@@ -379,31 +530,31 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
           tc_fence_after();
           const uint32_t a0 = sA(stage), b0 = sB(stage);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            umma_bf16(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32),
-                      (kb | kk) != 0);
-          }
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16<PAIR>(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32),
+                            (kb | kk) != 0);
           issued = true;
-          umma_commit(empty_bar(stage));
-          if (++stage == STAGES) {
+          umma_commit_all<PAIR>(empty_bar(stage));
+          if (++stage == G::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (stop) break;
-        umma_commit(tfull_bar(buf));
+        umma_commit_all<PAIR>(tfull_bar(buf));
         ++acc_it;
       }
       if (issued) {
         // every MMA this thread issued has completed once the drain barrier fires
-        umma_commit(drain_bar);
+        umma_commit_local<PAIR>(drain_bar);
         mbar_wait(drain_bar, 0, abort_flag, a.status, a.timeout_ns, false);
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..5)
-    const int quarter = warp & 3;  // TMEM lanes this warp may read: 32*quarter ..
-    const int rit = quarter * 32 + lane;  // row inside the tile
+    const int quarter = warp & 3;         // TMEM lanes this warp may read: 32*quarter ..
+    const int rit = quarter * 32 + lane;  // row inside this CTA's half
+    const int ew = warp - 2;              // staging slot of this warp
     int acc_it = 0;
     for (int it = 0;; ++it) {
       const int slot = it % RING;
@@ -413,12 +564,15 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       if (!__all_sync(0xffffffffu, have)) break;
       const int L = ring[slot];
       __syncwarp();
-      if (lane == 0) mbar_arrive(iempty_bar(slot));
+      if (lane == 0) {
+        if (mma_cta) mbar_arrive(iempty_bar(slot));
+        else mbar_arrive_remote(mapa(iempty_bar(slot), 0));
+      }
       if (L < 0) break;
-      int m, n;
-      sch.decode(L, m, n);
-      const TileInfo ti = read_tile(a, m);
-      if (!ti.ok) continue;
+      int m, n, half;
+      sch.decode(L, m, n, half);
+      const TileInfo ti = read_tile<PAIR>(a, m, PAIR ? (int)rank : half);
+      if (!ti.run) continue;
       const int buf = acc_it & 1;
       const uint32_t use = (uint32_t)(acc_it >> 1) & 1u;
       const bool got =
@@ -469,6 +623,8 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
           }
         }
       } else {
+        // fused combine: y[token] += gate * O, staged per 32 x 32 chunk so that lanes
+        // 8q..8q+7 of one reduction cover a whole 128-byte segment of one row
         int tok = -1;
         float gate = 0.f;
         if (valid) {
@@ -476,35 +632,49 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
           gate = __ldg(a.row_gate + row);
           if (tok >= a.T) tok = -1;
         }
-        float* y = reinterpret_cast<float*>(a.out) + (long long)(tok < 0 ? 0 : tok) * a.out_ld +
-                   n * BN;
+        s_tok[ew * 32 + lane] = tok;
+        float* my_row = stg + (ew * 32 + lane) * STG_STRIDE;
+        float* y = reinterpret_cast<float*>(a.out) + n * BN + 4 * (lane & 7);
+        __syncwarp();
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(taddr + c * 32, v);
           tmem_wait_ld();
-          if (tok >= 0) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              red_add_v4(y + c * 32 + 4 * i, gate * __uint_as_float(v[4 * i]),
-                         gate * __uint_as_float(v[4 * i + 1]),
-                         gate * __uint_as_float(v[4 * i + 2]),
-                         gate * __uint_as_float(v[4 * i + 3]));
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4*>(my_row + 4 * j) = make_float4(
+                gate * __uint_as_float(v[4 * j]), gate * __uint_as_float(v[4 * j + 1]),
+                gate * __uint_as_float(v[4 * j + 2]), gate * __uint_as_float(v[4 * j + 3]));
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + (lane >> 3);
+            const int tk = s_tok[ew * 32 + r];
+            if (tk >= 0) {
+              const float4 x = *reinterpret_cast<const float4*>(
+                  stg + (ew * 32 + r) * STG_STRIDE + 4 * (lane & 7));
+              red_add_v4(y + (long long)tk * a.out_ld + c * 32, x);
+            }
           }
+          __syncwarp();
         }
       }
       tc_fence_before();
-      mbar_arrive(tempty_bar(buf));
+      __syncwarp();
+      if (lane == 0) {
+        if (mma_cta) mbar_arrive(tempty_bar(buf));
+        else mbar_arrive_remote(mapa(tempty_bar(buf), 0));
+      }
       ++acc_it;
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(TMEM_COLS));
+    tmem_dealloc<PAIR>(tmem_base);
   }
 }
 
@@ -538,6 +708,41 @@ bool encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t oute
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int PHASE, bool PAIR>
+cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const FfnArgs& args,
+                       cudaStream_t st) {
+  auto kern = ffn_kernel<PHASE, PAIR>;
+  cudaError_t err =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Geo<PHASE, PAIR>::SMEM);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = Geo<PHASE, PAIR>::SMEM;
+  cfg.stream = st;
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(2);
+    int clusters = 0;
+    err = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+    if (err != cudaSuccess) return err;
+    if (clusters < 1) return cudaErrorInvalidConfiguration;
+    cfg.gridDim = dim3(2 * clusters);
+  } else {
+    cfg.gridDim = dim3(num_sms());
+  }
+  FfnArgs a = args;
+  const int units = PAIR ? (int)cfg.gridDim.x / 2 : (int)cfg.gridDim.x;
+  a.strict = a.strict && units >= a.P;
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, a);
+}
+
 }  // namespace
 
 cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
@@ -545,6 +750,7 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
                        const int32_t* row_token, const float* row_gate, int mode,
                        uint16_t* a_scratch, void* out, int32_t* status, cudaStream_t st) {
   const bool write_o = (mode & MOE_FFN_WRITE_O) != 0;
+  const bool pair = (mode & MOE_FFN_SM_PAIR) != 0;
   const long long r_max = max_rows(c);
   cudaError_t err;
   if (!write_o && c.T > 0) {
@@ -552,7 +758,6 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
     if (err != cudaSuccess) return err;
   }
   if (r_max == 0) return cudaSuccess;
-
   // scheduler counters after A in the scratch buffer: [0, 8) FC1, [8, 16) FC2
   int32_t* sched = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(a_scratch) +
                                               ffn_a_bytes(c));
@@ -563,17 +768,9 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   if (!encode_2d(&tm_xp, xp, c.d, r_max, BM) ||
       !encode_2d(&tm_w1, w1, c.d, (uint64_t)c.E * 2 * c.f, BN / 2) ||
       !encode_2d(&tm_a, a_scratch, c.f, r_max, BM) ||
-      !encode_2d(&tm_w2, w2, c.f, (uint64_t)c.E * c.d, BN))
+      !encode_2d(&tm_w2, w2, c.f, (uint64_t)c.E * c.d, pair ? BN / 2 : BN))
     return cudaErrorInvalidValue;
 
-  err = cudaFuncSetAttribute(ffn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES);
-  if (err != cudaSuccess) return err;
-  err = cudaFuncSetAttribute(ffn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES);
-  if (err != cudaSuccess) return err;
-
-  const int grid = num_sms();
   FfnArgs a1{};
   a1.tiles = tiles;
   a1.plan_info = plan_info;
@@ -586,28 +783,28 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   a1.f = c.f;
   a1.E = c.E;
   a1.P = c.P;
-  a1.strict = (mode & MOE_FFN_STRICT_SLOTS) && grid >= c.P;
+  a1.strict = (mode & MOE_FFN_STRICT_SLOTS) != 0;
   a1.timeout_ns = kTimeoutNs;
 
   FfnArgs a2 = a1;
   a1.sched = sched;
-  a2.sched = sched + 8;
   a1.out = a_scratch;
   a1.n_k = c.d / BK;
   a1.n_n = c.f / (BN / 2);
   a1.out_ld = c.f;
   a1.write_o = 0;
-  ffn_kernel<1><<<grid, THREADS, SMEM_BYTES, st>>>(tm_xp, tm_w1, a1);
-  err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-
+  a2.sched = sched + 8;
   a2.out = out;
   a2.n_k = c.f / BK;
   a2.n_n = c.d / BN;
   a2.out_ld = c.d;
   a2.write_o = write_o;
-  ffn_kernel<2><<<grid, THREADS, SMEM_BYTES, st>>>(tm_a, tm_w2, a2);
-  return cudaGetLastError();
+
+  err = pair ? launch_one<1, true>(tm_xp, tm_w1, a1, st)
+             : launch_one<1, false>(tm_xp, tm_w1, a1, st);
+  if (err != cudaSuccess) return err;
+  return pair ? launch_one<2, true>(tm_a, tm_w2, a2, st)
+              : launch_one<2, false>(tm_a, tm_w2, a2, st);
 }
 
 }  // namespace moe

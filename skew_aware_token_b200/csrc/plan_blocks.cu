@@ -31,6 +31,7 @@ namespace moe {
 namespace {
 
 constexpr int kPlanThreads = 128;  // 4 warps = 4 greedy variants
+constexpr int kTileRows = 256;     // rows of one execution tile of the FFN
 constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ int home_lo(int r, int E, int P) { return (r * E + P - 1) / P; }
@@ -267,7 +268,7 @@ plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
     int nt = 0;
     for (int e = 0; e < E; ++e) {
       const int qer = qb[e * P + r];
-      nt += beta == 128 ? qer : (qer + 1) / 2;
+      nt += (qer * beta + kTileRows - 1) / kTileRows;
     }
     misc[3 + r] = nt;  // temporarily the count
     int fixed = 0;
@@ -319,7 +320,7 @@ plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
     for (int e = e0; e < e1; ++e) {
       const int qer = qb[e * P + r];
       nb += qer;
-      nt += beta == 128 ? qer : (qer + 1) / 2;
+      nt += (qer * beta + kTileRows - 1) / kTileRows;
     }
     int pb = misc[12 + r] + warp_excl_scan(nb, lane);
     int pt = misc[3 + r] + warp_excl_scan(nt, lane);
@@ -333,12 +334,12 @@ plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
           blocks[2 * pb + 1] = j0 + i;
         }
       }
-      const int per = beta == 128 ? 1 : 2;
-      for (int i = 0; i < qer; i += per, ++pt) {
+      const int rows = qer * beta;
+      for (int i = 0; i < rows; i += kTileRows, ++pt) {
         if (pt < b_max) {
           tiles[4 * pt + 0] = e;
-          tiles[4 * pt + 1] = beta * (boff[e] + j0 + i);
-          tiles[4 * pt + 2] = (i + per <= qer) ? 128 : beta;
+          tiles[4 * pt + 1] = beta * (boff[e] + j0) + i;
+          tiles[4 * pt + 2] = min(kTileRows, rows - i);
           tiles[4 * pt + 3] = r;
         }
       }

@@ -29,19 +29,18 @@ def host_inputs(wl):
 
 
 def expected_tiles(q, block_off, beta):
-    """The executor's 128-row tiles: per slot, experts ascending, each run of q[e][r]
-    blocks cut into tiles of 128 rows (two 64-row blocks share a tile)."""
+    """The executor's tiles: per slot, experts ascending, each run of q[e][r] blocks
+    (q[e][r] * beta consecutive rows) cut into tiles of 256 rows, the last possibly
+    shorter."""
     q = np.asarray(q)
     E, P = q.shape
-    per = 128 // beta
     tiles, slot_tile_off = [], [0]
     for r in range(P):
         for e in range(E):
             j0 = int(q[e, :r].sum())
-            qer = int(q[e, r])
-            for i in range(0, qer, per):
-                nrows = 128 if i + per <= qer else beta
-                tiles.append((e, beta * (block_off[e] + j0 + i), nrows, r))
+            rows = int(q[e, r]) * beta
+            for i in range(0, rows, 256):
+                tiles.append((e, beta * (block_off[e] + j0) + i, min(256, rows - i), r))
         slot_tile_off.append(len(tiles))
     return tiles, slot_tile_off
 

@@ -27,7 +27,9 @@ FULL_CASES = [
 ]
 MODES = [N.MOE_FFN_FUSED_COMBINE, N.MOE_FFN_WRITE_O,
          N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_STRICT_SLOTS,
-         N.MOE_FFN_WRITE_O | N.MOE_FFN_STRICT_SLOTS]
+         N.MOE_FFN_WRITE_O | N.MOE_FFN_STRICT_SLOTS,
+         N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_SM_PAIR,
+         N.MOE_FFN_WRITE_O | N.MOE_FFN_SM_PAIR | N.MOE_FFN_STRICT_SLOTS]
 
 
 def _oracle_full(wl, w1, w2):
