@@ -285,15 +285,17 @@ def run_ours(args, wl, world, rank, local):
     tflops = wl.flops * args.steps * world / elapsed / 1e12
     ffn_s = stage_ms["ffn"] / 1e3
     ffn_tflops = wl.flops / ffn_s / 1e12
-    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    # the FFN runs inside a long loop of back-to-back steps: the sustained peak applies
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     weight_bytes = 6 * wl.d * wl.f * sum(1 for c in layer.view("counts").cpu().tolist() if c)
     roofline = {"bound": "tensor", "kernel": "expert FFN (FC1+SwiGLU, FC2+combine)",
                 "achieved": round(ffn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(ffn_tflops / peak, 4), "peak_source": f"bf16 burst {peak_src}",
+                "frac": round(ffn_tflops / peak, 4),
+                "peak_source": f"bf16 sustained {peak_src} (timed inside a long step loop)",
                 "traffic": None, "flops_per_launch": wl.flops,
                 "ms_per_launch": round(stage_ms["ffn"], 4),
-                "frac_of_sustained": round(ffn_tflops / peaks.get(
-                    "bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]), 4)}
+                "frac_of_burst": round(ffn_tflops / burst, 4)}
     traffic_path = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(traffic_path):
         with open(traffic_path) as fh:

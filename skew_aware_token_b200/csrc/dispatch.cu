@@ -7,26 +7,30 @@
 // preserved (every pair lands on exactly one row, with its own gate).
 //
 // Pass 1 (rank): one CTA per expert scans the flattened topk_ids in pair order
-// i = t*k + j, four ids per thread (16-byte loads), and ranks its matches with a
-// warp-shuffle scan plus a CTA scan of the 32 warp totals; the running total carries the
-// order across chunks, so ranks follow the pair order (stable).  It writes row_token,
+// i = t*k + j, sixteen consecutive ids per thread per pass (16-byte loads), and ranks its
+// matches with a warp-shuffle scan plus a CTA scan of the 32 warp totals; the running
+// total carries the order across passes, so ranks follow the pair order (stable).  It writes row_token,
 // row_gate and tok_row, then marks the expert's padding rows.
 // Pass 2 (gather): one warp per padded row copies x[row_token] (or zeros) with 16-byte
-// vector loads and stores; the grid strides over the rows of the plan (read on device).
+// vector loads (eight in flight per lane) and stores; the grid strides over the rows of
+// the plan (read on device).
 #include "moe_common.cuh"
 
 namespace moe {
 namespace {
 
 constexpr int kRankThreads = 1024;
+constexpr int kIdsPerThread = 16;  // consecutive pairs ranked by one thread per pass
 constexpr int kGatherThreads = 256;
+constexpr int kGatherUnroll = 8;   // 16-byte loads in flight per lane before the stores
 constexpr unsigned kFull = 0xffffffffu;
 
 __global__ void __launch_bounds__(kRankThreads)
 dispatch_rank_kernel(const int32_t* __restrict__ ids, const float* __restrict__ gates,
                      const int32_t* __restrict__ block_off, int N, int k, int E, int beta,
-                     long long r_max, int32_t* __restrict__ row_token, float* __restrict__ row_gate,
-                     int32_t* __restrict__ tok_row, int32_t* __restrict__ status) {
+                     long long r_max, int32_t* __restrict__ row_token,
+                     float* __restrict__ row_gate, int32_t* __restrict__ tok_row,
+                     int32_t* __restrict__ status) {
   __shared__ int warp_tot[32];
   const int e = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -37,22 +41,26 @@ dispatch_rank_kernel(const int32_t* __restrict__ ids, const float* __restrict__ 
   else if (base + cap > r_max) cap = r_max - base;
   long long running = 0;
   bool overflow = false, bad = false;
-  for (int chunk = 0; chunk < N; chunk += 4 * kRankThreads) {
-    const int i0 = chunk + 4 * threadIdx.x;
-    int id[4];
-    if (i0 + 3 < N) {
-      const int4 v = __ldg(reinterpret_cast<const int4*>(ids + i0));
-      id[0] = v.x; id[1] = v.y; id[2] = v.z; id[3] = v.w;
+  for (int chunk = 0; chunk < N; chunk += kIdsPerThread * kRankThreads) {
+    const int i0 = chunk + kIdsPerThread * threadIdx.x;
+    int id[kIdsPerThread];
+    if (i0 + kIdsPerThread <= N) {
+#pragma unroll
+      for (int q = 0; q < kIdsPerThread / 4; ++q) {
+        const int4 v = __ldg(reinterpret_cast<const int4*>(ids + i0) + q);
+        id[4 * q] = v.x; id[4 * q + 1] = v.y; id[4 * q + 2] = v.z; id[4 * q + 3] = v.w;
+      }
     } else {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) id[j] = i0 + j < N ? __ldg(ids + i0 + j) : -1;
+      for (int j = 0; j < kIdsPerThread; ++j) id[j] = i0 + j < N ? __ldg(ids + i0 + j) : -1;
     }
-    int cnt = 0;
+    uint32_t match = 0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      cnt += id[j] == e;
+    for (int j = 0; j < kIdsPerThread; ++j) {
+      match |= (uint32_t)(id[j] == e) << j;
       if (blockIdx.x == 0 && i0 + j < N && (id[j] < 0 || id[j] >= E)) bad = true;
     }
+    const int cnt = __popc(match);
     int incl = cnt;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -73,23 +81,22 @@ dispatch_rank_kernel(const int32_t* __restrict__ ids, const float* __restrict__ 
     __syncthreads();
     long long pos = running + (warp ? warp_tot[warp - 1] : 0) + incl - cnt;
     const int total = warp_tot[31];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (id[j] == e) {
-        const int i = i0 + j;
-        if (pos < cap) {
-          const long long row = base + pos;
-          row_token[row] = i / k;
-          row_gate[row] = __ldg(gates + i);
-          tok_row[i] = (int32_t)row;
-        } else {
-          overflow = true;
-        }
-        ++pos;
+    while (match) {
+      const int j = __ffs(match) - 1;
+      match &= match - 1;
+      const int i = i0 + j;
+      if (pos < cap) {
+        const long long row = base + pos;
+        row_token[row] = i / k;
+        row_gate[row] = __ldg(gates + i);
+        tok_row[i] = (int32_t)row;
+      } else {
+        overflow = true;
       }
+      ++pos;
     }
     running += total;
-    __syncthreads();  // warp_tot is rewritten by the next chunk
+    __syncthreads();  // warp_tot is rewritten by the next pass
   }
   for (long long i = running + threadIdx.x; i < cap; i += blockDim.x) {
     row_token[base + i] = -1;
@@ -110,14 +117,20 @@ dispatch_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ 
        r += warps) {
     const int t = row_token[r];
     uint4* dst = xp + r * d8;
-    if (t >= 0 && t < T) {
-      const uint4* src = x + (long long)t * d8;
-#pragma unroll 4
-      for (int c = lane; c < d8; c += 32) dst[c] = __ldg(src + c);
-    } else {
-      const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll 4
-      for (int c = lane; c < d8; c += 32) dst[c] = z;
+    const bool copy = t >= 0 && t < T;
+    const uint4* src = x + (long long)(copy ? t : 0) * d8;
+    for (int c0 = lane; c0 < d8; c0 += 32 * kGatherUnroll) {
+      uint4 v[kGatherUnroll];
+#pragma unroll
+      for (int u = 0; u < kGatherUnroll; ++u) {
+        const int c = c0 + 32 * u;
+        v[u] = (copy && c < d8) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kGatherUnroll; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < d8) dst[c] = v[u];
+      }
     }
   }
 }

@@ -140,7 +140,9 @@ cudaError_t launch_epl(const moe_cfg& c, const float* logits, int32_t* ids, floa
                        int32_t* counts, int32_t* status, cudaStream_t st) {
   const int warps = kRouteThreads / 32;
   long long want = ((long long)c.T + warps - 1) / warps;
-  long long cap = (long long)num_sms() * 4;
+  // two CTAs per SM: each warp ranks a few rows, and few per-CTA histograms contend on
+  // the global counters
+  long long cap = (long long)num_sms() * 2;
   int grid = (int)(want < cap ? want : cap);
   if (grid < 1) grid = 1;
   route_topk_hist_kernel<EPL><<<grid, kRouteThreads, 0, st>>>(logits, c.T, c.E, c.k, ids,
