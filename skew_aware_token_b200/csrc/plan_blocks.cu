@@ -63,48 +63,50 @@ __device__ __forceinline__ int warp_excl_scan(int v, int lane) {
 }
 
 struct VariantState {
-  int* q;      // [E * P]
-  int* load;   // [P]
-  int* rep;    // [P]
-  int* newc;   // [E]
-  int* order;  // [E]
+  int* q;      // [E * P] blocks of expert e on slot r
+  int* load;   // [P] final slot loads (written at the end)
+  int* order;  // [E] home experts of the current donor, in visiting order
   int* donors; // [P]
 };
 
+// min over lanes 0..7 of a key (lanes >= 8 hold INT_MAX), broadcast to the warp
+__device__ __forceinline__ int min8(int v) {
+  v = min(v, __shfl_xor_sync(kFull, v, 4));
+  v = min(v, __shfl_xor_sync(kFull, v, 2));
+  v = min(v, __shfl_xor_sync(kFull, v, 1));
+  return __shfl_sync(kFull, v, 0);
+}
+
 // Runs greedy variant v on the calling warp; returns (makespan, replicas, rounds) in lane 0.
+// Lane t < P holds slot t's load and replica count in registers; q lives in shared memory
+// and, while one expert moves, each lane touches only its own slot's entry.
 __device__ void greedy_variant(int v, int E, int P, int s, int tau, const int* b,
                                VariantState st, int* out_makespan, int* out_replicas,
                                int* out_rounds) {
   const int lane = threadIdx.x & 31;
   const int D = v >> 1, F = v & 1;
   int* q = st.q;
-  int* load = st.load;
-  int* rep = st.rep;
 
   for (int i = lane; i < E * P; i += 32) q[i] = 0;
   __syncwarp();
   for (int e = lane; e < E; e += 32) q[e * P + e * P / E] = b[e];
-  if (lane < P) {
-    int sum = 0;
-    for (int e = home_lo(lane, E, P); e < home_lo(lane + 1, E, P); ++e) sum += b[e];
-    load[lane] = sum;
-    rep[lane] = 0;
-  }
+  int load = 0, rep = 0;  // lane t < P: slot t
+  if (lane < P)
+    for (int e = home_lo(lane, E, P); e < home_lo(lane + 1, E, P); ++e) load += b[e];
   __syncwarp();
 
   int rounds = 0;
   while (true) {
-    const int maxload = warp_max(lane < P ? load[lane] : INT_MIN);
+    const int maxload = warp_max(lane < P ? load : INT_MIN);
     if (maxload <= tau) break;
     ++rounds;
-    for (int e = lane; e < E; e += 32) st.newc[e] = 0;
 
     // donor order, keys taken at the start of the round
-    const bool is_donor = lane < P && load[lane] > tau;
+    const bool is_donor = lane < P && load > tau;
     int key = 0;
     if (lane < P) {
       if (D == 0) {
-        key = load[lane];
+        key = load;
       } else {
         for (int e = home_lo(lane, E, P); e < home_lo(lane + 1, E, P); ++e)
           key = max(key, q[e * P + lane]);
@@ -135,47 +137,52 @@ __device__ void greedy_variant(int v, int E, int P, int s, int tau, const int* b
         st.order[rk] = e;
       }
       __syncwarp();
-      for (int oi = 0; oi < n; ++oi) {
+      int lr = __shfl_sync(kFull, load, r);  // donor load, warp-uniform
+      for (int oi = 0; oi < n && lr > tau; ++oi) {
         const int e = st.order[oi];
-        while (true) {
-          const int lr = load[r], qer = q[e * P + r];
-          if (!(lr > tau && qer > 0)) break;
+        int qer = q[e * P + r];              // donor's blocks of e, warp-uniform
+        int qt = lane < P ? q[e * P + lane] : 0;
+        int newc = 0;                        // copies of e opened in this round
+        while (lr > tau && qer > 0) {
           int ck = INT_MAX;
-          if (lane < P && lane != r) {
-            const int lt = load[lane];
-            if (lt < tau && (q[e * P + lane] > 0 || (rep[lane] < s && (F || st.newc[e] == 0))))
-              ck = (lt << 4) | lane;
-          }
-          ck = warp_min(ck);
+          if (lane < P && lane != r && load < tau &&
+              (qt > 0 || (rep < s && (F || newc == 0))))
+            ck = (load << 4) | lane;
+          ck = min8(ck);
           if (ck == INT_MAX) break;
           const int t = ck & 15, lt = ck >> 4;
           const int delta = min(min(lr - tau, tau - lt), qer);
-          __syncwarp();
-          if (lane == 0) {
-            if (q[e * P + t] == 0) {
-              rep[t] += 1;
-              st.newc[e] += 1;
-            }
-            q[e * P + r] -= delta;
-            q[e * P + t] += delta;
-            load[r] -= delta;
-            load[t] += delta;
+          const bool opened = __shfl_sync(kFull, qt == 0, t);
+          if (lane == t) {
+            load += delta;
+            rep += opened ? 1 : 0;
+            qt += delta;
           }
-          __syncwarp();
+          if (lane == r) {
+            load -= delta;
+            qt -= delta;
+          }
+          newc += opened ? 1 : 0;
+          lr -= delta;
+          qer -= delta;
           progress = true;
         }
+        if (lane < P) q[e * P + lane] = qt;
+        __syncwarp();
       }
       __syncwarp();
     }
     if (!progress) break;
   }
-  const int mk = warp_max(lane < P ? load[lane] : 0);
-  const int reps = warp_sum(lane < P ? rep[lane] : 0);
+  const int mk = warp_max(lane < P ? load : 0);
+  const int reps = warp_sum(lane < P ? rep : 0);
+  if (lane < P) st.load[lane] = load;
   if (lane == 0) {
     *out_makespan = mk;
     *out_replicas = reps;
     *out_rounds = rounds;
   }
+  __syncwarp();
 }
 
 __global__ void __launch_bounds__(kPlanThreads, 1)
@@ -189,9 +196,7 @@ plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
   int* boff = b + E;                    // E + 1
   int* qv = boff + E + 1;               // 4 * E * P
   int* loadv = qv + 4 * E * P;          // 4 * 8
-  int* repv = loadv + 4 * kMaxP;        // 4 * 8
-  int* newc = repv + 4 * kMaxP;         // 4 * E
-  int* order = newc + 4 * E;            // 4 * E
+  int* order = loadv + 4 * kMaxP;       // 4 * E
   int* donors = order + 4 * E;          // 4 * 8
   int* res = donors + 4 * kMaxP;        // 12: makespan[4], replicas[4], rounds[4]
   int* misc = res + 12;                 // [0] B, [1] tau, [2] best, [3..3+P] slot tile offsets
@@ -231,8 +236,6 @@ plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
     VariantState st;
     st.q = qv + warp * E * P;
     st.load = loadv + warp * kMaxP;
-    st.rep = repv + warp * kMaxP;
-    st.newc = newc + warp * E;
     st.order = order + warp * E;
     st.donors = donors + warp * kMaxP;
     if (mask >> warp & 1u) {
@@ -354,8 +357,7 @@ cudaError_t launch_plan(const moe_cfg& c, const int32_t* counts, uint32_t mask,
                         int32_t* slot_off, int32_t* blocks, int32_t* tiles,
                         int32_t* plan_info, int32_t* status, cudaStream_t st) {
   const int E = c.E, P = c.P;
-  const size_t words = (size_t)E + (E + 1) + 4 * E * P + 4 * kMaxP + 4 * kMaxP + 4 * E +
-                       4 * E + 4 * kMaxP + 12 + 40;
+  const size_t words = (size_t)E + (E + 1) + 4 * E * P + 4 * kMaxP + 4 * E + 4 * kMaxP + 12 + 40;
   const size_t bytes = words * sizeof(int);
   if (bytes > 48 * 1024) {
     cudaError_t err = cudaFuncSetAttribute(plan_kernel,

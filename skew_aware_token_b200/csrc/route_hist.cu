@@ -4,9 +4,11 @@
 // expert-computation equation, and "Routing Skew Problem": c_e and
 // kappa = E * sum_e (c_e / sum_j c_j)^2.
 //
-// One warp per token row.  Lane l holds logits l, l+32, ... of the row (coalesced 128-byte
-// loads); k rounds of a warp arg-max (larger value first, ties to the lower expert id)
-// pick the top-k in descending order.  Gates are the softmax over the k chosen logits.
+// One warp ranks a few token rows together.  Lane l holds logits l, l+32, ... of each row
+// (coalesced 128-byte loads); k rounds of a warp arg-max (larger value first, ties to the
+// lower expert id) pick the top-k in descending order, the rows' shuffle chains
+// interleaved.  Lane j keeps the j-th choice; gates are the softmax over the k chosen
+// logits, normalised with a warp sum.
 // Each CTA counts its tokens' choices in a shared-memory histogram and merges the non-zero
 // bins into `counts` with one global atomic each; a one-CTA kernel then forms S and kappa.
 #include <cfloat>
@@ -19,7 +21,9 @@ namespace {
 
 constexpr int kRouteThreads = 256;
 
-template <int EPL>  // experts per lane = ceil(E / 32)
+// EPL experts per lane = ceil(E / 32); TPW token rows ranked together by one warp, so the
+// shuffle chains of different rows interleave.
+template <int EPL, int TPW>
 __global__ void __launch_bounds__(kRouteThreads)
 route_topk_hist_kernel(const float* __restrict__ logits, int T, int E, int k,
                        int32_t* __restrict__ topk_ids, float* __restrict__ topk_gates,
@@ -31,66 +35,94 @@ route_topk_hist_kernel(const float* __restrict__ logits, int T, int E, int k,
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
   bool bad = false;
-  for (long long t = (long long)blockIdx.x * warps + (threadIdx.x >> 5); t < T;
-       t += (long long)gridDim.x * warps) {
-    const float* row = logits + t * E;
-    float v[EPL];
+  for (long long t0 = ((long long)blockIdx.x * warps + (threadIdx.x >> 5)) * TPW; t0 < T;
+       t0 += (long long)gridDim.x * warps * TPW) {
+    float v[TPW][EPL];
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      float x = e < E ? __ldg(row + e) : -INFINITY;
-      if (e < E && !isfinite(x)) {
-        bad = true;
-        if (x != x) x = -INFINITY;  // NaN never wins; the status bit reports it
+    for (int u = 0; u < TPW; ++u) {
+      const long long t = t0 + u;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        float x = (t < T && e < E) ? __ldg(logits + t * E + e) : -INFINITY;
+        if (t < T && e < E && !isfinite(x)) {
+          bad = true;
+          if (x != x) x = -INFINITY;  // NaN never wins; the status bit reports it
+        }
+        v[u][i] = x;
       }
-      v[i] = x;
     }
-    uint32_t taken = 0;
-    float selv[kMaxK];
-    int seli[kMaxK];
+    uint32_t taken[TPW];
+    float myv[TPW], top[TPW];  // lane j keeps the j-th choice; top = the largest logit
+    int myi[TPW];
+#pragma unroll
+    for (int u = 0; u < TPW; ++u) {
+      taken[u] = 0;
+      myv[u] = -INFINITY;
+      top[u] = 0.f;
+      myi[u] = 0;
+    }
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
       if (j < k) {
-        float bv = -INFINITY;
-        int bi = INT_MAX;
+        float bv[TPW];
+        int bi[TPW];
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-          const int e = lane + 32 * i;
-          if (e < E && !(taken >> i & 1u) && (v[i] > bv || (v[i] == bv && e < bi))) {
-            bv = v[i];
-            bi = e;
+        for (int u = 0; u < TPW; ++u) {
+          bv[u] = -INFINITY;
+          bi[u] = INT_MAX;
+#pragma unroll
+          for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !(taken[u] >> i & 1u) &&
+                (v[u][i] > bv[u] || (v[u][i] == bv[u] && e < bi[u]))) {
+              bv[u] = v[u][i];
+              bi[u] = e;
+            }
           }
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-          if (ov > bv || (ov == bv && oi < bi)) {
-            bv = ov;
-            bi = oi;
+#pragma unroll
+          for (int u = 0; u < TPW; ++u) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv[u], off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi[u], off);
+            if (ov > bv[u] || (ov == bv[u] && oi < bi[u])) {
+              bv[u] = ov;
+              bi[u] = oi;
+            }
           }
         }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        selv[j] = bv;
-        seli[j] = bi;
+#pragma unroll
+        for (int u = 0; u < TPW; ++u) {
+          if ((bi[u] & 31) == lane) taken[u] |= 1u << (bi[u] >> 5);
+          if (lane == j) {
+            myv[u] = bv[u];
+            myi[u] = bi[u];
+          }
+          if (j == 0) top[u] = bv[u];
+        }
       }
     }
-    // gates: softmax over the chosen logits; selv[0] is the largest
-    float w[kMaxK];
-    float sum = 0.f;
+    // gates: softmax over the chosen logits (lanes 0..k-1 hold them, in order)
+    float w[TPW], sum[TPW];
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      if (j < k) {
-        w[j] = expf(selv[j] - selv[0]);
-        sum += w[j];
-      }
+    for (int u = 0; u < TPW; ++u) {
+      w[u] = lane < k ? expf(myv[u] - top[u]) : 0.f;
+      sum[u] = w[u];
     }
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      if (j < k && lane == j) {
-        topk_ids[t * k + j] = seli[j];
-        topk_gates[t * k + j] = w[j] / sum;
-        atomicAdd(&hist[seli[j]], 1);
+    for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+      for (int u = 0; u < TPW; ++u) sum[u] += __shfl_xor_sync(0xffffffffu, sum[u], off);
+    }
+#pragma unroll
+    for (int u = 0; u < TPW; ++u) {
+      const long long t = t0 + u;
+      if (t < T && lane < k) {
+        topk_ids[t * k + lane] = myi[u];
+        topk_gates[t * k + lane] = w[u] / sum[u];
+        atomicAdd(&hist[myi[u]], 1);
       }
     }
   }
@@ -138,15 +170,15 @@ kappa_kernel(const int32_t* __restrict__ counts, int E, int64_t* __restrict__ su
 template <int EPL>
 cudaError_t launch_epl(const moe_cfg& c, const float* logits, int32_t* ids, float* gates,
                        int32_t* counts, int32_t* status, cudaStream_t st) {
-  const int warps = kRouteThreads / 32;
-  long long want = ((long long)c.T + warps - 1) / warps;
-  // two CTAs per SM: each warp ranks a few rows, and few per-CTA histograms contend on
-  // the global counters
-  long long cap = (long long)num_sms() * 2;
+  constexpr int TPW = EPL <= 4 ? 4 : 2;
+  const int rows_per_cta = (kRouteThreads / 32) * TPW;
+  long long want = ((long long)c.T + rows_per_cta - 1) / rows_per_cta;
+  long long cap = (long long)num_sms() * 4;
   int grid = (int)(want < cap ? want : cap);
   if (grid < 1) grid = 1;
-  route_topk_hist_kernel<EPL><<<grid, kRouteThreads, 0, st>>>(logits, c.T, c.E, c.k, ids,
-                                                               gates, counts, status);
+  route_topk_hist_kernel<EPL, TPW><<<grid, kRouteThreads, 0, st>>>(logits, c.T, c.E, c.k,
+                                                                    ids, gates, counts,
+                                                                    status);
   return cudaGetLastError();
 }
 

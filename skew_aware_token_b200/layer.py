@@ -65,30 +65,31 @@ class MoeLayer:
                                self.xp, self.row_token, self.row_gate, self.tok_row,
                                self.status, stream)
 
-    def ffn(self, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, stream=None):
-        out = self.o if mode & N.MOE_FFN_WRITE_O else self.y
+    def ffn(self, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, stream=None, y=None):
+        out = self.o if mode & N.MOE_FFN_WRITE_O else (self.y if y is None else y)
         if out is None:
             raise ValueError("layer built without an O buffer (write_o=False)")
         N.moe_expert_ffn(self.cfg, self.xp, w1, w2, self.tiles, self.plan_info,
                          self.row_token, self.row_gate, mode, self.a_scratch, out,
                          self.status, stream)
 
-    def combine(self, stream=None):
-        N.moe_combine(self.cfg, self.o, self.tok_row, self.topk_gates, self.y, self.status,
-                      stream)
+    def combine(self, stream=None, y=None):
+        N.moe_combine(self.cfg, self.o, self.tok_row, self.topk_gates,
+                      self.y if y is None else y, self.status, stream)
 
     # ------------------------------------------------------------------ whole layer
     def __call__(self, logits, x, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, variant_mask=0,
-                 stream=None):
-        """Route, plan, dispatch, FFN (+ combine): returns y fp32 [T, d] (a view of the
-        layer's buffer, valid until the next call)."""
+                 stream=None, y=None):
+        """Route, plan, dispatch, FFN (+ combine): returns y fp32 [T, d], by default a view
+        of the layer's buffer (valid until the next call), or the caller's `y`."""
         self.route(logits, stream)
         self.plan(variant_mask, stream)
         self.dispatch(x, stream)
-        self.ffn(w1, w2, mode, stream)
+        self.ffn(w1, w2, mode, stream, y)
         if mode & N.MOE_FFN_WRITE_O:
-            self.combine(stream)
-        return self.y[: self.wl.T * self.wl.d].view(self.wl.T, self.wl.d)
+            self.combine(stream, y)
+        out = self.y if y is None else y
+        return out[: self.wl.T * self.wl.d].view(self.wl.T, self.wl.d)
 
     def forward_host(self, logits_h, x_h, w1, w2, y_h, logits_d, x_d, mode=0, stream=None):
         """End to end from pinned host buffers: copies logits and x in, runs the layer,
@@ -98,6 +99,7 @@ class MoeLayer:
         y = self(logits_d, x_d, w1, w2, mode=mode, stream=stream)
         y_h.copy_(y, non_blocking=True)
         return y_h
+
 
     def clear_status(self):
         self.status.zero_()
@@ -127,3 +129,57 @@ class MoeLayer:
         for s in shape:
             n *= s
         return buf[:n].view(*shape)
+
+
+class HostPipeline:
+    """Runs a MoeLayer over a stream of batches held in pinned host memory, overlapping
+    the host-to-device copy of batch i+1 and the device-to-host copy of batch i-1 with the
+    layer's work on batch i (three CUDA streams, two device buffer sets).
+
+        pipe = HostPipeline(layer)
+        for logits_h, x_h, y_h in batches:
+            pipe.submit(logits_h, x_h, y_h, w1, w2)
+        pipe.drain()
+    """
+
+    def __init__(self, layer: MoeLayer, depth: int = 2):
+        wl, dev = layer.wl, layer.device
+        self.layer, self.depth = layer, depth
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_run = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+        self.logits = [torch.empty(wl.T, wl.E, device=dev) for _ in range(depth)]
+        self.x = [torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
+                  for _ in range(depth)]
+        self.y = [torch.empty(max(wl.T * wl.d, 4), device=dev) for _ in range(depth)]
+        ev = lambda: torch.cuda.Event()
+        self.in_done = [ev() for _ in range(depth)]    # inputs of slot landed
+        self.run_done = [ev() for _ in range(depth)]   # layer finished with slot
+        self.out_done = [ev() for _ in range(depth)]   # y of slot read back
+        self.used = [False] * depth
+        self.i = 0
+
+    def submit(self, logits_h, x_h, y_h, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE):
+        b = self.i % self.depth
+        self.i += 1
+        if self.used[b]:
+            # the slot's inputs are free once the layer ran, its y once it was read back
+            self.s_in.wait_event(self.run_done[b])
+            self.s_run.wait_event(self.out_done[b])
+        self.used[b] = True
+        with torch.cuda.stream(self.s_in):
+            self.logits[b].copy_(logits_h, non_blocking=True)
+            self.x[b].copy_(x_h, non_blocking=True)
+            self.in_done[b].record(self.s_in)
+        self.s_run.wait_event(self.in_done[b])
+        with torch.cuda.stream(self.s_run):
+            y = self.layer(self.logits[b], self.x[b], w1, w2, mode=mode, y=self.y[b])
+            self.run_done[b].record(self.s_run)
+        self.s_out.wait_event(self.run_done[b])
+        with torch.cuda.stream(self.s_out):
+            y_h.copy_(y, non_blocking=True)
+            self.out_done[b].record(self.s_out)
+
+    def drain(self):
+        for s in (self.s_in, self.s_run, self.s_out):
+            s.synchronize()

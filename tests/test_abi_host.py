@@ -102,3 +102,12 @@ def test_status_strings():
 def test_binding_refuses_host_tensors():
     with pytest.raises(TypeError):
         N.moe_route_hist(WORKLOADS["tiny"], torch.zeros(4), *[torch.zeros(4)] * 6)
+
+
+def test_layer_api_surface():
+    from skew_aware_token_b200.layer import HostPipeline, MoeLayer
+    for name in ("route", "plan", "dispatch", "ffn", "combine", "forward_host", "clear_status",
+                 "read_status", "view", "__call__"):
+        assert callable(getattr(MoeLayer, name)), name
+    for name in ("submit", "drain"):
+        assert callable(getattr(HostPipeline, name)), name

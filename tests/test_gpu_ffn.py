@@ -117,3 +117,24 @@ def test_repeated_calls_reuse_buffers():
     assert layer.read_status() == 0
     # fp32 atomic accumulation order may differ in the last bits only
     torch.testing.assert_close(layer.view("y"), y1, rtol=1e-5, atol=1e-6)
+
+
+def test_host_pipeline_matches_direct_calls():
+    """The overlapped host-buffer runner gives, batch by batch, what direct calls give."""
+    from skew_aware_token_b200.layer import HostPipeline
+    wl = FULL_CASES[1]
+    w1, w2 = synth.make_weights(wl, "cuda")
+    layer = MoeLayer(wl, "cuda")
+    pipe = HostPipeline(layer)
+    batches = []
+    for seed in range(5):
+        b = wl.with_(seed=seed)
+        batches.append((synth.make_logits(b).pin_memory(), synth.make_x(b).pin_memory(),
+                        torch.empty(wl.T, wl.d).pin_memory()))
+    for logits_h, x_h, y_h in batches:
+        pipe.submit(logits_h, x_h, y_h, w1, w2)
+    pipe.drain()
+    assert layer.read_status() == 0
+    for logits_h, x_h, y_h in batches:
+        want = layer(logits_h.cuda(), x_h.cuda(), w1, w2).cpu()
+        torch.testing.assert_close(y_h, want, rtol=1e-5, atol=1e-6)
