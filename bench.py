@@ -34,7 +34,7 @@ from skew_aware_token_b200 import synth  # noqa: E402
 METRIC = "MoE-layer fwd routed tokens/s and TFLOP/s on 1 B200; % of roofline vs kappa"
 DEFAULT_WORKLOAD = "olmoe_a1"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 7  # route, kappa, plan, rank, gather, fc1, fc2
+LAUNCHES_PER_STEP = 7  # route, kappa, plan, rank, gather, fc1, fc2 (+ combine)
 
 
 def load_peaks():
@@ -226,7 +226,7 @@ def run_ours(args, wl, world, rank, local):
     logits = logits_h.to(dev)
     x = x_h.to(dev)
     write_o = args.ffn == "write_o"
-    layer = MoeLayer(wl, dev, write_o=write_o)
+    layer = MoeLayer(wl, dev, write_o=write_o, gather_x=args.gather_x)
     stream = torch.cuda.current_stream(dev)
     mode = ((N.MOE_FFN_STRICT_SLOTS if args.strict else 0) |
             (N.MOE_FFN_WRITE_O if write_o else 0) | (N.MOE_FFN_SM_PAIR if args.sm_pair else 0))
@@ -245,7 +245,7 @@ def run_ours(args, wl, world, rank, local):
         record[2].record(stream)
         layer.dispatch(x)
         record[3].record(stream)
-        layer.ffn(w1, w2, mode)
+        layer.ffn(w1, w2, mode, x=x)
         if write_o:
             layer.combine()
         record[4].record(stream)
@@ -329,6 +329,8 @@ def run_ours(args, wl, world, rank, local):
                 "weights N(0, 1/sqrt(fan_in)), random-init)",
         "config": workload_config(wl, {"kappa": kappa, "strict_slots": bool(args.strict),
                                        "ffn": args.ffn, "sm_pair": bool(args.sm_pair),
+                                       "fc1_rows": "gathered from x by row_token"
+                                       if args.gather_x else "Xp (dispatched copy)",
                                        "l2": "inputs larger than L2 "
                                        f"(expert weights {weight_bytes / 1e9:.2f} GB > 126 MB)",
                                        "B": pi[0], "tau": pi[1], "makespan": pi[2],
@@ -336,7 +338,7 @@ def run_ours(args, wl, world, rank, local):
         "tflops": round(tflops, 2), "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roofline, "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": (LAUNCHES_PER_STEP + (1 if write_o else 0)) * args.steps,
+        "gpu_launches": (LAUNCHES_PER_STEP + int(write_o) - int(args.gather_x)) * args.steps,
         "clocks": clocks.summary(),
         "impl": "ours",
     }
@@ -398,6 +400,8 @@ def main():
                     help="seconds of CPU work for the whole reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--gather-x", action="store_true",
+                    help="FC1 gathers its rows from x by row_token (no Xp, no gather kernel)")
     ap.add_argument("--ffn", default="fused", choices=["fused", "write_o"],
                     help="fused: FC2 adds gate*O into y; write_o: FC2 stores O, then moe_combine")
     ap.add_argument("--sm-pair", action="store_true",

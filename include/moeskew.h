@@ -105,9 +105,15 @@ enum {
                                 slot (u mod P)'s tiles, so the layer time follows the
                                 plan's makespan (one GPU standing in for P); without it
                                 every unit takes tiles of any slot */
-  MOE_FFN_SM_PAIR = 4        /* flag: run each tile on a pair of SMs (a cluster of two
+  MOE_FFN_SM_PAIR = 4,       /* flag: run each tile on a pair of SMs (a cluster of two
                                 CTAs, tcgen05 cta_group::2, M = 256) instead of each
                                 128-row half on one SM (cta_group::1, the default) */
+  MOE_FFN_GATHER_X = 8       /* flag: the `xp` argument is x itself (bf16 [T, d]); FC1
+                                gathers each tile's rows x[row_token[r]] straight into
+                                shared memory (TMA row gather), so the dispatched copy
+                                Xp is never written (moe_dispatch_permute with
+                                xp = NULL).  Padding rows of A (and of O) then hold
+                                unspecified finite values instead of zeros. */
 };
 
 /* Upper bounds: which = MOE_WS_ROWS -> R_max rows (Xp, A, O, row_token, row_gate);
@@ -160,7 +166,8 @@ MOE_API int moe_plan_blocks(const moe_cfg* cfg, const int32_t* counts, uint32_t 
  *   x          bf16 [T, d]; topk_ids, topk_gates [T, k]; block_off [E+1].
  *   xp         bf16 [R_max, d]: row beta*block_off[e] + i holds x[t] of expert e's i-th
  *              pair in token order; padding rows of each expert's blocks are zero; rows at
- *              or beyond beta*B are not written.
+ *              or beyond beta*B are not written.  May be NULL: then only the row maps
+ *              below are written (for moe_expert_ffn with MOE_FFN_GATHER_X).
  *   row_token  int32 [R_max]: t on valid rows, -1 on padding rows.
  *   row_gate   fp32 [R_max]: topk_gates[t, j] on valid rows, 0 on padding rows.
  *   tok_row    int32 [T, k]: the padded row of pair (t, j).
@@ -174,6 +181,8 @@ MOE_API int moe_dispatch_permute(const moe_cfg* cfg, const uint16_t* x, const in
 /* Grouped SwiGLU expert FFN over the planner's tiles (expert-computation equation):
  * for each tile of expert e, Z = Xp[rows] W1_e^T (fp32 accumulate on the tensor cores),
  * A = SiLU(G) * U rounded to bf16 into a_scratch, then O = A W2_e^T.
+ *   xp         bf16 [R_max, d] from moe_dispatch_permute, or with MOE_FFN_GATHER_X the
+ *              token rows x bf16 [T, d] (Xp[r] = x[row_token[r]] is then read in place).
  *   w1         bf16 [E, 2f, d] (rows 0..f-1 = G, f..2f-1 = U; K-major).
  *   w2         bf16 [E, d, f] (K-major).
  *   tiles, plan_info from moe_plan_blocks; row_token, row_gate from moe_dispatch_permute.
@@ -184,8 +193,8 @@ MOE_API int moe_dispatch_permute(const moe_cfg* cfg, const uint16_t* x, const in
  *              y[row_token[r]] += row_gate[r] * O[r] for every valid row (fp32 atomic
  *              adds: the summation order, and so the last bits, may vary run to run).
  *              MOE_FFN_WRITE_O: O bf16 [R_max, d] (rows of the plan's tiles).
- *   mode       MOE_FFN_FUSED_COMBINE or MOE_FFN_WRITE_O, optionally | MOE_FFN_STRICT_SLOTS
- *              and | MOE_FFN_SM_PAIR.
+ *   mode       MOE_FFN_FUSED_COMBINE or MOE_FFN_WRITE_O, optionally | MOE_FFN_STRICT_SLOTS,
+ *              | MOE_FFN_SM_PAIR and | MOE_FFN_GATHER_X.
  * Two persistent kernels (FC1+SwiGLU, then FC2) of one CTA per SM (in clusters of two
  * CTAs with MOE_FFN_SM_PAIR); every wait inside them is bounded and sets
  * MOE_STATUS_TIMEOUT instead of hanging. */

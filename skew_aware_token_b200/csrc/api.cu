@@ -83,7 +83,8 @@ int moe_dispatch_permute(const moe_cfg* cfg, const uint16_t* x, const int32_t* t
   int rc = check_cfg(cfg);
   if (rc != MOE_OK) return rc;
   if (cfg->d % 8) return MOE_ERR_UNSUPPORTED;
-  rc = check_ptrs({x, topk_ids, topk_gates, block_off, xp, row_token, row_gate, tok_row, status});
+  rc = check_ptrs({x, topk_ids, topk_gates, block_off, row_token, row_gate, tok_row, status});
+  if (rc == MOE_OK && xp) rc = check_ptrs({xp});  // NULL: row maps only
   if (rc != MOE_OK) return rc;
   return cuda_result(launch_dispatch(*cfg, x, topk_ids, topk_gates, block_off, xp, row_token,
                                      row_gate, tok_row, status, (cudaStream_t)stream));
@@ -95,7 +96,7 @@ int moe_expert_ffn(const moe_cfg* cfg, const uint16_t* xp, const uint16_t* w1,
                    uint16_t* a_scratch, void* out, int32_t* status, moe_stream_t stream) {
   int rc = check_cfg(cfg);
   if (rc != MOE_OK) return rc;
-  if (mode & ~(MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR)) return MOE_ERR_INVALID_ARG;
+  if (mode & ~kFfnModes) return MOE_ERR_INVALID_ARG;
   if (cfg->d % 256 || cfg->f % 128) return MOE_ERR_UNSUPPORTED;
   rc = check_ptrs({xp, w1, w2, tiles, plan_info, row_token, row_gate, a_scratch, out, status});
   if (rc != MOE_OK) return rc;

@@ -13,7 +13,8 @@
 // row_gate and tok_row, then marks the expert's padding rows.
 // Pass 2 (gather): one warp per padded row copies x[row_token] (or zeros) with 16-byte
 // vector loads (eight in flight per lane) and stores; the grid strides over the rows of
-// the plan (read on device).
+// the plan (read on device).  Skipped when the caller passes no Xp: the expert FFN can
+// gather the rows itself.
 #include "moe_common.cuh"
 
 namespace moe {
@@ -147,7 +148,7 @@ cudaError_t launch_dispatch(const moe_cfg& c, const uint16_t* x, const int32_t* 
                                                      c.beta, max_rows(c), row_token,
                                                      row_gate, tok_row, status);
   cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
+  if (err != cudaSuccess || xp == nullptr) return err;
   const int grid = num_sms() * 8;
   dispatch_gather_kernel<<<grid, kGatherThreads, 0, st>>>(
       reinterpret_cast<const uint4*>(x), row_token, block_off, c.E, c.beta, c.T,

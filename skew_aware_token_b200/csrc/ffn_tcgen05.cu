@@ -22,7 +22,16 @@
 // Roles in every CTA (192 threads, one CTA per SM, persistent):
 //   warp 0      TMA producer: A [128 x 64] and B [128 or 256 x 64] bf16 tiles per K step
 //               into a ring of shared-memory stages (128-byte swizzle).  In a pair, both
-//               CTAs' copies signal CTA 0's stage barrier.
+//               CTAs' copies signal CTA 0's stage barrier.  With MOE_FFN_GATHER_X, FC1's A
+//               tile is gathered from x itself (rows x[row_token[row]]), so the dispatched
+//               copy Xp is never written.  Single SM: the warp's lanes copy the tile with
+//               16-byte cp.async (8 lanes per 128-byte row segment, written at its
+//               128-byte-swizzled place; padding rows copy token 0's row), each lane's copies
+//               counted on the stage barrier by a cp.async mbarrier arrive; the MMA thread
+//               fences the generic and async proxies before reading the stage.  SM pair:
+//               lane l copies rows 4l..4l+3 with one TMA row-gather (tile::gather4) per K
+//               step (fewer instructions for the warp, but the TMA unit takes ~1.8x longer
+//               per stage than the MMAs need, so this variant is slower).
 //   warp 1      MMA issuer (CTA 0 of a pair): one thread issues the MMAs of a stage into a
 //               TMEM accumulator; tcgen05.commit frees the stage (in both CTAs of a pair)
 //               and, after the last K step, hands the accumulator to the epilogue.
@@ -104,6 +113,8 @@ struct FfnArgs {
   int n_n;       // n-tiles per tile
   int out_ld;    // output row length (elements)
   int write_o;   // FC2: store O (1) or fused combine (0)
+  int gather;    // FC1: A rows gathered from x by row_token (tmA maps x [T, d], box 1 row)
+  const void* x; // the token rows x bf16 [T, d] (gather)
   int strict;
   unsigned long long timeout_ns;
 };
@@ -195,6 +206,29 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(map), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+// Row gather: rows r0..r3 of a 2-D tensor map whose box is one row of 64 columns, columns
+// [x, x + 64), into four consecutive 128-byte rows at dst (the same swizzle as a tile
+// load), completion counted on the pair's first CTA's barrier (cluster address `bar`).
+__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t bar, int x, int4 r) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
+      ".mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(r.x), "r"(r.y), "r"(r.z), "r"(r.w), "r"(bar)
+      : "memory");
+}
+// 16-byte copy global -> shared (through L2 only).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has landed (the barrier's
+// expected count includes this arrival).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
@@ -392,9 +426,12 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
   auto sA = [&](int s) { return smem_u32(smem + s * G::STAGE_BYTES); };
   auto sB = [&](int s) { return smem_u32(smem + s * G::STAGE_BYTES + A_BYTES); };
 
+  // single-SM FC1 gathering A with cp.async: every producer lane arrives on the stage
+  const bool lsu_gather = PHASE == 1 && !PAIR && a.gather;
   if (threadIdx.x == 0) {
     for (int s = 0; s < G::STAGES; ++s) {
-      mbar_init(full_bar(s), 1);   // the MMA CTA's producer (expect_tx)
+      // the MMA CTA's producer (expect_tx), plus the 32 lanes' cp.async arrivals
+      mbar_init(full_bar(s), lsu_gather ? 33 : 1);
       mbar_init(empty_bar(s), 1);  // the MMA thread's commit
     }
     for (int b = 0; b < 2; ++b) {
@@ -423,61 +460,155 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t pending = 0, pend_parity = 0;
-      bool bad_tile = false;
-      for (int it = 0;; ++it) {
-        const int slot = it % RING;
-        const uint32_t ph = (uint32_t)(it / RING) & 1u;
-        int L;
+    // The whole warp walks the items; lane 0 alone draws items and handles the barriers,
+    // and broadcasts what the other lanes need.  Item it+1 is drawn, located and its row
+    // tokens loaded while item it's K steps are issued, so the counter, tile and token
+    // round trips stay off the critical path between items.
+    const bool gather = PHASE == 1 && a.gather;
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t pending = 0, pend_parity = 0;
+    bool bad_tile = false;
+    long long drawn = 0;  // lane 0 of the MMA CTA: the counter value taken for the next item
+    // lane 0 of the MMA CTA: wait until item it's ring slot is free, then take a number
+    auto take = [&](int it) -> bool {
+      if (!mbar_wait(iempty_bar(it % RING), ((uint32_t)(it / RING) & 1u) ^ 1u, abort_flag,
+                     a.status, a.timeout_ns, true))
+        return false;
+      drawn = atomicAdd(sch.counter, 1);
+      return true;
+    };
+    // hand item it to the other roles (MMA CTA) or receive it (other CTA of a pair);
+    // returns the item number, or -1 when the work is done or a wait gave up
+    auto publish = [&](int it, bool took) -> int {
+      const int slot = it % RING;
+      int L = -1;
+      if (lane == 0) {
         if (mma_cta) {
-          if (!mbar_wait(iempty_bar(slot), ph ^ 1u, abort_flag, a.status, a.timeout_ns, true))
-            break;
-          const long long v = atomicAdd(sch.counter, 1);
-          L = v < sch.total ? (int)v : -1;
-          ring[slot] = L;
-          if constexpr (PAIR) {
-            st_remote_u32(mapa(smem_u32((const void*)(ring + slot)), 1), (uint32_t)L);
-            mbar_arrive_remote(mapa(ifull_bar(slot), 1));
+          if (took) {
+            L = drawn < sch.total ? (int)drawn : -1;
+            ring[slot] = L;
+            if constexpr (PAIR) {
+              st_remote_u32(mapa(smem_u32((const void*)(ring + slot)), 1), (uint32_t)L);
+              mbar_arrive_remote(mapa(ifull_bar(slot), 1));
+            }
+            mbar_arrive(ifull_bar(slot));
           }
-          mbar_arrive(ifull_bar(slot));
-        } else {
-          if (!mbar_wait(ifull_bar(slot), ph, abort_flag, a.status, a.timeout_ns, true)) break;
+        } else if (mbar_wait(ifull_bar(slot), (uint32_t)(it / RING) & 1u, abort_flag, a.status,
+                             a.timeout_ns, true)) {
           L = ring[slot];
           mbar_arrive_remote(mapa(iempty_bar(slot), 0));
         }
-        if (L < 0) break;
-        int m, n, half;
-        sch.decode(L, m, n, half);
-        const TileInfo ti = read_tile<PAIR>(a, m, PAIR ? (int)rank : half);
-        if (!ti.ok) bad_tile = true;
-        if (!ti.run) continue;
-        int brow;
-        if (PHASE == 1) brow = ti.e * 2 * a.f + n * (BN / 2) + (PAIR ? (int)rank * a.f : 0);
-        else brow = ti.e * a.d + n * BN + (PAIR ? (int)rank * (BN / 2) : 0);
-        bool stop = false;
+      }
+      return __shfl_sync(0xffffffffu, L, 0);
+    };
+    struct Item {
+      int L;        // item number, -1: none
+      int brow;     // first B row
+      TileInfo ti;
+      int mt[4];    // cp.async gather: tokens of rows lane + 32q (padding rows: token 0)
+      int4 tok;     // row gather: tokens of rows 4 lane .. 4 lane + 3
+    };
+    auto locate = [&](Item& w) {
+      int m, n, half;
+      sch.decode(w.L, m, n, half);
+      w.ti = read_tile<PAIR>(a, m, PAIR ? (int)rank : half);
+      if (PHASE == 1) w.brow = w.ti.e * 2 * a.f + n * (BN / 2) + (PAIR ? (int)rank * a.f : 0);
+      else w.brow = w.ti.e * a.d + n * BN + (PAIR ? (int)rank * (BN / 2) : 0);
+    };
+    // rows outside the tile and padding rows read token 0's row; their results are dropped
+    auto load_tokens = [&](Item& w) {
+      if (!gather || !w.ti.run) return;
+      if (lsu_gather) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = 32 * q + lane;
+          const long long r = (long long)w.ti.row0 + i;
+          const int t = (i < w.ti.nrows && r < a.r_max) ? __ldg(a.row_token + r) : 0;
+          w.mt[q] = (t >= 0 && t < a.T) ? t : 0;
+        }
+      } else {
+        const int i0 = 4 * lane;
+        const long long r0 = (long long)w.ti.row0 + i0;
+        int4 t = make_int4(0, 0, 0, 0);
+        // r_max and row0 are multiples of 64, so the four rows are all in range or none is
+        if (i0 < w.ti.nrows && r0 + 3 < a.r_max)
+          t = __ldg(reinterpret_cast<const int4*>(a.row_token + r0));
+        t.x = (i0 + 0 < w.ti.nrows && t.x >= 0 && t.x < a.T) ? t.x : 0;
+        t.y = (i0 + 1 < w.ti.nrows && t.y >= 0 && t.y < a.T) ? t.y : 0;
+        t.z = (i0 + 2 < w.ti.nrows && t.z >= 0 && t.z < a.T) ? t.z : 0;
+        t.w = (i0 + 3 < w.ti.nrows && t.w >= 0 && t.w < a.T) ? t.w : 0;
+        w.tok = t;
+      }
+    };
+    // cp.async gather: copy j (0..31) of a K step moves 16-byte chunk c = lane & 7 of tile
+    // row 4j + rl (rl = lane >> 3) to its 128-byte-swizzled place: chunk c ^ (row & 7),
+    // where row & 7 = 4 (j & 1) + rl
+    const int rl = lane >> 3, ck = lane & 7;
+    const uint32_t off_even = 128 * rl + ((ck ^ rl) << 4);
+    const uint32_t off_odd = 128 * rl + ((ck ^ (rl + 4)) << 4);
+    const int k_pub = min(2, a.n_k - 1), k_tok = min(4, a.n_k - 1);  // n_k >= 2
+
+    Item cur, nxt;
+    bool took = lane == 0 && mma_cta ? take(0) : true;
+    cur.L = publish(0, took);
+    if (cur.L >= 0) {
+      locate(cur);
+      load_tokens(cur);
+    }
+    for (int it = 0; cur.L >= 0; ++it) {
+      if (!cur.ti.ok) bad_tile = true;
+      bool drew = false, located = false, loaded = false;
+      took = true;
+      nxt.L = -1;
+      bool stop = false;
+      if (cur.ti.run) {
+        int tj[32];  // cp.async gather: token of row 4j + rl
+        if (lsu_gather) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            tj[j] = __shfl_sync(0xffffffffu, cur.mt[j >> 3], (4 * j + rl) & 31);
+        }
         for (int kb = 0; kb < a.n_k; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status, a.timeout_ns,
-                         true)) {
+          int ready = 1;
+          if (lane == 0) {
+            ready = mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status, a.timeout_ns,
+                              true);
+            if (ready) {
+              if (mma_cta)
+                mbar_expect_tx(full_bar(stage),
+                               lsu_gather ? G::TX_BYTES - A_BYTES : G::TX_BYTES);
+              // B first: the weights come from the farthest memory
+              if constexpr (PAIR) {
+                const uint32_t fb = mapa(full_bar(stage), 0);
+                tma_load_2d_pair(sB(stage), &tmB, fb, kb * BK, cur.brow);
+                if (!gather) tma_load_2d_pair(sA(stage), &tmA, fb, kb * BK, cur.ti.a_row);
+              } else {
+                tma_load_2d(sB(stage), &tmB, full_bar(stage), kb * BK, cur.brow);
+                if (PHASE == 1)
+                  tma_load_2d(sB(stage) + G::B_BYTES / 2, &tmB, full_bar(stage), kb * BK,
+                              cur.brow + a.f);
+                if (!gather) tma_load_2d(sA(stage), &tmA, full_bar(stage), kb * BK, cur.ti.a_row);
+              }
+            }
+          }
+          if (!__shfl_sync(0xffffffffu, ready, 0)) {
             stop = true;
             break;
           }
-          if (mma_cta) mbar_expect_tx(full_bar(stage), G::TX_BYTES);
           if constexpr (PAIR) {
-            const uint32_t fb = mapa(full_bar(stage), 0);
-            tma_load_2d_pair(sA(stage), &tmA, fb, kb * BK, ti.a_row);
-            tma_load_2d_pair(sB(stage), &tmB, fb, kb * BK, brow);
-          } else {
-            tma_load_2d(sA(stage), &tmA, full_bar(stage), kb * BK, ti.a_row);
-            if (PHASE == 1) {
-              tma_load_2d(sB(stage), &tmB, full_bar(stage), kb * BK, brow);
-              tma_load_2d(sB(stage) + G::B_BYTES / 2, &tmB, full_bar(stage), kb * BK,
-                          brow + a.f);
-            } else {
-              tma_load_2d(sB(stage), &tmB, full_bar(stage), kb * BK, brow);
-            }
+            if (gather)
+              tma_gather4_pair(sA(stage) + lane * 512, &tmA, mapa(full_bar(stage), 0), kb * BK,
+                               cur.tok);
+          } else if (lsu_gather) {
+            const uint32_t a0 = sA(stage);
+            const __nv_bfloat16* xk =
+                reinterpret_cast<const __nv_bfloat16*>(a.x) + kb * BK + 8 * ck;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              cp_async16(a0 + 512 * j + ((j & 1) ? off_odd : off_even),
+                         xk + (long long)tj[j] * a.d);
+            cp_async_arrive(full_bar(stage));
           }
           pending |= 1u << stage;
           pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
@@ -485,9 +616,32 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             stage = 0;
             phase ^= 1u;
           }
+          // the next item, overlapped with this one's copies
+          if (kb == 0) {
+            if (lane == 0 && mma_cta) took = take(it + 1);
+            drew = true;
+          }
+          if (kb == k_pub) {
+            nxt.L = publish(it + 1, took);
+            if (nxt.L >= 0) locate(nxt);
+            located = true;
+          }
+          if (kb == k_tok) {
+            if (nxt.L >= 0) load_tokens(nxt);
+            loaded = true;
+          }
         }
         if (stop) break;
       }
+      if (!drew && lane == 0 && mma_cta) took = take(it + 1);
+      if (!located) {
+        nxt.L = publish(it + 1, took);
+        if (nxt.L >= 0) locate(nxt);
+      }
+      if (!loaded && nxt.L >= 0) load_tokens(nxt);
+      cur = nxt;
+    }
+    if (lane == 0) {
       if (bad_tile && mma_cta) set_status(a.status, MOE_STATUS_PLAN);
       if (*abort_flag && mma_cta) {
         // let the copies already armed land before shared memory goes away
@@ -528,6 +682,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             break;
           }
           tc_fence_after();
+          if (lsu_gather) fence_proxy_async();  // A arrived through the generic proxy
           const uint32_t a0 = sA(stage), b0 = sB(stage);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
@@ -764,8 +919,11 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   err = cudaMemsetAsync(sched, 0, 16 * sizeof(int32_t), st);
   if (err != cudaSuccess) return err;
 
+  const bool gather = (mode & MOE_FFN_GATHER_X) != 0;
   CUtensorMap tm_xp, tm_w1, tm_a, tm_w2;
-  if (!encode_2d(&tm_xp, xp, c.d, r_max, BM) ||
+  // gather: `xp` is x [T, d], read one row per box by the row-gather copies
+  if (!(gather ? encode_2d(&tm_xp, xp, c.d, (uint64_t)c.T, 1)
+               : encode_2d(&tm_xp, xp, c.d, r_max, BM)) ||
       !encode_2d(&tm_w1, w1, c.d, (uint64_t)c.E * 2 * c.f, BN / 2) ||
       !encode_2d(&tm_a, a_scratch, c.f, r_max, BM) ||
       !encode_2d(&tm_w2, w2, c.f, (uint64_t)c.E * c.d, pair ? BN / 2 : BN))
@@ -793,6 +951,8 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   a1.n_n = c.f / (BN / 2);
   a1.out_ld = c.f;
   a1.write_o = 0;
+  a1.gather = gather;
+  a1.x = gather ? xp : nullptr;
   a2.sched = sched + 8;
   a2.out = out;
   a2.n_k = c.f / BK;

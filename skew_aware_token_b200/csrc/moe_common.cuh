@@ -12,6 +12,9 @@ constexpr int kMaxE = 256;
 constexpr int kMaxK = 8;
 constexpr int kMaxP = 8;
 constexpr long long kMaxN = 1LL << 22;
+// every flag moe_expert_ffn accepts
+constexpr int kFfnModes =
+    MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR | MOE_FFN_GATHER_X;
 
 // Bound on the number of token blocks over every routing of N rows into E experts:
 // sum_e ceil(c_e / beta) <= (N + min(E, N) * (beta - 1)) / beta.

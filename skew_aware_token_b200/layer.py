@@ -13,8 +13,13 @@ from . import native as N
 
 
 class MoeLayer:
-    def __init__(self, wl, device="cuda", write_o: bool = False, guard: int = 0):
-        """`guard` adds that many spare elements after every buffer (canary checks)."""
+    def __init__(self, wl, device="cuda", write_o: bool = False, guard: int = 0,
+                 gather_x: bool = False):
+        """`guard` adds that many spare elements after every buffer (canary checks).
+        `gather_x`: FC1 gathers its rows from x by row_token (MOE_FFN_GATHER_X) and the
+        dispatched copy Xp is neither allocated nor written (saves R_max * d * 2 bytes; as
+        fast while x stays resident in L2, slower once it does not); False (default)
+        materialises Xp with the dispatch gather."""
         self.cfg = N.MoeCfg.of(wl)
         self.wl = wl
         dev = torch.device(device)
@@ -40,7 +45,8 @@ class MoeLayer:
         self.blocks = z(max(2 * Bm, 4))
         self.tiles = z(max(4 * Bm, 4))
         self.plan_info = z(N.PI["LEN"])
-        self.xp = z(max(R * d, 8), dt=torch.bfloat16)
+        self.gather_x = gather_x
+        self.xp = None if gather_x else z(max(R * d, 8), dt=torch.bfloat16)
         self.row_token = z(max(R, 4))
         self.row_gate = z(max(R, 4), dt=f32)
         self.tok_row = z(max(T * k, 4))
@@ -61,15 +67,23 @@ class MoeLayer:
                           self.plan_info, self.status, stream)
 
     def dispatch(self, x, stream=None):
+        """Row maps (and, without gather_x, the dispatched rows Xp)."""
         N.moe_dispatch_permute(self.cfg, x, self.topk_ids, self.topk_gates, self.block_off,
                                self.xp, self.row_token, self.row_gate, self.tok_row,
                                self.status, stream)
 
-    def ffn(self, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, stream=None, y=None):
+    def ffn(self, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, stream=None, y=None, x=None):
+        """The expert FFN; `x` (the token rows) is needed when the layer gathers them."""
         out = self.o if mode & N.MOE_FFN_WRITE_O else (self.y if y is None else y)
         if out is None:
             raise ValueError("layer built without an O buffer (write_o=False)")
-        N.moe_expert_ffn(self.cfg, self.xp, w1, w2, self.tiles, self.plan_info,
+        if self.gather_x:
+            if x is None:
+                raise ValueError("gather_x layer: ffn() needs the token rows x")
+            src, mode = x, mode | N.MOE_FFN_GATHER_X
+        else:
+            src = self.xp
+        N.moe_expert_ffn(self.cfg, src, w1, w2, self.tiles, self.plan_info,
                          self.row_token, self.row_gate, mode, self.a_scratch, out,
                          self.status, stream)
 
@@ -85,7 +99,7 @@ class MoeLayer:
         self.route(logits, stream)
         self.plan(variant_mask, stream)
         self.dispatch(x, stream)
-        self.ffn(w1, w2, mode, stream, y)
+        self.ffn(w1, w2, mode, stream, y, x)
         if mode & N.MOE_FFN_WRITE_O:
             self.combine(stream, y)
         out = self.y if y is None else y
@@ -117,13 +131,15 @@ class MoeLayer:
             "counts": (self.counts, (E,)), "block_off": (self.block_off, (E + 1,)),
             "q": (self.q, (E, P)), "slot_load": (self.slot_load, (P,)),
             "slot_off": (self.slot_off, (P + 1,)), "blocks": (self.blocks, (Bm, 2)),
-            "tiles": (self.tiles, (Bm, 4)), "xp": (self.xp, (R, d)),
+            "tiles": (self.tiles, (Bm, 4)),
             "row_token": (self.row_token, (R,)), "row_gate": (self.row_gate, (R,)),
             "tok_row": (self.tok_row, (T, k)), "a_scratch": (self.a_scratch, (R, wl.f)),
             "y": (self.y, (T, d)),
         }
         if self.o is not None:
             shapes["o"] = (self.o, (R, d))
+        if self.xp is not None:
+            shapes["xp"] = (self.xp, (R, d))
         buf, shape = shapes[name]
         n = 1
         for s in shape:

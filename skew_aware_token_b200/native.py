@@ -23,6 +23,7 @@ MOE_STATUS_BAD_ID, MOE_STATUS_OVERFLOW, MOE_STATUS_NONFINITE = 1, 2, 4
 MOE_STATUS_TIMEOUT, MOE_STATUS_PLAN = 8, 16
 MOE_WS_ROWS, MOE_WS_BLOCKS, MOE_WS_FFN_SCRATCH = 0, 1, 2
 MOE_FFN_FUSED_COMBINE, MOE_FFN_WRITE_O, MOE_FFN_STRICT_SLOTS, MOE_FFN_SM_PAIR = 0, 1, 2, 4
+MOE_FFN_GATHER_X = 8
 PI = dict(B=0, TAU=1, MAKESPAN=2, VARIANT=3, NTILES=4, FIXED_MAKESPAN=5, REPLICAS=6,
           ROUNDS=7, SLOT_TILE_OFF=8, VAR_MAKESPAN=17, VAR_REPLICAS=21, VAR_ROUNDS=25, LEN=32)
 

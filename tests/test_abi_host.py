@@ -85,8 +85,14 @@ def test_null_and_misaligned_pointers_rejected():
         args = [ok] * 10
         args[i] = ok + 8
         assert lib.moe_expert_ffn(cfg, *args[:7], 0, *args[7:], None) == N.MOE_ERR_UNSUPPORTED
+    # dispatch: xp may be NULL (row maps only), but not misaligned; the rest are required
+    disp = [ok] * 9  # x, ids, gates, block_off, xp, row_token, row_gate, tok_row, status
+    disp[4], disp[5] = None, None
+    assert lib.moe_dispatch_permute(cfg, *disp, None) == N.MOE_ERR_INVALID_ARG
+    disp[4], disp[5] = ok + 8, ok
+    assert lib.moe_dispatch_permute(cfg, *disp, None) == N.MOE_ERR_UNSUPPORTED
     assert lib.moe_plan_blocks(cfg, ok, 16, *[ok] * 8, None) == N.MOE_ERR_INVALID_ARG
-    assert lib.moe_expert_ffn(cfg, *[ok] * 7, 8, *[ok] * 3, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_ffn(cfg, *[ok] * 7, 16, *[ok] * 3, None) == N.MOE_ERR_INVALID_ARG
     bad_d = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(d=320)))
     assert lib.moe_expert_ffn(bad_d, *[ok] * 7, 0, *[ok] * 3, None) == N.MOE_ERR_UNSUPPORTED
     bad_f = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(f=192)))

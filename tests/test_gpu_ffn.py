@@ -32,7 +32,19 @@ MODES = [N.MOE_FFN_FUSED_COMBINE, N.MOE_FFN_WRITE_O,
          N.MOE_FFN_WRITE_O | N.MOE_FFN_SM_PAIR | N.MOE_FFN_STRICT_SLOTS]
 
 
+_ORACLE = {}
+
+
 def _oracle_full(wl, w1, w2):
+    """The oracle's whole layer on the workload's inputs (weights are a function of the
+    workload, so the result is kept for the next test of the same workload)."""
+    if wl not in _ORACLE:
+        _ORACLE.clear()
+        _ORACLE[wl] = _oracle_run(wl, w1, w2)
+    return _ORACLE[wl]
+
+
+def _oracle_run(wl, w1, w2):
     logits, x = host_inputs(wl)
     W1 = f32(w1)
     W2 = f32(w2)
@@ -40,11 +52,13 @@ def _oracle_full(wl, w1, w2):
                          k=wl.k, beta=wl.beta, P=wl.P, s=wl.s)
 
 
+@pytest.mark.parametrize("gather_x", [True, False], ids=["gather_x", "xp"])
 @pytest.mark.parametrize("wl", FULL_CASES, ids=lambda w: w.name)
-def test_ffn_every_element(wl):
+def test_ffn_every_element(wl, gather_x):
+    """Both A sources of FC1: rows gathered from x by row_token, and the dispatched Xp."""
     w1, w2 = synth.make_weights(wl, "cuda")
     ref = _oracle_full(wl, w1, w2)
-    layer = MoeLayer(wl, "cuda", write_o=True)
+    layer = MoeLayer(wl, "cuda", write_o=True, gather_x=gather_x)
     for mode in MODES:
         layer.y.fill_(float("nan"))
         run_gpu(wl, w1, w2, mode=mode, layer=layer)
@@ -76,14 +90,17 @@ def test_intermediate_a_matches_swiglu():
     check_y(A, want, "A = SiLU(G) * U")
 
 
-@pytest.mark.parametrize("name", ["qwen3_a1.5", "sweep_all4_p0.5_b128", "sweep_one_p0.3_b64",
-                                  "sweep_all4_p1_b128_zipf1.5", "dsv3_a1"])
-def test_full_size_sampled_tokens(name):
-    """Full-size layers in the benchmark's launch configuration; the oracle recomputes a
-    sample of tokens one by one (rows of the FFN are independent)."""
+@pytest.mark.parametrize("name,gather_x", [
+    ("qwen3_a1.5", False), ("sweep_all4_p0.5_b128", False), ("sweep_one_p0.3_b64", False),
+    ("sweep_all4_p1_b128_zipf1.5", False), ("dsv3_a1", False),
+    ("sweep_all4_p1_b128_zipf1.5", True), ("dsv3_a1", True)])
+def test_full_size_sampled_tokens(name, gather_x):
+    """Full-size layers in the benchmark's launch configuration (and with FC1 gathering
+    its rows from x); the oracle recomputes a sample of tokens one by one (rows of the
+    FFN are independent)."""
     wl = WORKLOADS[name]
     w1, w2 = synth.make_weights(wl, "cuda")
-    layer = run_gpu(wl, w1, w2)
+    layer = run_gpu(wl, w1, w2, layer=MoeLayer(wl, "cuda", gather_x=gather_x))
     assert layer.read_status() == 0
     logits, x = host_inputs(wl)
     ids = layer.view("topk_ids").cpu().numpy()

@@ -34,7 +34,7 @@ def _wl(name):
 def test_route_hist_and_plan_and_dispatch(case):
     wl = _wl(case)
     logits, x = host_inputs(wl)
-    layer = MoeLayer(wl, "cuda")
+    layer = MoeLayer(wl, "cuda", gather_x=False)  # materialise Xp to check its rows
     layer.clear_status()
     layer.route(logits.cuda())
     layer.plan(0)
@@ -169,7 +169,7 @@ def test_nonfinite_logit_sets_status():
 def test_bad_ids_and_overflow_are_reported_not_written_out_of_bounds():
     wl = WORKLOADS["tiny"]
     logits, x = host_inputs(wl)
-    layer = MoeLayer(wl, "cuda", guard=256)
+    layer = MoeLayer(wl, "cuda", guard=256, gather_x=False)
     layer.route(logits.cuda())
     layer.plan(0)
     torch.cuda.synchronize()

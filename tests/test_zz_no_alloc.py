@@ -36,7 +36,7 @@ def test_noalloc_matches_scratch_entry_point_twice(wl, mode):
     torch.manual_seed(0)
     logits, x = synth.make_logits(wl).cuda(), synth.make_x(wl).cuda()
     w1, w2 = synth.make_weights(wl, "cuda")
-    layer = MoeLayer(wl, "cuda", write_o=True)
+    layer = MoeLayer(wl, "cuda", write_o=True, gather_x=False)
     layer.clear_status()
     layer.route(logits)
     layer.plan(0)
@@ -66,7 +66,7 @@ def test_noalloc_refuses_a_problem_larger_than_its_array():
     wl = WORKLOADS["olmoe_a1"]
     assert N.moe_workspace_size(wl, N.MOE_WS_FFN_SCRATCH) > N.MOE_NOALLOC_SCRATCH_BYTES
     w1, w2 = synth.make_weights(wl, "cuda")
-    layer = MoeLayer(wl, "cuda")
+    layer = MoeLayer(wl, "cuda", gather_x=False)
     cfg = N.MoeCfg.of(wl)
     rc = N.lib().moe_expert_ffn_noalloc(
         ctypes.byref(cfg), layer.xp.data_ptr(), w1.data_ptr(), w2.data_ptr(),
