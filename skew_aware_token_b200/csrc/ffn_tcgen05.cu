@@ -15,10 +15,11 @@
 //     loads its own 128 rows of the A tile and half of the B tile (128 of its 256 rows)
 //     into its shared memory; CTA 0 issues tcgen05.mma.cta_group::2 (M=256, N=256), whose
 //     accumulator lands in both CTAs' TMEM (each CTA: its 128 rows x 256 columns).  Each SM
-//     therefore moves 32 KB per K step instead of 48 KB, and six stages fit where four did;
-//     but a tile whose second half is empty still costs a full pair MMA.  On the MoE
-//     workloads measured here the single-SM variant is as fast or faster (the pair wins on
-//     long dense tiles), hence the default.
+//     therefore moves 32 KB per K step instead of 48 KB, and six stages fit where four did.
+//     A tile of at most 128 rows runs as an M=128 pair MMA (64 rows per CTA; each CTA's
+//     TMEM then holds its rows' first N/2 columns in lanes 0..63 and the other N/2 in
+//     lanes 64..127), so no tensor work is spent on an empty half.  On the MoE workloads
+//     measured here the two variants are within a few per cent; single SM is the default.
 // Roles in every CTA (192 threads, one CTA per SM, persistent):
 //   warp 0      TMA producer: A [128 x 64] and B [128 or 256 x 64] bf16 tiles per K step
 //               into a ring of shared-memory stages (128-byte swizzle).  In a pair, both
@@ -88,8 +89,12 @@ struct Geo {
   static constexpr int M = PAIR ? 2 * BM : BM;
   // kind::f16 instruction descriptor: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 = 1),
   // B bf16 (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bit 17, M >> 4 at 24.
-  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
-                                    ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+  static constexpr uint32_t idesc(int m) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+           ((uint32_t)(m >> 4) << 24);
+  }
+  static constexpr uint32_t IDESC = idesc(M);
+  static constexpr uint32_t IDESC_M128 = idesc(BM);  // SM pair: a tile of at most 128 rows
   static constexpr int NBARS = 2 * STAGES + 5 + 2 * RING;
   static constexpr int STG = PHASE == 2 ? STG_BYTES : 0;  // FC2 combine staging
   static constexpr int SMEM = STAGES * STAGE_BYTES + STG + META_BYTES + 1024;
@@ -243,17 +248,17 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 }
 template <bool PAIR>
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t accumulate) {
+                                          uint32_t idesc, uint32_t accumulate) {
   if constexpr (PAIR) {
     asm volatile(
         "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
         "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(Geo<1, true>::IDESC), "r"(accumulate));
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
   } else {
     asm volatile(
         "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(Geo<1, false>::IDESC), "r"(accumulate));
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
   }
 }
 // Arrive on `bar` (same offset in both CTAs of a pair) once this thread's MMAs complete.
@@ -377,22 +382,27 @@ __device__ Sched make_sched(const FfnArgs& a) {
 }
 
 struct TileInfo {
-  int e, row0, nrows;  // row0 / nrows of this CTA's 128-row half
+  int e, row0, nrows;  // row0 / nrows of this CTA's share of the tile
   int a_row;           // A rows this CTA loads (moved inside the buffer when empty)
   bool ok;             // a well-formed tile (all roles of both CTAs agree)
   bool run;            // this work item is executed (single SM: its half has rows)
+  bool m128;           // SM pair: the tile has at most 128 rows, so the pair runs an M = 128
+                       // MMA and each CTA holds 64 of them
 };
+// `part`: single SM, the 128-row half; SM pair, the CTA's rank
 template <bool PAIR>
-__device__ __forceinline__ TileInfo read_tile(const FfnArgs& a, int m, int half) {
+__device__ __forceinline__ TileInfo read_tile(const FfnArgs& a, int m, int part) {
   TileInfo t;
   const int4 v = __ldg(reinterpret_cast<const int4*>(a.tiles) + m);
   t.e = v.x;
   t.ok = v.x >= 0 && v.x < a.E && v.y >= 0 && (long long)v.y < a.r_max && v.z > 0 &&
          v.z <= 2 * BM;
-  t.row0 = v.y + BM * half;
-  t.nrows = v.z - BM * half;
+  t.m128 = PAIR && v.z <= BM;
+  const int share = t.m128 ? BM / 2 : BM;  // rows per CTA
+  t.row0 = v.y + share * part;
+  t.nrows = min(v.z - share * part, share);
   t.run = t.ok && (PAIR || t.nrows > 0);
-  t.a_row = t.nrows > 0 ? t.row0 : (int)max(a.r_max - BM, 0LL);
+  t.a_row = t.nrows > 0 ? t.row0 : (int)max(a.r_max - share, 0LL);
   return t;
 }
 
@@ -400,7 +410,7 @@ __device__ __forceinline__ TileInfo read_tile(const FfnArgs& a, int m, int half)
 template <int PHASE, bool PAIR>  // PHASE 1: FC1 + SwiGLU, 2: FC2 (+ combine)
 __global__ void __launch_bounds__(THREADS, 1)
 ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-           const FfnArgs a) {
+           const __grid_constant__ CUtensorMap tmA64, const FfnArgs a) {
   using G = Geo<PHASE, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -450,6 +460,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (PAIR) prefetch_tmap(&tmA64);
   }
   if (warp == 1) tmem_alloc<PAIR>(smem_u32(tmem_slot));
   tc_fence_before();
@@ -513,7 +524,10 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       int m, n, half;
       sch.decode(w.L, m, n, half);
       w.ti = read_tile<PAIR>(a, m, PAIR ? (int)rank : half);
-      if (PHASE == 1) w.brow = w.ti.e * 2 * a.f + n * (BN / 2) + (PAIR ? (int)rank * a.f : 0);
+      // FC1 B rows: single SM, the n-tile's 128 G rows over its 128 U rows; SM pair, CTA
+      // `rank` holds G rows [64 rank, +64) of the n-tile over the matching U rows, so that
+      // in both accumulator layouts (M = 256 and M = 128) a row's G and U sit in one lane
+      if (PHASE == 1) w.brow = w.ti.e * 2 * a.f + n * (BN / 2) + (PAIR ? (int)rank * (BN / 4) : 0);
       else w.brow = w.ti.e * a.d + n * BN + (PAIR ? (int)rank * (BN / 2) : 0);
     };
     // rows outside the tile and padding rows read token 0's row; their results are dropped
@@ -575,14 +589,24 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             ready = mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status, a.timeout_ns,
                               true);
             if (ready) {
-              if (mma_cta)
-                mbar_expect_tx(full_bar(stage),
-                               lsu_gather ? G::TX_BYTES - A_BYTES : G::TX_BYTES);
+              if (mma_cta) {
+                uint32_t tx = lsu_gather ? G::TX_BYTES - A_BYTES : G::TX_BYTES;
+                if (PAIR && cur.ti.m128) tx = 2 * (A_BYTES / 2 + G::B_BYTES);  // 64 A rows
+                mbar_expect_tx(full_bar(stage), tx);
+              }
               // B first: the weights come from the farthest memory
               if constexpr (PAIR) {
                 const uint32_t fb = mapa(full_bar(stage), 0);
-                tma_load_2d_pair(sB(stage), &tmB, fb, kb * BK, cur.brow);
-                if (!gather) tma_load_2d_pair(sA(stage), &tmA, fb, kb * BK, cur.ti.a_row);
+                if (PHASE == 1) {
+                  tma_load_2d_pair(sB(stage), &tmB, fb, kb * BK, cur.brow);
+                  tma_load_2d_pair(sB(stage) + G::B_BYTES / 2, &tmB, fb, kb * BK,
+                                   cur.brow + a.f);
+                } else {
+                  tma_load_2d_pair(sB(stage), &tmB, fb, kb * BK, cur.brow);
+                }
+                if (!gather)
+                  tma_load_2d_pair(sA(stage), cur.ti.m128 ? &tmA64 : &tmA, fb, kb * BK,
+                                   cur.ti.a_row);
               } else {
                 tma_load_2d(sB(stage), &tmB, full_bar(stage), kb * BK, cur.brow);
                 if (PHASE == 1)
@@ -597,7 +621,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             break;
           }
           if constexpr (PAIR) {
-            if (gather)
+            if (gather && lane < (cur.ti.m128 ? 16 : 32))
               tma_gather4_pair(sA(stage) + lane * 512, &tmA, mapa(full_bar(stage), 0), kb * BK,
                                cur.tok);
           } else if (lsu_gather) {
@@ -675,6 +699,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
           break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+        const uint32_t idesc = ti.m128 ? G::IDESC_M128 : G::IDESC;
         bool stop = false;
         for (int kb = 0; kb < a.n_k; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, a.status, a.timeout_ns, true)) {
@@ -686,7 +711,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
           const uint32_t a0 = sA(stage), b0 = sB(stage);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16<PAIR>(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32),
+            umma_bf16<PAIR>(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc,
                             (kb | kk) != 0);
           issued = true;
           umma_commit_all<PAIR>(empty_bar(stage));
@@ -734,17 +759,42 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
           mbar_wait(tfull_bar(buf), use, abort_flag, a.status, a.timeout_ns, true);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      const long long row = (long long)ti.row0 + rit;
-      const bool valid = rit < ti.nrows && row < a.r_max;
+      // Accumulator layout in TMEM.  Single SM, or SM pair with M = 256: lane 32 quarter + i
+      // holds row 32 quarter + i of this CTA's rows, all N columns.  SM pair with M = 128:
+      // lanes 0..63 hold the CTA's 64 rows with columns [0, N/2), lanes 64..127 the same rows
+      // with columns [N/2, N), both at TMEM columns [0, N/2).
+      const bool m128 = PAIR && ti.m128;
+      const int lrow = m128 ? 32 * (quarter & 1) + lane : rit;
+      const int chalf = m128 ? (quarter >> 1) : 0;  // accumulator column half of this warp
+      const long long row = (long long)ti.row0 + lrow;
+      const bool valid = lrow < ti.nrows && row < a.r_max;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
       if (PHASE == 1) {
-        __nv_bfloat16* A = reinterpret_cast<__nv_bfloat16*>(a.out);
-        uint4* dst = reinterpret_cast<uint4*>(A + row * a.out_ld + n * (BN / 2));
+        // chunk cc: G at TMEM column gcol, U at ucol, giving A columns [ocol, ocol + 32) of
+        // the n-tile.  Single SM: B held the n-tile's 128 G rows over its 128 U rows.  SM
+        // pair: CTA r's B half held G rows [64 r, +64) over the matching U rows, so
+        // accumulator columns [128 r, +64) are G and [128 r + 64, +64) are U.
+        __nv_bfloat16* A = reinterpret_cast<__nv_bfloat16*>(a.out) + row * a.out_ld + n * (BN / 2);
+        const int ncc = m128 ? 2 : 4;
 #pragma unroll 1
-        for (int c = 0; c < (BN / 2) / 32; ++c) {
+        for (int cc = 0; cc < ncc; ++cc) {
+          int gcol, ucol, ocol;
+          if (!PAIR) {
+            gcol = 32 * cc;
+            ucol = BN / 2 + 32 * cc;
+            ocol = 32 * cc;
+          } else if (!m128) {
+            gcol = 128 * (cc >> 1) + 32 * (cc & 1);
+            ucol = gcol + 64;
+            ocol = 64 * (cc >> 1) + 32 * (cc & 1);
+          } else {
+            gcol = 32 * cc;
+            ucol = 64 + 32 * cc;
+            ocol = 64 * chalf + 32 * cc;
+          }
           uint32_t g[32], u[32];
-          tmem_ld32(taddr + c * 32, g);
-          tmem_ld32(taddr + BN / 2 + c * 32, u);
+          tmem_ld32(taddr + gcol, g);
+          tmem_ld32(taddr + ucol, u);
           tmem_wait_ld();
           uint32_t p[16];
 #pragma unroll
@@ -754,16 +804,19 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             p[i] = pack_bf16(a0, a1);
           }
           if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(A + ocol);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              dst[c * 4 + i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+              dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
           }
         }
       } else if (a.write_o) {
+        // chunk c: TMEM columns [32 c, +32) = output columns n BN + ocol0 + 32 c ..
+        const int ncc = m128 ? 4 : 8, ocol0 = 128 * chalf;
         __nv_bfloat16* O = reinterpret_cast<__nv_bfloat16*>(a.out);
-        uint4* dst = reinterpret_cast<uint4*>(O + row * a.out_ld + n * BN);
+        uint4* dst = reinterpret_cast<uint4*>(O + row * a.out_ld + n * BN + ocol0);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < ncc; ++c) {
           uint32_t v[32];
           tmem_ld32(taddr + c * 32, v);
           tmem_wait_ld();
@@ -780,6 +833,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       } else {
         // fused combine: y[token] += gate * O, staged per 32 x 32 chunk so that lanes
         // 8q..8q+7 of one reduction cover a whole 128-byte segment of one row
+        const int ncc = m128 ? 4 : 8, ocol0 = 128 * chalf;
         int tok = -1;
         float gate = 0.f;
         if (valid) {
@@ -789,10 +843,10 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         }
         s_tok[ew * 32 + lane] = tok;
         float* my_row = stg + (ew * 32 + lane) * STG_STRIDE;
-        float* y = reinterpret_cast<float*>(a.out) + n * BN + 4 * (lane & 7);
+        float* y = reinterpret_cast<float*>(a.out) + n * BN + ocol0 + 4 * (lane & 7);
         __syncwarp();
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < ncc; ++c) {
           uint32_t v[32];
           tmem_ld32(taddr + c * 32, v);
           tmem_wait_ld();
@@ -864,8 +918,8 @@ bool encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t oute
 }
 
 template <int PHASE, bool PAIR>
-cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const FfnArgs& args,
-                       cudaStream_t st) {
+cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ta64,
+                       const FfnArgs& args, cudaStream_t st) {
   auto kern = ffn_kernel<PHASE, PAIR>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -895,7 +949,7 @@ cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const FfnAr
   FfnArgs a = args;
   const int units = PAIR ? (int)cfg.gridDim.x / 2 : (int)cfg.gridDim.x;
   a.strict = a.strict && units >= a.P;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, a);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, ta64, a);
 }
 
 }  // namespace
@@ -920,12 +974,17 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   if (err != cudaSuccess) return err;
 
   const bool gather = (mode & MOE_FFN_GATHER_X) != 0;
-  CUtensorMap tm_xp, tm_w1, tm_a, tm_w2;
+  // A maps: boxes of 128 rows, and of 64 rows for the SM pair's tiles of at most 128 rows;
+  // B maps: one CTA's share of the n-tile (FC1 on a pair: 64 G rows, then 64 U rows)
+  CUtensorMap tm_xp, tm_xp64, tm_w1, tm_a, tm_a64, tm_w2;
   // gather: `xp` is x [T, d], read one row per box by the row-gather copies
   if (!(gather ? encode_2d(&tm_xp, xp, c.d, (uint64_t)c.T, 1)
                : encode_2d(&tm_xp, xp, c.d, r_max, BM)) ||
-      !encode_2d(&tm_w1, w1, c.d, (uint64_t)c.E * 2 * c.f, BN / 2) ||
+      !(gather ? encode_2d(&tm_xp64, xp, c.d, (uint64_t)c.T, 1)
+               : encode_2d(&tm_xp64, xp, c.d, r_max, BM / 2)) ||
+      !encode_2d(&tm_w1, w1, c.d, (uint64_t)c.E * 2 * c.f, pair ? BN / 4 : BN / 2) ||
       !encode_2d(&tm_a, a_scratch, c.f, r_max, BM) ||
+      !encode_2d(&tm_a64, a_scratch, c.f, r_max, BM / 2) ||
       !encode_2d(&tm_w2, w2, c.f, (uint64_t)c.E * c.d, pair ? BN / 2 : BN))
     return cudaErrorInvalidValue;
 
@@ -960,11 +1019,11 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   a2.out_ld = c.d;
   a2.write_o = write_o;
 
-  err = pair ? launch_one<1, true>(tm_xp, tm_w1, a1, st)
-             : launch_one<1, false>(tm_xp, tm_w1, a1, st);
+  err = pair ? launch_one<1, true>(tm_xp, tm_w1, tm_xp64, a1, st)
+             : launch_one<1, false>(tm_xp, tm_w1, tm_xp64, a1, st);
   if (err != cudaSuccess) return err;
-  return pair ? launch_one<2, true>(tm_a, tm_w2, a2, st)
-              : launch_one<2, false>(tm_a, tm_w2, a2, st);
+  return pair ? launch_one<2, true>(tm_a, tm_w2, tm_a64, a2, st)
+              : launch_one<2, false>(tm_a, tm_w2, tm_a64, a2, st);
 }
 
 }  // namespace moe
