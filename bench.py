@@ -230,7 +230,7 @@ def run_ours(args, wl, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     mode = ((N.MOE_FFN_STRICT_SLOTS if args.strict else 0) |
             (N.MOE_FFN_WRITE_O if write_o else 0) | (N.MOE_FFN_SM_PAIR if args.sm_pair else 0))
-    vmask = 0
+    vmask = args.variant_mask
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
@@ -334,7 +334,10 @@ def run_ours(args, wl, world, rank, local):
                                        "l2": "inputs larger than L2 "
                                        f"(expert weights {weight_bytes / 1e9:.2f} GB > 126 MB)",
                                        "B": pi[0], "tau": pi[1], "makespan": pi[2],
-                                       "fixed_makespan": pi[5], "variant": pi[3]}),
+                                       "fixed_makespan": pi[5], "variant": pi[3],
+                                       "variant_mask": args.variant_mask,
+                                       "variant_makespans": pi[N.PI["VAR_MAKESPAN"]:
+                                                              N.PI["VAR_MAKESPAN"] + 5]}),
         "tflops": round(tflops, 2), "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roofline, "cpu_baseline": cpu,
         "e2e": e2e,
@@ -400,6 +403,9 @@ def main():
                     help="seconds of CPU work for the whole reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--variant-mask", type=lambda v: int(v, 0), default=0,
+                    help="planner variants (bits 0..3 bounded greedy, bit 4 quota solver; "
+                         "0 = all five) and, in bits 8..15, the quota floor u_min")
     ap.add_argument("--gather-x", action="store_true",
                     help="FC1 gathers its rows from x by row_token (no Xp, no gather kernel)")
     ap.add_argument("--ffn", default="fused", choices=["fused", "write_o"],

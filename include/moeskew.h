@@ -84,16 +84,18 @@ enum {
   MOE_PI_B = 0,              /* B = sum_e b_e */
   MOE_PI_TAU = 1,            /* tau = ceil(B / P) */
   MOE_PI_MAKESPAN = 2,       /* max_r l_r of the chosen plan */
-  MOE_PI_VARIANT = 3,        /* chosen greedy variant (0..3) */
+  MOE_PI_VARIANT = 3,        /* chosen variant (0..3 greedy, 4 quota solver) */
   MOE_PI_NTILES = 4,         /* number of execution tiles (up to 256 rows each) */
   MOE_PI_FIXED_MAKESPAN = 5, /* max_r l_r of the no-replica (fixed placement) plan */
   MOE_PI_REPLICAS = 6,       /* total replicas of the chosen plan */
-  MOE_PI_ROUNDS = 7,         /* greedy rounds of the chosen plan */
+  MOE_PI_ROUNDS = 7,         /* greedy rounds (quota solver: search iterations) of the
+                                chosen plan */
   MOE_PI_SLOT_TILE_OFF = 8,  /* P+1 entries: first tile of each slot */
-  MOE_PI_VAR_MAKESPAN = 17,  /* 4 entries: makespan per variant, -1 when disabled */
-  MOE_PI_VAR_REPLICAS = 21,  /* 4 entries */
-  MOE_PI_VAR_ROUNDS = 25,    /* 4 entries */
-  MOE_PI_LEN = 32
+  MOE_PI_VAR_MAKESPAN = 17,  /* 5 entries: makespan per variant, -1 when disabled */
+  MOE_PI_VAR_REPLICAS = 22,  /* 5 entries */
+  MOE_PI_VAR_ROUNDS = 27,    /* 5 entries */
+  MOE_PI_QUOTA_TAU = 32,     /* threshold the quota solver's search ended on (-1: off) */
+  MOE_PI_LEN = 40
 };
 
 /* moe_expert_ffn modes */
@@ -141,7 +143,12 @@ MOE_API int moe_route_hist(const moe_cfg* cfg, const float* logits, int32_t* top
  *   counts       int32 [E] (from moe_route_hist).
  *   variant_mask bits 0..3 enable greedy variants v = 2*D + F (D donor priority:
  *                0 total overload, 1 largest home-expert load; F fan-out: 0 one new copy
- *                per expert per round, 1 several); 0 means all four.
+ *                per expert per round, 1 several); bit 4 enables variant 4, the quota
+ *                solver ("UltraEP" notes, section 4, Algorithm 1: binary search on the
+ *                threshold with a greedy feasibility oracle); bits 0..4 all clear means
+ *                the four greedy variants (the method's planner; 0x1F runs all five).
+ *                Bits 8..15: the quota solver's floor u_min in blocks (0 means 1).  Other
+ *                bits are invalid.
  *   block_off    int32 [E+1]: exclusive prefix sum of b_e = ceil(c_e / beta).
  *   q            int32 [E, P] row-major: blocks of expert e run by slot r, of the best
  *                enabled variant (least makespan, then fewest replicas, then lowest v).

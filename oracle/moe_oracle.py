@@ -20,9 +20,14 @@ Sources (cited by page title and section; the pages print no code and no worked 
             A_e = SiLU(G_e) * U_e, O_e = A_e W2_e, y_t = sum_{e in S_t} p_{t,e} O_e[t];
           - Summary and "Theoretical Contributions" 1: router outputs, token counts,
             expert selections and routing weights are preserved.
-  [UE]  "UltraEP: Exact Load Balancing for Rack-Scale MoE" reading notes, section 4,
-        Algorithm 1: the receiver of a shifted quota is the rank with the most slack that
-        does not already host the expert (used here as the receiver rule).
+  [UE]  "UltraEP: Exact Load Balancing for Rack-Scale MoE" reading notes, section 4
+        ("The Quota-Driven Planning Solver", Algorithm 1 "joint solving"): binary search
+        for the smallest load threshold tau a greedy feasibility oracle satisfies; excess
+        exc_r = max(l_r - tau, 0) and slack slk_r = max(tau - l_r, 0); overloaded ranks by
+        descending excess, their hot experts by descending load; receiver t* = the rank
+        with the most slack that does not host the expert; delta = min(exc_r, slk_t*,
+        remaining load of e), transferred only if delta >= the quota floor u_min.  The
+        receiver rule also serves the bounded greedy search (R4).
   [TE]  TopoEP abstract: plans are deterministic and bitwise identical.
 
 Readings where the pages leave a step open (each is also listed in the design notes):
@@ -38,12 +43,23 @@ Readings where the pages leave a step open (each is also listed in the design no
       inside an expert; expert e's i-th row goes to padded row beta*block_off[e] + i.
   R6  the FFN is evaluated in fp32 from the exact bf16 input values; A is kept in fp32.
   R7  the combine sums j = 0..k-1 in ascending order in fp32.
+  R8  the quota solver of `plan_quota` (variant 4) in this block formulation: ranks are
+      the P slots, the load of expert e is b_e blocks, N_slot = s; the search runs over
+      integer tau in [ceil(B / P), max_r home load] exactly as printed (while lo < hi,
+      tau = floor((lo + hi) / 2); the target coefficient beta does not enter the printed
+      loop and is not used); the oracle makes one transfer per hot expert (as printed),
+      receivers are ranks other than the donor with slack > 0 and a free replica slot
+      (rep_t < s), ties of slack to the lower rank; u_min is counted in blocks (default 1);
+      the plan is the oracle's quota table at the tau the search ends on.
 """
 from __future__ import annotations
 
 import numpy as np
 
-VARIANT_NAMES = ("over/one", "over/multi", "hot/one", "hot/multi")
+VARIANT_NAMES = ("over/one", "over/multi", "hot/one", "hot/multi", "quota")
+QUOTA_VARIANT = 4
+GREEDY_VARIANTS = 0xF
+ALL_VARIANTS = 0x1F
 
 
 # --------------------------------------------------------------------------- routing
@@ -182,6 +198,74 @@ def plan_variant(b, P: int, s: int, v: int) -> dict:
             "B": B, "variant": v, "rounds": rounds}
 
 
+def quota_feasible(b, P: int, s: int, u_min: int, tau: int) -> dict:
+    """[UE] Algorithm 1's greedy feasibility oracle at one threshold tau; reading R8.
+
+    Start from the home placement q[e][h(e)] = b_e.  exc_r = max(l_r - tau, 0) and
+    slk_r = max(tau - l_r, 0).  Overloaded ranks in order of descending excess (ties to the
+    lower rank); for each, its hot experts (h(e) = r, b_e > 0) in order of descending load
+    (ties to the lower id): t* = the rank != r with the most slack among those with slack
+    left and a free replica slot (ties to the lower rank); delta = min(exc_r, slk_t*,
+    q[e][r]); if delta >= u_min the quota moves to t*, which then hosts a replica of e.
+    Feasible when no rank keeps an excess."""
+    E = len(b)
+    h = [owner(e, E, P) for e in range(E)]
+    q = [[0] * P for _ in range(E)]
+    load = [0] * P
+    for e in range(E):
+        q[e][h[e]] = int(b[e])
+        load[h[e]] += int(b[e])
+    exc = [max(load[r] - tau, 0) for r in range(P)]
+    slk = [max(tau - load[r], 0) for r in range(P)]
+    rep = [0] * P
+    for r in sorted((r for r in range(P) if exc[r] > 0), key=lambda r: (-exc[r], r)):
+        hot = sorted((e for e in range(E) if h[e] == r and b[e] > 0), key=lambda e: (-b[e], e))
+        for e in hot:
+            cand = [t for t in range(P) if t != r and q[e][t] == 0 and slk[t] > 0 and rep[t] < s]
+            if not cand:
+                continue
+            t = min(cand, key=lambda t: (-slk[t], t))
+            delta = min(exc[r], slk[t], q[e][r])
+            if delta >= u_min:
+                q[e][r] -= delta
+                q[e][t] += delta
+                exc[r] -= delta
+                slk[t] -= delta
+                load[r] -= delta
+                load[t] += delta
+                rep[t] += 1
+    return {"feasible": all(x == 0 for x in exc), "q": q, "load": load, "rep": rep}
+
+
+def plan_quota(b, P: int, s: int, u_min: int = 1) -> dict:
+    """[UE] Algorithm 1 (joint solving): binary search for the smallest tau that
+    `quota_feasible` satisfies, on [ceil(B / P), max_r home load]; the plan is the quota
+    table at that tau.  Reading R8.  'rounds' counts the search iterations."""
+    E = len(b)
+    b = [int(x) for x in b]
+    u_min = max(int(u_min), 1)
+    B = sum(b)
+    lo = -(-B // P)
+    home = [0] * P
+    for e in range(E):
+        home[owner(e, E, P)] += b[e]
+    hi = max(home) if P else 0
+    rounds = 0
+    while lo < hi:
+        rounds += 1
+        tau = (lo + hi) // 2
+        if quota_feasible(b, P, s, u_min, tau)["feasible"]:
+            hi = tau
+        else:
+            lo = tau + 1
+    res = quota_feasible(b, P, s, u_min, hi)
+    load = res["load"]
+    return {"q": np.array(res["q"], dtype=np.int32).reshape(E, P), "load": load,
+            "makespan": max(load) if P else 0, "replicas": sum(res["rep"]),
+            "tau": -(-B // P), "tau_star": hi, "B": B, "variant": QUOTA_VARIANT,
+            "rounds": rounds}
+
+
 def fixed_makespan(b, P: int) -> int:
     """Largest slot load of the no-replica (fixed placement) assignment."""
     E = len(b)
@@ -191,11 +275,15 @@ def fixed_makespan(b, P: int) -> int:
     return max(load)
 
 
-def plan(b, P: int, s: int, variant_mask: int = 0xF) -> dict:
-    """Run the enabled variants and keep the best.  Reading R4: the best is the
-    lexicographic minimum of (makespan, total replicas, variant index)."""
-    mask = variant_mask & 0xF or 0xF
+def plan(b, P: int, s: int, variant_mask: int = GREEDY_VARIANTS, u_min: int = 1) -> dict:
+    """Run the enabled variants (bits 0..3: the greedy searches, bit 4: the quota solver;
+    0 means the four greedy searches, the method's planner) and keep the best.  Reading
+    R4: the best is the lexicographic minimum of (makespan, total replicas, variant
+    index)."""
+    mask = variant_mask & ALL_VARIANTS or GREEDY_VARIANTS
     results = [plan_variant(b, P, s, v) for v in range(4) if mask >> v & 1]
+    if mask >> QUOTA_VARIANT & 1:
+        results.append(plan_quota(b, P, s, u_min))
     best = min(results, key=lambda r: (r["makespan"], r["replicas"], r["variant"]))
     out = dict(best)
     out["all"] = {r["variant"]: r for r in results}
@@ -290,7 +378,7 @@ def combine(O_rows: np.ndarray, tok_row: np.ndarray, gates: np.ndarray) -> np.nd
 
 
 def moe_forward(logits, x, get_expert, k: int, beta: int, P: int, s: int,
-                variant_mask: int = 0xF) -> dict:
+                variant_mask: int = GREEDY_VARIANTS) -> dict:
     """The whole forward layer: route, histogram + kappa, blocks, plan, dispatch,
     per-expert FFN, combine.  `x` is [T, d] fp32 holding bf16 values; `get_expert(e)`
     returns (w1 [2f, d], w2 [d, f]) as fp32 arrays holding bf16 values."""

@@ -20,6 +20,15 @@
 //          A round that moves nothing ends the search.
 //   best   least (makespan, total replicas, variant index) among enabled variants.
 //
+// Variant 4 is the quota solver of the UltraEP notes (section 4, Algorithm 1): a binary
+// search over integer thresholds tau in [ceil(B / P), max_r home load] (tau = floor((lo +
+// hi) / 2); feasible -> hi = tau, else lo = tau + 1) around a greedy feasibility oracle:
+// from the home placement, overloaded slots by (excess desc, r asc), each one's loaded
+// home experts by (b_e desc, e asc), one transfer per expert to the slot t != r of most
+// slack among those with slack left and a free replica slot (rep_t < s; ties to the lower
+// slot), of delta = min(excess, slack, b_e) blocks, made only if delta >= u_min; tau is
+// feasible when no excess is left.  The plan is the oracle's quota table at the final tau.
+//
 // One warp runs one variant: slot-parallel work (candidate test, arg-min, maxima) uses
 // lanes 0..P-1 and warp shuffles; expert-parallel work strides the lanes over experts.
 // Lane 0 applies each move; __syncwarp() orders it against the next read.
@@ -30,7 +39,9 @@
 namespace moe {
 namespace {
 
-constexpr int kPlanThreads = 128;  // 4 warps = 4 greedy variants
+constexpr int kVariants = 5;       // 4 greedy variants + the quota solver, one warp each
+constexpr int kPlanThreads = 32 * kVariants;
+constexpr int kQuota = 4;          // variant index of the quota solver
 constexpr int kTileRows = 256;     // rows of one execution tile of the FFN
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -39,11 +50,6 @@ __device__ __forceinline__ int home_lo(int r, int E, int P) { return (r * E + P 
 __device__ __forceinline__ int warp_max(int v) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) v = max(v, __shfl_xor_sync(kFull, v, off));
-  return v;
-}
-__device__ __forceinline__ int warp_min(int v) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v = min(v, __shfl_xor_sync(kFull, v, off));
   return v;
 }
 __device__ __forceinline__ int warp_sum(int v) {
@@ -185,21 +191,128 @@ __device__ void greedy_variant(int v, int E, int P, int s, int tau, const int* b
   __syncwarp();
 }
 
+// Orders the lanes 0..P-1 flagged in `is_donor` by (key desc, lane asc) into donors[].
+__device__ __forceinline__ int order_donors(bool is_donor, int key, int P, int* donors) {
+  const int lane = threadIdx.x & 31;
+  const unsigned dmask = __ballot_sync(kFull, is_donor);
+  int rank = 0;
+  for (int r2 = 0; r2 < P; ++r2) {
+    const int k2 = __shfl_sync(kFull, key, r2);
+    if (is_donor && (dmask >> r2 & 1u) && (k2 > key || (k2 == key && r2 < lane))) ++rank;
+  }
+  if (is_donor) donors[rank] = lane;
+  __syncwarp();
+  return __popc(dmask);
+}
+
+// Runs the quota solver on the calling warp; the plan lands in st.q.  Lane t < P holds
+// slot t's home load, and during an oracle pass its load and replica count.
+__device__ void quota_variant(int E, int P, int s, int u_min, int B, const int* b,
+                              VariantState st, int* out_makespan, int* out_replicas,
+                              int* out_rounds, int* out_tau) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kBig = 1 << 26;  // slack < B < 2^17; (kBig - slack) << 4 | slot fits an int
+  // each slot's home experts by (b_e desc, e asc), at st.order[home_lo(r) ..)
+  for (int r = 0; r < P; ++r) {
+    const int lo = home_lo(r, E, P), n = home_lo(r + 1, E, P) - lo;
+    for (int i = lane; i < n; i += 32) {
+      const int be = b[lo + i];
+      int rk = 0;
+      for (int i2 = 0; i2 < n; ++i2) {
+        const int b2 = b[lo + i2];
+        rk += (b2 > be) || (b2 == be && i2 < i);
+      }
+      st.order[lo + rk] = lo + i;
+    }
+  }
+  int home = 0;
+  if (lane < P)
+    for (int e = home_lo(lane, E, P); e < home_lo(lane + 1, E, P); ++e) home += b[e];
+  __syncwarp();
+
+  // One oracle pass at tau: returns feasibility; load / rep end in the lanes' registers;
+  // with `write`, the transfers are applied to st.q (which then holds the home placement).
+  auto oracle = [&](int tau, bool write, int& load, int& rep) -> bool {
+    load = lane < P ? home : 0;
+    rep = 0;
+    const int ndon = order_donors(lane < P && load > tau, load, P, st.donors);
+    bool stuck = false;  // no slot can receive any more
+    for (int di = 0; di < ndon && !stuck; ++di) {
+      const int r = st.donors[di];
+      int exc = __shfl_sync(kFull, load, r) - tau;  // warp-uniform
+      for (int oi = home_lo(r, E, P); oi < home_lo(r + 1, E, P) && exc > 0; ++oi) {
+        const int e = st.order[oi], be = b[e];
+        if (be == 0) break;  // the rest of this slot's experts carry no load
+        const int slk = lane < P ? max(tau - load, 0) : 0;
+        int ck = INT_MAX;
+        if (lane < P && lane != r && slk > 0 && rep < s) ck = ((kBig - slk) << 4) | lane;
+        ck = min8(ck);
+        if (ck == INT_MAX) {  // slack and free slots only shrink: nobody can receive later
+          stuck = true;
+          break;
+        }
+        const int t = ck & 15, slk_t = kBig - (ck >> 4);
+        const int delta = min(min(exc, slk_t), be);
+        if (delta >= u_min) {
+          if (lane == t) {
+            load += delta;
+            rep += 1;
+          }
+          if (lane == r) load -= delta;
+          exc -= delta;
+          if (write && lane == 0) {
+            st.q[e * P + r] -= delta;
+            st.q[e * P + t] += delta;
+          }
+        }
+        __syncwarp();
+      }
+    }
+    return warp_max(lane < P ? load : INT_MIN) <= tau;
+  };
+
+  int lo = P > 0 ? (B + P - 1) / P : 0;
+  int hi = warp_max(lane < P ? home : 0);
+  int rounds = 0, load = 0, rep = 0;
+  while (lo < hi) {
+    ++rounds;
+    const int tau = (lo + hi) / 2;
+    if (oracle(tau, false, load, rep)) hi = tau;
+    else lo = tau + 1;
+  }
+  for (int i = lane; i < E * P; i += 32) st.q[i] = 0;
+  __syncwarp();
+  for (int e = lane; e < E; e += 32) st.q[e * P + e * P / E] = b[e];
+  __syncwarp();
+  oracle(hi, true, load, rep);
+  __syncwarp();
+  const int mk = warp_max(lane < P ? load : 0);
+  const int reps = warp_sum(lane < P ? rep : 0);
+  if (lane < P) st.load[lane] = load;
+  if (lane == 0) {
+    *out_makespan = mk;
+    *out_replicas = reps;
+    *out_rounds = rounds;
+    *out_tau = hi;
+  }
+  __syncwarp();
+}
+
 __global__ void __launch_bounds__(kPlanThreads, 1)
 plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
-            unsigned mask, int b_max, int32_t* __restrict__ block_off, int32_t* __restrict__ q_out,
+            unsigned mask, int u_min, int b_max, int32_t* __restrict__ block_off, int32_t* __restrict__ q_out,
             int32_t* __restrict__ slot_load, int32_t* __restrict__ slot_off,
             int32_t* __restrict__ blocks, int32_t* __restrict__ tiles,
             int32_t* __restrict__ plan_info, int32_t* __restrict__ status) {
   extern __shared__ int sm[];
   int* b = sm;                          // E
   int* boff = b + E;                    // E + 1
-  int* qv = boff + E + 1;               // 4 * E * P
-  int* loadv = qv + 4 * E * P;          // 4 * 8
-  int* order = loadv + 4 * kMaxP;       // 4 * E
-  int* donors = order + 4 * E;          // 4 * 8
-  int* res = donors + 4 * kMaxP;        // 12: makespan[4], replicas[4], rounds[4]
-  int* misc = res + 12;                 // [0] B, [1] tau, [2] best, [3..3+P] slot tile offsets
+  int* qv = boff + E + 1;               // 5 * E * P
+  int* loadv = qv + kVariants * E * P;  // 5 * 8
+  int* order = loadv + kVariants * kMaxP;  // 5 * E
+  int* donors = order + kVariants * E;  // 5 * 8
+  int* res = donors + kVariants * kMaxP;  // 16: makespan[5], replicas[5], rounds[5], tau*
+  int* misc = res + 16;                 // [0] B, [1] tau, [2] best, [3..3+P] slot tile offsets
                                         // [12..12+P] slot_off, [24..] fixed loads (P)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -231,19 +344,26 @@ plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
   __syncthreads();
   const int B = misc[0], tau = misc[1];
 
-  // ---- four greedy variants, one per warp
+  // ---- four greedy variants and the quota solver, one per warp
   {
     VariantState st;
     st.q = qv + warp * E * P;
     st.load = loadv + warp * kMaxP;
     st.order = order + warp * E;
     st.donors = donors + warp * kMaxP;
-    if (mask >> warp & 1u) {
-      greedy_variant(warp, E, P, s, tau, b, st, &res[warp], &res[4 + warp], &res[8 + warp]);
-    } else if (lane == 0) {
-      res[warp] = INT_MAX;
-      res[4 + warp] = INT_MAX;
-      res[8 + warp] = 0;
+    if (!(mask >> warp & 1u)) {
+      if (lane == 0) {
+        res[warp] = INT_MAX;
+        res[kVariants + warp] = INT_MAX;
+        res[2 * kVariants + warp] = 0;
+        if (warp == kQuota) res[3 * kVariants] = -1;
+      }
+    } else if (warp == kQuota) {
+      quota_variant(E, P, s, u_min, B, b, st, &res[warp], &res[kVariants + warp],
+                    &res[2 * kVariants + warp], &res[3 * kVariants]);
+    } else {
+      greedy_variant(warp, E, P, s, tau, b, st, &res[warp], &res[kVariants + warp],
+                     &res[2 * kVariants + warp]);
     }
   }
   __syncthreads();
@@ -251,9 +371,10 @@ plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
   // ---- best variant: least (makespan, replicas, v)
   if (tid == 0) {
     int best = -1;
-    for (int v = 0; v < 4; ++v) {
+    for (int v = 0; v < kVariants; ++v) {
       if (!(mask >> v & 1u)) continue;
-      if (best < 0 || res[v] < res[best] || (res[v] == res[best] && res[4 + v] < res[4 + best]))
+      if (best < 0 || res[v] < res[best] ||
+          (res[v] == res[best] && res[kVariants + v] < res[kVariants + best]))
         best = v;
     }
     misc[2] = best;
@@ -301,22 +422,23 @@ plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
     plan_info[MOE_PI_VARIANT] = best;
     plan_info[MOE_PI_NTILES] = min(tacc, b_max);
     plan_info[MOE_PI_FIXED_MAKESPAN] = fixed_max;
-    plan_info[MOE_PI_REPLICAS] = res[4 + best];
-    plan_info[MOE_PI_ROUNDS] = res[8 + best];
+    plan_info[MOE_PI_REPLICAS] = res[kVariants + best];
+    plan_info[MOE_PI_ROUNDS] = res[2 * kVariants + best];
     for (int r = 0; r <= kMaxP; ++r)
       plan_info[MOE_PI_SLOT_TILE_OFF + r] = r <= P ? min(misc[3 + r], b_max) : min(tacc, b_max);
-    for (int v = 0; v < 4; ++v) {
+    for (int v = 0; v < kVariants; ++v) {
       const bool on = mask >> v & 1u;
       plan_info[MOE_PI_VAR_MAKESPAN + v] = on ? res[v] : -1;
-      plan_info[MOE_PI_VAR_REPLICAS + v] = on ? res[4 + v] : -1;
-      plan_info[MOE_PI_VAR_ROUNDS + v] = on ? res[8 + v] : -1;
+      plan_info[MOE_PI_VAR_REPLICAS + v] = on ? res[kVariants + v] : -1;
+      plan_info[MOE_PI_VAR_ROUNDS + v] = on ? res[2 * kVariants + v] : -1;
     }
-    for (int i = MOE_PI_VAR_ROUNDS + 4; i < MOE_PI_LEN; ++i) plan_info[i] = 0;
+    plan_info[MOE_PI_QUOTA_TAU] = res[3 * kVariants];
+    for (int i = MOE_PI_QUOTA_TAU + 1; i < MOE_PI_LEN; ++i) plan_info[i] = 0;
   }
   __syncthreads();
 
-  // ---- block list and tile list: warp w expands slots w, w+4
-  for (int r = warp; r < P; r += 4) {
+  // ---- block list and tile list: warp w expands slots w, w + 5
+  for (int r = warp; r < P; r += kVariants) {
     const int C = (E + 31) / 32;
     const int e0 = min(lane * C, E), e1 = min(e0 + C, E);
     int nb = 0, nt = 0;
@@ -357,7 +479,8 @@ cudaError_t launch_plan(const moe_cfg& c, const int32_t* counts, uint32_t mask,
                         int32_t* slot_off, int32_t* blocks, int32_t* tiles,
                         int32_t* plan_info, int32_t* status, cudaStream_t st) {
   const int E = c.E, P = c.P;
-  const size_t words = (size_t)E + (E + 1) + 4 * E * P + 4 * kMaxP + 4 * E + 4 * kMaxP + 12 + 40;
+  const size_t words = (size_t)E + (E + 1) + kVariants * ((size_t)E * P + kMaxP + E + kMaxP) +
+                       16 + 40;
   const size_t bytes = words * sizeof(int);
   if (bytes > 48 * 1024) {
     cudaError_t err = cudaFuncSetAttribute(plan_kernel,
@@ -365,8 +488,10 @@ cudaError_t launch_plan(const moe_cfg& c, const int32_t* counts, uint32_t mask,
                                            (int)bytes);
     if (err != cudaSuccess) return err;
   }
-  const unsigned m = (mask & 0xFu) ? (mask & 0xFu) : 0xFu;
-  plan_kernel<<<1, kPlanThreads, bytes, st>>>(counts, E, P, c.s, c.beta, m,
+  const unsigned all = (1u << kVariants) - 1u;
+  const unsigned m = (mask & all) ? (mask & all) : 0xFu;  // default: the four greedy searches
+  const int u_min = (mask >> 8 & 0xFFu) ? (int)(mask >> 8 & 0xFFu) : 1;
+  plan_kernel<<<1, kPlanThreads, bytes, st>>>(counts, E, P, c.s, c.beta, m, u_min,
                                               (int)max_blocks(c), block_off, q, slot_load,
                                               slot_off, blocks, tiles, plan_info, status);
   return cudaGetLastError();

@@ -25,7 +25,23 @@ MOE_WS_ROWS, MOE_WS_BLOCKS, MOE_WS_FFN_SCRATCH = 0, 1, 2
 MOE_FFN_FUSED_COMBINE, MOE_FFN_WRITE_O, MOE_FFN_STRICT_SLOTS, MOE_FFN_SM_PAIR = 0, 1, 2, 4
 MOE_FFN_GATHER_X = 8
 PI = dict(B=0, TAU=1, MAKESPAN=2, VARIANT=3, NTILES=4, FIXED_MAKESPAN=5, REPLICAS=6,
-          ROUNDS=7, SLOT_TILE_OFF=8, VAR_MAKESPAN=17, VAR_REPLICAS=21, VAR_ROUNDS=25, LEN=32)
+          ROUNDS=7, SLOT_TILE_OFF=8, VAR_MAKESPAN=17, VAR_REPLICAS=22, VAR_ROUNDS=27,
+          QUOTA_TAU=32, LEN=40)
+N_VARIANTS = 5          # planner variants: 0..3 bounded greedy, 4 quota solver
+QUOTA_VARIANT = 4
+
+
+def variant_mask(variants=(), u_min: int = 1) -> int:
+    """moe_plan_blocks's variant_mask: enabled variants (none = all five) and the quota
+    solver's floor u_min in blocks."""
+    m = 0
+    for v in variants:
+        m |= 1 << v
+    if not 1 <= u_min <= 255:
+        raise ValueError("u_min must be in 1..255 blocks")
+    if u_min != 1:
+        m |= u_min << 8
+    return m
 
 
 class MoeError(RuntimeError):

@@ -91,7 +91,8 @@ def test_null_and_misaligned_pointers_rejected():
     assert lib.moe_dispatch_permute(cfg, *disp, None) == N.MOE_ERR_INVALID_ARG
     disp[4], disp[5] = ok + 8, ok
     assert lib.moe_dispatch_permute(cfg, *disp, None) == N.MOE_ERR_UNSUPPORTED
-    assert lib.moe_plan_blocks(cfg, ok, 16, *[ok] * 8, None) == N.MOE_ERR_INVALID_ARG
+    for bad_mask in (1 << 5, 1 << 7, 1 << 16, 0xFFFFFFFF):  # only variants 0..4 and u_min
+        assert lib.moe_plan_blocks(cfg, ok, bad_mask, *[ok] * 8, None) == N.MOE_ERR_INVALID_ARG
     assert lib.moe_expert_ffn(cfg, *[ok] * 7, 16, *[ok] * 3, None) == N.MOE_ERR_INVALID_ARG
     bad_d = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(d=320)))
     assert lib.moe_expert_ffn(bad_d, *[ok] * 7, 0, *[ok] * 3, None) == N.MOE_ERR_UNSUPPORTED
@@ -117,3 +118,17 @@ def test_layer_api_surface():
         assert callable(getattr(MoeLayer, name)), name
     for name in ("submit", "drain"):
         assert callable(getattr(HostPipeline, name)), name
+
+
+def test_header_constants_match_binding():
+    """plan_info indices, FFN modes and error codes: the header's enums and the binding's
+    constants are the same numbers."""
+    import re
+    text = open(N.HEADER_PATH).read()
+    enum = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(MOE_\w+)\s*=\s*(-?\d+)", text)}
+    for key, val in N.PI.items():
+        assert enum["MOE_PI_" + key] == val, key
+    for name in ("MOE_FFN_FUSED_COMBINE", "MOE_FFN_WRITE_O", "MOE_FFN_STRICT_SLOTS",
+                 "MOE_FFN_SM_PAIR", "MOE_FFN_GATHER_X", "MOE_ERR_TOO_LARGE"):
+        assert enum[name] == getattr(N, name), name
+    assert N.variant_mask() == 0 and N.variant_mask([4], u_min=3) == (1 << 4) | (3 << 8)

@@ -26,6 +26,9 @@ SMALL = [
 ]
 
 
+ALL5 = N.variant_mask(range(N.N_VARIANTS))
+
+
 def _wl(name):
     return WORKLOADS[name] if isinstance(name, str) else name
 
@@ -37,7 +40,7 @@ def test_route_hist_and_plan_and_dispatch(case):
     layer = MoeLayer(wl, "cuda", gather_x=False)  # materialise Xp to check its rows
     layer.clear_status()
     layer.route(logits.cuda())
-    layer.plan(0)
+    layer.plan(ALL5)
     layer.dispatch(x.cuda())
     torch.cuda.synchronize()
     assert layer.read_status() == 0
@@ -58,7 +61,7 @@ def test_route_hist_and_plan_and_dispatch(case):
     b = O.block_counts(counts_ref, wl.beta)
     boff = O.block_offsets(b)
     assert layer.view("block_off").cpu().tolist() == boff
-    ref = O.plan(b, wl.P, wl.s)
+    ref = O.plan(b, wl.P, wl.s, variant_mask=ALL5)  # all five variants, best kept
     q = layer.view("q").cpu().numpy()
     assert np.array_equal(q, ref["q"])
     pi = layer.plan_info.cpu().tolist()
@@ -66,9 +69,11 @@ def test_route_hist_and_plan_and_dispatch(case):
     assert pi[N.PI["MAKESPAN"]] == ref["makespan"] and pi[N.PI["VARIANT"]] == ref["variant"]
     assert pi[N.PI["REPLICAS"]] == ref["replicas"] and pi[N.PI["ROUNDS"]] == ref["rounds"]
     assert pi[N.PI["FIXED_MAKESPAN"]] == ref["fixed_makespan"]
-    for v in range(4):
+    for v in range(N.N_VARIANTS):
         assert pi[N.PI["VAR_MAKESPAN"] + v] == ref["all"][v]["makespan"]
         assert pi[N.PI["VAR_REPLICAS"] + v] == ref["all"][v]["replicas"]
+        assert pi[N.PI["VAR_ROUNDS"] + v] == ref["all"][v]["rounds"]
+    assert pi[N.PI["QUOTA_TAU"]] == ref["all"][N.QUOTA_VARIANT]["tau_star"]
     assert layer.view("slot_load").cpu().tolist() == ref["load"]
     blocks_ref, slot_off_ref = O.block_list(ref["q"])
     assert layer.view("slot_off").cpu().tolist() == slot_off_ref
@@ -111,15 +116,19 @@ def test_planner_every_variant_bit_exact(E, P):
         layer = MoeLayer(wl, "cuda")
         layer.counts[:E] = torch.from_numpy(counts).cuda()
         b = O.block_counts(counts, beta)
-        for v in range(4):
+        # the four greedy searches, then the quota solver with three quota floors
+        for v, u_min in [(0, 1), (1, 1), (2, 1), (3, 1), (4, 1), (4, 2), (4, 7)]:
             layer.clear_status()
-            layer.plan(1 << v)
+            layer.plan(N.variant_mask([v], u_min=u_min))
             torch.cuda.synchronize()
-            ref = O.plan_variant(b, P, s, v)
-            assert np.array_equal(layer.view("q").cpu().numpy(), ref["q"]), (E, P, s, v)
+            ref = O.plan_variant(b, P, s, v) if v < 4 else O.plan_quota(b, P, s, u_min)
+            assert np.array_equal(layer.view("q").cpu().numpy(), ref["q"]), (E, P, s, v, u_min)
             pi = layer.plan_info.cpu().tolist()
             assert pi[N.PI["MAKESPAN"]] == ref["makespan"] and pi[N.PI["VARIANT"]] == v
+            assert pi[N.PI["REPLICAS"]] == ref["replicas"]
             assert pi[N.PI["ROUNDS"]] == ref["rounds"]
+            if v == 4:
+                assert pi[N.PI["QUOTA_TAU"]] == ref["tau_star"]
             assert layer.read_status() == 0
 
 

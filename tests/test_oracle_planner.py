@@ -63,8 +63,10 @@ def test_constraints_and_bounds_random(E, P, s):
             assert res["q"].sum(axis=0).tolist() == res["load"]
             assert tau <= res["makespan"] <= fixed
             assert res["tau"] == tau and res["B"] == B
-        best = O.plan(b, P, s)
-        assert best["makespan"] == min(O.plan_variant(b, P, s, v)["makespan"] for v in range(4))
+        greedy = min(O.plan_variant(b, P, s, v)["makespan"] for v in range(4))
+        assert O.plan(b, P, s)["makespan"] == greedy          # default: the greedy searches
+        assert O.plan(b, P, s, variant_mask=O.ALL_VARIANTS)["makespan"] == min(
+            greedy, O.plan_quota(b, P, s)["makespan"])
 
 
 def test_zero_budget_is_fixed_placement():
