@@ -95,6 +95,8 @@ enum {
   MOE_PI_VAR_REPLICAS = 22,  /* 5 entries */
   MOE_PI_VAR_ROUNDS = 27,    /* 5 entries */
   MOE_PI_QUOTA_TAU = 32,     /* threshold the quota solver's search ended on (-1: off) */
+  MOE_PI_COST = 33,          /* C_lambda of the chosen plan (-1: not reduction-aware) */
+  MOE_PI_VAR_COST = 34,      /* 5 entries: C_lambda per variant (-1: off) */
   MOE_PI_LEN = 40
 };
 
@@ -147,8 +149,13 @@ MOE_API int moe_route_hist(const moe_cfg* cfg, const float* logits, int32_t* top
  *                solver ("UltraEP" notes, section 4, Algorithm 1: binary search on the
  *                threshold with a greedy feasibility oracle); bits 0..4 all clear means
  *                the four greedy variants (the method's planner; 0x1F runs all five).
- *                Bits 8..15: the quota solver's floor u_min in blocks (0 means 1).  Other
- *                bits are invalid.
+ *                Bit 5: reduction-aware selection for backward with the proxy
+ *                C_lambda(q) = max_r (l_r + lambda n_r), n_r = remote copies of slot r's
+ *                experts ("Methodology" 1): each greedy search returns its plan of least
+ *                C_lambda (its start or the plan after some move) and the variant of least
+ *                (C_lambda, makespan, replicas, v) wins.  Bits 8..15: the quota solver's
+ *                floor u_min in blocks (0 means 1).  Bits 16..23: lambda (0 means 12).
+ *                Other bits are invalid.
  *   block_off    int32 [E+1]: exclusive prefix sum of b_e = ceil(c_e / beta).
  *   q            int32 [E, P] row-major: blocks of expert e run by slot r, of the best
  *                enabled variant (least makespan, then fewest replicas, then lowest v).

@@ -15,7 +15,9 @@ Sources (cited by page title and section; the pages print no code and no worked 
           - Methodology 1, "Bounded Greedy Search": four greedy searches from the
             no-replica assignment toward tau = ceil(sum_e b_e / P), donor priority
             (total overload | largest remaining home-expert load) x fan-out (one new copy
-            per expert per round | several);
+            per expert per round | several); the reduction-aware proxy
+            C_lambda(q) = max_r (l_r + lambda n_r), n_r = remote replicas of experts owned
+            by r, lambda = 12;
           - Methodology 2, expert-computation equation: Z_e = X_e W1_e, Z_e = [G_e, U_e],
             A_e = SiLU(G_e) * U_e, O_e = A_e W2_e, y_t = sum_{e in S_t} p_{t,e} O_e[t];
           - Summary and "Theoretical Contributions" 1: router outputs, token counts,
@@ -51,6 +53,11 @@ Readings where the pages leave a step open (each is also listed in the design no
       receivers are ranks other than the donor with slack > 0 and a free replica slot
       (rep_t < s), ties of slack to the lower rank; u_min is counted in blocks (default 1);
       the plan is the oracle's quota table at the tau the search ends on.
+  R9  the reduction-aware variant (C_lambda) keeps each greedy search's moves and returns
+      the plan, among the search's start and the plan after each move, of least C_lambda
+      (the earliest on ties; n_r grows by one whenever a move opens a copy of one of r's
+      experts); the quota solver's plan is scored as it ends; the best variant is then
+      the least (C_lambda, makespan, replicas, variant index).
 """
 from __future__ import annotations
 
@@ -126,8 +133,22 @@ def owner(e: int, E: int, P: int) -> int:
 
 
 # --------------------------------------------------------------------------- planner
-def plan_variant(b, P: int, s: int, v: int) -> dict:
-    """One bounded greedy search of [MF] "Bounded Greedy Search"; reading R4.
+def reduction_cost(q, P: int, lam: int) -> int:
+    """[MF] C_lambda(q) = max_r (l_r + lambda n_r), n_r = the remote replicas of experts
+    owned by r: #{(e, t) : h(e) = r, t != r, q_et > 0}."""
+    q = np.asarray(q)
+    E = q.shape[0]
+    n = [0] * P
+    for e in range(E):
+        h = owner(e, E, P)
+        n[h] += sum(1 for t in range(P) if t != h and q[e, t] > 0)
+    loads = q.sum(axis=0)
+    return max(int(loads[r]) + lam * n[r] for r in range(P)) if P else 0
+
+
+def plan_variant(b, P: int, s: int, v: int, lam: int | None = None) -> dict:
+    """One bounded greedy search of [MF] "Bounded Greedy Search"; reading R4 (and with
+    `lam`, the reduction-aware variant of reading R9).
 
     Variant v = 2*D + F with donor priority D (0: decreasing total overload l_r,
     1: largest remaining home-expert load max_{h(e)=r} q_er) and fan-out F (0: at most
@@ -161,6 +182,11 @@ def plan_variant(b, P: int, s: int, v: int) -> dict:
     B = sum(b)
     tau = -(-B // P)
     rounds = 0
+    # reading R9: the least C_lambda along the search (start, then after every move)
+    best = None
+    if lam is not None:
+        best = {"cost": reduction_cost(q, P, lam), "q": [row[:] for row in q],
+                "load": load[:], "rep": rep[:], "rounds": 0}
     while max(load) > tau:
         rounds += 1
         newcopies = [0] * E
@@ -191,11 +217,21 @@ def plan_variant(b, P: int, s: int, v: int) -> dict:
                     load[r] -= delta
                     load[t] += delta
                     progress = True
+                    if best is not None:
+                        c = reduction_cost(q, P, lam)
+                        if c < best["cost"]:
+                            best = {"cost": c, "q": [row[:] for row in q], "load": load[:],
+                                    "rep": rep[:], "rounds": rounds}
         if not progress:
             break
-    return {"q": np.array(q, dtype=np.int32).reshape(E, P), "load": load,
-            "makespan": max(load) if P else 0, "replicas": sum(rep), "tau": tau,
-            "B": B, "variant": v, "rounds": rounds}
+    out = {"q": np.array(q, dtype=np.int32).reshape(E, P), "load": load,
+           "makespan": max(load) if P else 0, "replicas": sum(rep), "tau": tau,
+           "B": B, "variant": v, "rounds": rounds}
+    if best is not None:
+        out.update(q=np.array(best["q"], dtype=np.int32).reshape(E, P), load=best["load"],
+                   makespan=max(best["load"]) if P else 0, replicas=sum(best["rep"]),
+                   rounds=best["rounds"], cost=best["cost"])
+    return out
 
 
 def quota_feasible(b, P: int, s: int, u_min: int, tau: int) -> dict:
@@ -275,16 +311,23 @@ def fixed_makespan(b, P: int) -> int:
     return max(load)
 
 
-def plan(b, P: int, s: int, variant_mask: int = GREEDY_VARIANTS, u_min: int = 1) -> dict:
+def plan(b, P: int, s: int, variant_mask: int = GREEDY_VARIANTS, u_min: int = 1,
+         lam: int | None = None) -> dict:
     """Run the enabled variants (bits 0..3: the greedy searches, bit 4: the quota solver;
     0 means the four greedy searches, the method's planner) and keep the best.  Reading
     R4: the best is the lexicographic minimum of (makespan, total replicas, variant
-    index)."""
+    index); with `lam` (reading R9), of (C_lambda, makespan, replicas, variant index)."""
     mask = variant_mask & ALL_VARIANTS or GREEDY_VARIANTS
-    results = [plan_variant(b, P, s, v) for v in range(4) if mask >> v & 1]
+    results = [plan_variant(b, P, s, v, lam) for v in range(4) if mask >> v & 1]
     if mask >> QUOTA_VARIANT & 1:
         results.append(plan_quota(b, P, s, u_min))
-    best = min(results, key=lambda r: (r["makespan"], r["replicas"], r["variant"]))
+        if lam is not None:
+            results[-1]["cost"] = reduction_cost(results[-1]["q"], P, lam)
+    if lam is None:
+        best = min(results, key=lambda r: (r["makespan"], r["replicas"], r["variant"]))
+    else:
+        best = min(results, key=lambda r: (r["cost"], r["makespan"], r["replicas"],
+                                           r["variant"]))
     out = dict(best)
     out["all"] = {r["variant"]: r for r in results}
     out["fixed_makespan"] = fixed_makespan(b, P)

@@ -69,7 +69,7 @@ int moe_plan_blocks(const moe_cfg* cfg, const int32_t* counts, uint32_t variant_
                     moe_stream_t stream) {
   int rc = check_cfg(cfg);
   if (rc != MOE_OK) return rc;
-  if (variant_mask & ~0xFF1Fu) return MOE_ERR_INVALID_ARG;  // variants 0..4, u_min
+  if (variant_mask & ~0xFFFF3Fu) return MOE_ERR_INVALID_ARG;  // variants, C_lambda, u_min, lambda
   rc = check_ptrs({counts, block_off, q, slot_load, slot_off, blocks, tiles, plan_info, status});
   if (rc != MOE_OK) return rc;
   return cuda_result(launch_plan(*cfg, counts, variant_mask, block_off, q, slot_load, slot_off,

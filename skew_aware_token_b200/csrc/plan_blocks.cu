@@ -29,6 +29,13 @@
 // slot), of delta = min(excess, slack, b_e) blocks, made only if delta >= u_min; tau is
 // feasible when no excess is left.  The plan is the oracle's quota table at the final tau.
 //
+// Reduction-aware selection (the summary's proxy for backward, C_lambda(q) = max_r (l_r +
+// lambda n_r), n_r = remote copies of slot r's experts): each greedy search keeps its
+// moves and returns the plan of least C_lambda among its start and the plan after each
+// move (the earliest on ties; found by tracking C_lambda, then replaying the search up to
+// that move); the quota solver's plan is scored as it ends; the best variant is the least
+// (C_lambda, makespan, replicas, variant).
+//
 // One warp runs one variant: slot-parallel work (candidate test, arg-min, maxima) uses
 // lanes 0..P-1 and warp shuffles; expert-parallel work strides the lanes over experts.
 // Lane 0 applies each move; __syncwarp() orders it against the next read.
@@ -86,9 +93,14 @@ __device__ __forceinline__ int min8(int v) {
 // Runs greedy variant v on the calling warp; returns (makespan, replicas, rounds) in lane 0.
 // Lane t < P holds slot t's load and replica count in registers; q lives in shared memory
 // and, while one expert moves, each lane touches only its own slot's entry.
+// lam >= 0 (the reduction-aware proxy C = max_r (l_r + lam n_r), n_r = remote copies of
+// slot r's experts): also tracks C after every move and returns the least C seen, the move
+// count and round where it was first reached (start: 0, 0).  max_moves >= 0: the search
+// stops before move max_moves + 1, leaving the plan after max_moves moves in q.
 __device__ void greedy_variant(int v, int E, int P, int s, int tau, const int* b,
-                               VariantState st, int* out_makespan, int* out_replicas,
-                               int* out_rounds) {
+                               VariantState st, int lam, int max_moves, int* out_makespan,
+                               int* out_replicas, int* out_rounds, int* out_best_cost,
+                               int* out_best_moves, int* out_best_rounds) {
   const int lane = threadIdx.x & 31;
   const int D = v >> 1, F = v & 1;
   int* q = st.q;
@@ -101,8 +113,11 @@ __device__ void greedy_variant(int v, int E, int P, int s, int tau, const int* b
     for (int e = home_lo(lane, E, P); e < home_lo(lane + 1, E, P); ++e) load += b[e];
   __syncwarp();
 
-  int rounds = 0;
-  while (true) {
+  int rounds = 0, moves = 0, nown = 0;  // nown, lane r: remote copies of r's experts
+  int best_cost = lam >= 0 ? warp_max(lane < P ? load : INT_MIN) : 0;
+  int best_moves = 0, best_rounds = 0;
+  bool halt = false;
+  while (!halt) {
     const int maxload = warp_max(lane < P ? load : INT_MIN);
     if (maxload <= tau) break;
     ++rounds;
@@ -129,7 +144,7 @@ __device__ void greedy_variant(int v, int E, int P, int s, int tau, const int* b
     __syncwarp();
 
     bool progress = false;
-    for (int di = 0; di < ndon; ++di) {
+    for (int di = 0; di < ndon && !halt; ++di) {
       const int r = st.donors[di];
       const int lo = home_lo(r, E, P), n = home_lo(r + 1, E, P) - lo;
       // home experts by (q[e][r] desc, e asc)
@@ -144,12 +159,16 @@ __device__ void greedy_variant(int v, int E, int P, int s, int tau, const int* b
       }
       __syncwarp();
       int lr = __shfl_sync(kFull, load, r);  // donor load, warp-uniform
-      for (int oi = 0; oi < n && lr > tau; ++oi) {
+      for (int oi = 0; oi < n && lr > tau && !halt; ++oi) {
         const int e = st.order[oi];
         int qer = q[e * P + r];              // donor's blocks of e, warp-uniform
         int qt = lane < P ? q[e * P + lane] : 0;
         int newc = 0;                        // copies of e opened in this round
         while (lr > tau && qer > 0) {
+          if (moves == max_moves) {
+            halt = true;
+            break;
+          }
           int ck = INT_MAX;
           if (lane < P && lane != r && load < tau &&
               (qt > 0 || (rep < s && (F || newc == 0))))
@@ -167,11 +186,21 @@ __device__ void greedy_variant(int v, int E, int P, int s, int tau, const int* b
           if (lane == r) {
             load -= delta;
             qt -= delta;
+            nown += opened ? 1 : 0;  // r owns e: only home blocks move
           }
           newc += opened ? 1 : 0;
           lr -= delta;
           qer -= delta;
           progress = true;
+          ++moves;
+          if (lam >= 0) {
+            const int c = warp_max(lane < P ? load + lam * nown : INT_MIN);
+            if (c < best_cost) {
+              best_cost = c;
+              best_moves = moves;
+              best_rounds = rounds;
+            }
+          }
         }
         if (lane < P) q[e * P + lane] = qt;
         __syncwarp();
@@ -187,6 +216,9 @@ __device__ void greedy_variant(int v, int E, int P, int s, int tau, const int* b
     *out_makespan = mk;
     *out_replicas = reps;
     *out_rounds = rounds;
+    *out_best_cost = best_cost;
+    *out_best_moves = lam >= 0 ? best_moves : moves;
+    *out_best_rounds = lam >= 0 ? best_rounds : rounds;
   }
   __syncwarp();
 }
@@ -208,8 +240,8 @@ __device__ __forceinline__ int order_donors(bool is_donor, int key, int P, int* 
 // Runs the quota solver on the calling warp; the plan lands in st.q.  Lane t < P holds
 // slot t's home load, and during an oracle pass its load and replica count.
 __device__ void quota_variant(int E, int P, int s, int u_min, int B, const int* b,
-                              VariantState st, int* out_makespan, int* out_replicas,
-                              int* out_rounds, int* out_tau) {
+                              VariantState st, int lam, int* out_makespan, int* out_replicas,
+                              int* out_rounds, int* out_tau, int* out_cost) {
   const int lane = threadIdx.x & 31;
   constexpr int kBig = 1 << 26;  // slack < B < 2^17; (kBig - slack) << 4 | slot fits an int
   // each slot's home experts by (b_e desc, e asc), at st.order[home_lo(r) ..)
@@ -232,9 +264,11 @@ __device__ void quota_variant(int E, int P, int s, int u_min, int B, const int* 
 
   // One oracle pass at tau: returns feasibility; load / rep end in the lanes' registers;
   // with `write`, the transfers are applied to st.q (which then holds the home placement).
+  int nown = 0;  // lane r: transfers of r's experts (remote copies), counted in each pass
   auto oracle = [&](int tau, bool write, int& load, int& rep) -> bool {
     load = lane < P ? home : 0;
     rep = 0;
+    nown = 0;
     const int ndon = order_donors(lane < P && load > tau, load, P, st.donors);
     bool stuck = false;  // no slot can receive any more
     for (int di = 0; di < ndon && !stuck; ++di) {
@@ -258,7 +292,10 @@ __device__ void quota_variant(int E, int P, int s, int u_min, int B, const int* 
             load += delta;
             rep += 1;
           }
-          if (lane == r) load -= delta;
+          if (lane == r) {
+            load -= delta;
+            nown += 1;
+          }
           exc -= delta;
           if (write && lane == 0) {
             st.q[e * P + r] -= delta;
@@ -288,19 +325,21 @@ __device__ void quota_variant(int E, int P, int s, int u_min, int B, const int* 
   __syncwarp();
   const int mk = warp_max(lane < P ? load : 0);
   const int reps = warp_sum(lane < P ? rep : 0);
+  const int cost = lam >= 0 ? warp_max(lane < P ? load + lam * nown : INT_MIN) : -1;
   if (lane < P) st.load[lane] = load;
   if (lane == 0) {
     *out_makespan = mk;
     *out_replicas = reps;
     *out_rounds = rounds;
     *out_tau = hi;
+    *out_cost = cost;
   }
   __syncwarp();
 }
 
 __global__ void __launch_bounds__(kPlanThreads, 1)
 plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
-            unsigned mask, int u_min, int b_max, int32_t* __restrict__ block_off, int32_t* __restrict__ q_out,
+            unsigned mask, int u_min, int lam, int b_max, int32_t* __restrict__ block_off, int32_t* __restrict__ q_out,
             int32_t* __restrict__ slot_load, int32_t* __restrict__ slot_off,
             int32_t* __restrict__ blocks, int32_t* __restrict__ tiles,
             int32_t* __restrict__ plan_info, int32_t* __restrict__ status) {
@@ -311,8 +350,10 @@ plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
   int* loadv = qv + kVariants * E * P;  // 5 * 8
   int* order = loadv + kVariants * kMaxP;  // 5 * E
   int* donors = order + kVariants * E;  // 5 * 8
-  int* res = donors + kVariants * kMaxP;  // 16: makespan[5], replicas[5], rounds[5], tau*
-  int* misc = res + 16;                 // [0] B, [1] tau, [2] best, [3..3+P] slot tile offsets
+  // res: makespan[5], replicas[5], rounds[5], quota tau*, C_lambda[5], 3 spare, then per
+  // greedy warp (C_lambda, moves, round) at its least C_lambda
+  int* res = donors + kVariants * kMaxP;  // 40
+  int* misc = res + 40;                 // [0] B, [1] tau, [2] best, [3..3+P] slot tile offsets
                                         // [12..12+P] slot_off, [24..] fixed loads (P)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -351,29 +392,55 @@ plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
     st.load = loadv + warp * kMaxP;
     st.order = order + warp * E;
     st.donors = donors + warp * kMaxP;
+    int* cost = res + 16;
     if (!(mask >> warp & 1u)) {
       if (lane == 0) {
         res[warp] = INT_MAX;
         res[kVariants + warp] = INT_MAX;
         res[2 * kVariants + warp] = 0;
+        cost[warp] = INT_MAX;
         if (warp == kQuota) res[3 * kVariants] = -1;
       }
     } else if (warp == kQuota) {
-      quota_variant(E, P, s, u_min, B, b, st, &res[warp], &res[kVariants + warp],
-                    &res[2 * kVariants + warp], &res[3 * kVariants]);
+      quota_variant(E, P, s, u_min, B, b, st, lam, &res[warp], &res[kVariants + warp],
+                    &res[2 * kVariants + warp], &res[3 * kVariants], &cost[warp]);
     } else {
-      greedy_variant(warp, E, P, s, tau, b, st, &res[warp], &res[kVariants + warp],
-                     &res[2 * kVariants + warp]);
+      int* aux = res + 24 + 3 * warp;
+      greedy_variant(warp, E, P, s, tau, b, st, lam, -1, &res[warp], &res[kVariants + warp],
+                     &res[2 * kVariants + warp], &aux[0], &aux[1], &aux[2]);
+      if (lam >= 0) {
+        // replay the search up to its least C_lambda (the plan after aux[1] moves)
+        const int bc = aux[0], bm = aux[1], br = aux[2];
+        __syncwarp();
+        greedy_variant(warp, E, P, s, tau, b, st, -1, bm, &res[warp], &res[kVariants + warp],
+                       &aux[0], &aux[0], &aux[1], &aux[2]);
+        if (lane == 0) {
+          res[2 * kVariants + warp] = br;
+          cost[warp] = bc;
+        }
+      } else if (lane == 0) {
+        cost[warp] = -1;
+      }
+      __syncwarp();
     }
   }
   __syncthreads();
 
-  // ---- best variant: least (makespan, replicas, v)
+  // ---- best variant: least (makespan, replicas, v), or (C_lambda, makespan, replicas, v)
   if (tid == 0) {
+    const int* cost = res + 16;
     int best = -1;
     for (int v = 0; v < kVariants; ++v) {
       if (!(mask >> v & 1u)) continue;
-      if (best < 0 || res[v] < res[best] ||
+      if (best < 0) {
+        best = v;
+        continue;
+      }
+      if (lam >= 0 && cost[v] != cost[best]) {
+        if (cost[v] < cost[best]) best = v;
+        continue;
+      }
+      if (res[v] < res[best] ||
           (res[v] == res[best] && res[kVariants + v] < res[kVariants + best]))
         best = v;
     }
@@ -433,7 +500,10 @@ plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
       plan_info[MOE_PI_VAR_ROUNDS + v] = on ? res[2 * kVariants + v] : -1;
     }
     plan_info[MOE_PI_QUOTA_TAU] = res[3 * kVariants];
-    for (int i = MOE_PI_QUOTA_TAU + 1; i < MOE_PI_LEN; ++i) plan_info[i] = 0;
+    plan_info[MOE_PI_COST] = lam >= 0 ? res[16 + best] : -1;
+    for (int v = 0; v < kVariants; ++v)
+      plan_info[MOE_PI_VAR_COST + v] = (lam >= 0 && (mask >> v & 1u)) ? res[16 + v] : -1;
+    for (int i = MOE_PI_VAR_COST + kVariants; i < MOE_PI_LEN; ++i) plan_info[i] = 0;
   }
   __syncthreads();
 
@@ -480,7 +550,7 @@ cudaError_t launch_plan(const moe_cfg& c, const int32_t* counts, uint32_t mask,
                         int32_t* plan_info, int32_t* status, cudaStream_t st) {
   const int E = c.E, P = c.P;
   const size_t words = (size_t)E + (E + 1) + kVariants * ((size_t)E * P + kMaxP + E + kMaxP) +
-                       16 + 40;
+                       40 + 40;
   const size_t bytes = words * sizeof(int);
   if (bytes > 48 * 1024) {
     cudaError_t err = cudaFuncSetAttribute(plan_kernel,
@@ -491,7 +561,8 @@ cudaError_t launch_plan(const moe_cfg& c, const int32_t* counts, uint32_t mask,
   const unsigned all = (1u << kVariants) - 1u;
   const unsigned m = (mask & all) ? (mask & all) : 0xFu;  // default: the four greedy searches
   const int u_min = (mask >> 8 & 0xFFu) ? (int)(mask >> 8 & 0xFFu) : 1;
-  plan_kernel<<<1, kPlanThreads, bytes, st>>>(counts, E, P, c.s, c.beta, m, u_min,
+  const int lam = !(mask >> 5 & 1u) ? -1 : (mask >> 16 & 0xFFu) ? (int)(mask >> 16 & 0xFFu) : 12;
+  plan_kernel<<<1, kPlanThreads, bytes, st>>>(counts, E, P, c.s, c.beta, m, u_min, lam,
                                               (int)max_blocks(c), block_off, q, slot_load,
                                               slot_off, blocks, tiles, plan_info, status);
   return cudaGetLastError();

@@ -26,14 +26,15 @@ MOE_FFN_FUSED_COMBINE, MOE_FFN_WRITE_O, MOE_FFN_STRICT_SLOTS, MOE_FFN_SM_PAIR = 
 MOE_FFN_GATHER_X = 8
 PI = dict(B=0, TAU=1, MAKESPAN=2, VARIANT=3, NTILES=4, FIXED_MAKESPAN=5, REPLICAS=6,
           ROUNDS=7, SLOT_TILE_OFF=8, VAR_MAKESPAN=17, VAR_REPLICAS=22, VAR_ROUNDS=27,
-          QUOTA_TAU=32, LEN=40)
+          QUOTA_TAU=32, COST=33, VAR_COST=34, LEN=40)
 N_VARIANTS = 5          # planner variants: 0..3 bounded greedy, 4 quota solver
 QUOTA_VARIANT = 4
 
 
-def variant_mask(variants=(), u_min: int = 1) -> int:
-    """moe_plan_blocks's variant_mask: enabled variants (none = all five) and the quota
-    solver's floor u_min in blocks."""
+def variant_mask(variants=(), u_min: int = 1, lam: int | None = None) -> int:
+    """moe_plan_blocks's variant_mask: enabled variants (none = the four greedy searches),
+    the quota solver's floor u_min in blocks and, with `lam`, reduction-aware selection
+    with that lambda (1..255; 12 on the pages)."""
     m = 0
     for v in variants:
         m |= 1 << v
@@ -41,6 +42,10 @@ def variant_mask(variants=(), u_min: int = 1) -> int:
         raise ValueError("u_min must be in 1..255 blocks")
     if u_min != 1:
         m |= u_min << 8
+    if lam is not None:
+        if not 1 <= lam <= 255:
+            raise ValueError("lambda must be in 1..255")
+        m |= 1 << 5 | (0 if lam == 12 else lam << 16)
     return m
 
 

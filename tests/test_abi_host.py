@@ -91,7 +91,7 @@ def test_null_and_misaligned_pointers_rejected():
     assert lib.moe_dispatch_permute(cfg, *disp, None) == N.MOE_ERR_INVALID_ARG
     disp[4], disp[5] = ok + 8, ok
     assert lib.moe_dispatch_permute(cfg, *disp, None) == N.MOE_ERR_UNSUPPORTED
-    for bad_mask in (1 << 5, 1 << 7, 1 << 16, 0xFFFFFFFF):  # only variants 0..4 and u_min
+    for bad_mask in (1 << 6, 1 << 7, 1 << 24, 0xFFFFFFFF):  # bits 6, 7 and 24..31 are unused
         assert lib.moe_plan_blocks(cfg, ok, bad_mask, *[ok] * 8, None) == N.MOE_ERR_INVALID_ARG
     assert lib.moe_expert_ffn(cfg, *[ok] * 7, 16, *[ok] * 3, None) == N.MOE_ERR_INVALID_ARG
     bad_d = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(d=320)))

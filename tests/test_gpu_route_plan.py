@@ -132,6 +132,52 @@ def test_planner_every_variant_bit_exact(E, P):
             assert layer.read_status() == 0
 
 
+@pytest.mark.parametrize("E,P", [(8, 4), (64, 8), (256, 8), (12, 5), (256, 2)])
+def test_reduction_aware_plans_bit_exact(E, P):
+    """C_lambda selection: every variant's least-C_lambda plan and the best of five."""
+    rng = np.random.default_rng(E * 7 + P)
+    for trial in range(5):
+        s = [1, 2, 4, 3, E][trial]
+        beta = (64, 128)[trial % 2]
+        zipf = 1.0 / np.arange(1, E + 1) ** rng.uniform(0.5, 2.5)
+        T = int(rng.integers(100, 3000))
+        k = int(min(E, 8))
+        counts = rng.multinomial(T * k, zipf / zipf.sum()).astype(np.int32)
+        wl = Workload("rand", T=T, d=256, E=E, k=k, f=128, beta=beta, P=P, s=s)
+        layer = MoeLayer(wl, "cuda")
+        layer.counts[:E] = torch.from_numpy(counts).cuda()
+        b = O.block_counts(counts, beta)
+        for lam in (3, 12):
+            for v in range(N.N_VARIANTS):
+                layer.clear_status()
+                layer.plan(N.variant_mask([v], lam=lam))
+                torch.cuda.synchronize()
+                if v < 4:
+                    ref = O.plan_variant(b, P, s, v, lam)
+                else:
+                    ref = O.plan_quota(b, P, s)
+                    ref["cost"] = O.reduction_cost(ref["q"], P, lam)
+                assert np.array_equal(layer.view("q").cpu().numpy(), ref["q"]), (E, P, s, v, lam)
+                pi = layer.plan_info.cpu().tolist()
+                assert pi[N.PI["COST"]] == ref["cost"] and pi[N.PI["VARIANT"]] == v
+                assert pi[N.PI["MAKESPAN"]] == ref["makespan"]
+                assert pi[N.PI["REPLICAS"]] == ref["replicas"]
+                assert pi[N.PI["ROUNDS"]] == ref["rounds"]
+                assert layer.read_status() == 0
+            layer.plan(N.variant_mask(range(N.N_VARIANTS), lam=lam))
+            torch.cuda.synchronize()
+            ref = O.plan(b, P, s, variant_mask=O.ALL_VARIANTS, lam=lam)
+            assert np.array_equal(layer.view("q").cpu().numpy(), ref["q"])
+            pi = layer.plan_info.cpu().tolist()
+            assert pi[N.PI["VARIANT"]] == ref["variant"] and pi[N.PI["COST"]] == ref["cost"]
+            assert pi[N.PI["VAR_COST"]:N.PI["VAR_COST"] + 5] == [ref["all"][v]["cost"]
+                                                                for v in range(5)]
+            # the tile list follows the chosen plan
+            nt = pi[N.PI["NTILES"]]
+            want, _ = expected_tiles(ref["q"], O.block_offsets(b), beta)
+            assert [tuple(r) for r in layer.view("tiles")[:nt].cpu().tolist()] == want
+
+
 def test_plan_is_deterministic():
     wl = WORKLOADS["dsv3_a1"]
     logits, _ = host_inputs(wl)
