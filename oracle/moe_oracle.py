@@ -20,6 +20,9 @@ Sources (cited by page title and section; the pages print no code and no worked 
             by r, lambda = 12;
           - Methodology 2, expert-computation equation: Z_e = X_e W1_e, Z_e = [G_e, U_e],
             A_e = SiLU(G_e) * U_e, O_e = A_e W2_e, y_t = sum_{e in S_t} p_{t,e} O_e[t];
+          - Methodology 2, "Backward gradients": dA_e = D_e W2_e^T, dX_e = dZ_e W1_e^T,
+            dW2_e = A_e^T D_e, dW1_e = X_e^T dZ_e; Backward item 3: token-axis D_e and
+            dZ_e are requantized;
           - Summary and "Theoretical Contributions" 1: router outputs, token counts,
             expert selections and routing weights are preserved.
   [UE]  "UltraEP: Exact Load Balancing for Rack-Scale MoE" reading notes, section 4
@@ -58,6 +61,13 @@ Readings where the pages leave a step open (each is also listed in the design no
       (the earliest on ties; n_r grows by one whenever a move opens a copy of one of r's
       experts); the quota solver's plan is scored as it ends; the best variant is then
       the least (C_lambda, makespan, replicas, variant index).
+  R10 backward: D = dL/dO on row r is row_gate[r] * dy[row_token[r]] (zero on padding
+      rows); the weights are stored w1 [2f, d], w2 [d, f], so each page formula is taken
+      with that transpose (dA = D w2, dX = dZ w1, dW2 = D^T A, dW1 = dZ^T X);
+      dZ = [dA * U * SiLU'(G), dA * SiLU(G)]; D and dZ are requantized to bf16
+      (round to nearest even) before they enter a product, everything else is fp32;
+      dx_t = sum_j dX[tok_row[t, j]], j ascending.  The gate gradient (router backward)
+      is not part of the expert computation and is left out.
 """
 from __future__ import annotations
 
@@ -396,19 +406,59 @@ def gather_rows(x: np.ndarray, row_token: np.ndarray) -> np.ndarray:
 def silu(g: np.ndarray) -> np.ndarray:
     """SiLU(g) = g / (1 + exp(-g))."""
     with np.errstate(over="ignore"):
-        return g / (np.float32(1.0) + np.exp(-g))
+        return g / (g.dtype.type(1.0) + np.exp(-g))
 
 
-def expert_ffn(x_rows: np.ndarray, w1: np.ndarray, w2: np.ndarray) -> np.ndarray:
+def silu_grad(g: np.ndarray) -> np.ndarray:
+    """d SiLU(g) / dg = s + g s (1 - s) with s = 1 / (1 + exp(-g))."""
+    one = g.dtype.type(1.0)
+    with np.errstate(over="ignore"):
+        sg = one / (one + np.exp(-g))
+    return sg * (one + g * (one - sg))
+
+
+def round_bf16(a: np.ndarray) -> np.ndarray:
+    """fp32 -> nearest bf16 value (ties to even), returned as fp32 (finite inputs)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    u = (u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))) & np.uint32(0xFFFF0000)
+    return u.view(np.float32)
+
+
+def expert_ffn(x_rows: np.ndarray, w1: np.ndarray, w2: np.ndarray,
+               dtype=np.float32) -> np.ndarray:
     """O_e = (SiLU(G_e) * U_e) W2_e for rows of one expert; [MF] expert-computation
     equation; reading R6.  Shapes: x_rows [n, d], w1 [2f, d] (rows: G then U),
-    w2 [d, f]; all fp32.  Returns O [n, d] fp32."""
-    x_rows = np.asarray(x_rows, dtype=np.float32)
+    w2 [d, f]; all fp32 (fp64 with dtype=np.float64).  Returns O [n, d]."""
+    x_rows = np.asarray(x_rows, dtype=dtype)
     f = w1.shape[0] // 2
-    Z = x_rows @ np.asarray(w1, dtype=np.float32).T
+    Z = x_rows @ np.asarray(w1, dtype=dtype).T
     G, U = Z[:, :f], Z[:, f:]
     A = silu(G) * U
-    return A @ np.asarray(w2, dtype=np.float32).T
+    return A @ np.asarray(w2, dtype=dtype).T
+
+
+def expert_ffn_backward(x_rows, w1, w2, d_rows, dtype=np.float32, requant=True) -> dict:
+    """[MF] "Backward gradients" for the rows of one expert, reading R10.  x_rows [n, d],
+    w1 [2f, d], w2 [d, f], d_rows = dL/dO [n, d].  Recomputes Z, G, U, A, then
+        dA = D w2,  dG = dA * U * SiLU'(G),  dU = dA * SiLU(G),  dZ = [dG, dU],
+        dX = dZ w1,  dW2 = D^T A  [d, f],  dW1 = dZ^T X  [2f, d];
+    with `requant`, D and dZ are rounded to bf16 before their products (fp32 only)."""
+    X = np.asarray(x_rows, dtype=dtype)
+    W1 = np.asarray(w1, dtype=dtype)
+    W2 = np.asarray(w2, dtype=dtype)
+    D = np.asarray(d_rows, dtype=dtype)
+    if requant:
+        D = round_bf16(D)
+    f = W1.shape[0] // 2
+    Z = X @ W1.T
+    G, U = Z[:, :f], Z[:, f:]
+    A = silu(G) * U
+    dA = D @ W2
+    dZ = np.concatenate([dA * U * silu_grad(G), dA * silu(G)], axis=1)
+    if requant:
+        dZ = round_bf16(dZ)
+    return {"Z": Z, "A": A, "D": D, "dA": dA, "dZ": dZ, "dX": dZ @ W1,
+            "dW2": D.T @ A, "dW1": dZ.T @ X}
 
 
 def combine(O_rows: np.ndarray, tok_row: np.ndarray, gates: np.ndarray) -> np.ndarray:
@@ -447,6 +497,49 @@ def moe_forward(logits, x, get_expert, k: int, beta: int, P: int, s: int,
     return {"ids": ids, "gates": gates, "counts": counts, "sumsq": S, "kappa": kappa,
             "b": b, "block_off": boff, "plan": pl, "row_token": row_token,
             "row_gate": row_gate, "tok_row": tok_row, "O": O, "y": y}
+
+
+def moe_backward(logits, x, get_expert, dy, k: int, beta: int, dtype=np.float32,
+                 requant=True) -> dict:
+    """Backward of the expert computation for upstream gradient dy = dL/dy [T, d]
+    (reading R10): D rows = row_gate * dy[row_token] in the dispatched row order, each
+    expert's rows through `expert_ffn_backward`, dx_t = sum_j dX[tok_row[t, j]].  Returns
+    dx [T, d], per-expert dW1 [E, 2f, d] and dW2 [E, d, f] (zero for idle experts), and
+    the row-wise D, Z, A, dZ, dX (zero on padding rows)."""
+    logits = np.asarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    ids, gates = route_topk(logits, k)
+    counts = expert_counts(ids, E)
+    boff = block_offsets(block_counts(counts, beta))
+    row_token, row_gate, tok_row = dispatch(ids, gates, boff, beta)
+    x = np.asarray(x, dtype=dtype)
+    dy = np.asarray(dy, dtype=dtype)
+    d = x.shape[1]
+    w1_0, _ = get_expert(0)
+    f = w1_0.shape[0] // 2
+    R = len(row_token)
+    out = {name: np.zeros((R, n), dtype=dtype) for name, n in
+           (("D", d), ("Z", 2 * f), ("A", f), ("dZ", 2 * f), ("dX", d))}
+    dW1 = np.zeros((E, 2 * f, d), dtype=dtype)
+    dW2 = np.zeros((E, d, f), dtype=dtype)
+    for e in range(E):
+        if counts[e] == 0:
+            continue
+        r0 = beta * boff[e]
+        rows = slice(r0, r0 + int(counts[e]))
+        w1, w2 = get_expert(e)
+        Drows = row_gate[rows, None].astype(dtype) * dy[row_token[rows]]
+        g = expert_ffn_backward(x[row_token[rows]], w1, w2, Drows, dtype, requant)
+        for name in ("D", "Z", "A", "dZ", "dX"):
+            out[name][rows] = g[name]
+        dW1[e] = g["dW1"]
+        dW2[e] = g["dW2"]
+    dx = np.zeros((T, d), dtype=dtype)
+    for j in range(k):
+        dx += out["dX"][tok_row[:, j]]
+    out.update(dx=dx, dW1=dW1, dW2=dW2, row_token=row_token, row_gate=row_gate,
+               tok_row=tok_row, block_off=boff, counts=counts)
+    return out
 
 
 def token_output(x_t: np.ndarray, experts, gates_t, get_expert) -> np.ndarray:
