@@ -77,7 +77,13 @@ enum {
 };
 
 /* moe_workspace_size(which) */
-enum { MOE_WS_ROWS = 0, MOE_WS_BLOCKS = 1, MOE_WS_FFN_SCRATCH = 2 };
+enum {
+  MOE_WS_ROWS = 0,
+  MOE_WS_BLOCKS = 1,
+  MOE_WS_FFN_SCRATCH = 2,
+  MOE_WS_FFN_SCRATCH_Z = 3,  /* a_scratch of moe_expert_ffn with MOE_FFN_SAVE_Z */
+  MOE_WS_BWD_SCRATCH = 4     /* bwd_scratch of moe_expert_ffn_backward */
+};
 
 /* plan_info layout (int32[MOE_PI_LEN]) written by moe_plan_blocks */
 enum {
@@ -112,6 +118,10 @@ enum {
   MOE_FFN_SM_PAIR = 4,       /* flag: run each tile on a pair of SMs (a cluster of two
                                 CTAs, tcgen05 cta_group::2, M = 256) instead of each
                                 128-row half on one SM (cta_group::1, the default) */
+  MOE_FFN_SAVE_Z = 16,       /* flag: FC1 also stores Z = [G, U] (bf16 [R_max, 2f]) after
+                                A and the counters in a_scratch, which must then hold
+                                moe_workspace_size(cfg, MOE_WS_FFN_SCRATCH_Z) bytes; the
+                                backward pass reads A and Z from there */
   MOE_FFN_GATHER_X = 8       /* flag: the `xp` argument is x itself (bf16 [T, d]); FC1
                                 gathers each tile's rows x[row_token[r]] straight into
                                 shared memory (TMA row gather), so the dispatched copy
@@ -123,7 +133,10 @@ enum {
 /* Upper bounds: which = MOE_WS_ROWS -> R_max rows (Xp, A, O, row_token, row_gate);
  * MOE_WS_BLOCKS -> B_max entries (blocks, tiles); MOE_WS_FFN_SCRATCH -> bytes of the
  * a_scratch buffer of moe_expert_ffn (A, bf16 [R_max, f], rounded up to 256 bytes, then
- * 256 bytes of tile-scheduler counters).  Returns 0 for an invalid cfg. */
+ * 256 bytes of tile-scheduler counters); MOE_WS_FFN_SCRATCH_Z -> the same followed by
+ * Z (bf16 [R_max, 2f], rounded up to 256 bytes); MOE_WS_BWD_SCRATCH -> bytes of the
+ * bwd_scratch buffer of moe_expert_ffn_backward (dZ, bf16 [R_max, 2f], rounded up to 256
+ * bytes, then 256 bytes of counters).  Returns 0 for an invalid cfg. */
 MOE_API size_t moe_workspace_size(const moe_cfg* cfg, int which);
 
 /* Router top-k, expert histogram and skew ("Routing Skew Problem"; router outputs of the
@@ -246,6 +259,43 @@ MOE_API int moe_expert_ffn_noalloc(const moe_cfg* cfg, const uint16_t* xp, const
                                    const int32_t* plan_info, const int32_t* row_token,
                                    const float* row_gate, int mode, void* out,
                                    int32_t* status, moe_stream_t stream);
+
+/* Backward, step 1: the gradient rows of the expert outputs ("MegaFlux" summary,
+ * Methodology 2, backward gradients: D_e = dL/dO_e; Backward item 3: D_e is requantized).
+ *   dy         fp32 [T, d]: dL/dy.
+ *   row_token, row_gate from moe_dispatch_permute; plan_info from moe_plan_blocks.
+ *   d_rows     bf16 [R_max, d]: row r < beta * B holds bf16(row_gate[r] * dy[row_token[r]])
+ *              (round to nearest even), zeros on padding rows.
+ * A token index outside [0, T) sets MOE_STATUS_BAD_ID and gives a zero row. */
+MOE_API int moe_dispatch_grad(const moe_cfg* cfg, const float* dy, const int32_t* row_token,
+                              const float* row_gate, const int32_t* plan_info,
+                              uint16_t* d_rows, int32_t* status, moe_stream_t stream);
+
+/* Backward, step 2: the expert computation's gradients (same section; the weights are
+ * stored w1 [E, 2f, d] and w2 [E, d, f], so each of the pages' products is taken with that
+ * transpose), on the tensor cores, bf16 operands and fp32 accumulation:
+ *   dA = D w2_e, dZ = [dA * U * SiLU'(G), dA * SiLU(G)] (bf16, requantized), dX = dZ w1_e,
+ *   dx[t] = sum over t's rows of dX (fp32 atomic adds; the order of the adds, and so the
+ *   last bits, may vary), dW2_e = D^T A and dW1_e = dZ^T Xp over expert e's rows.
+ *   xp         bf16 [R_max, d] from moe_dispatch_permute (zero padding rows).
+ *   w1, w2, tiles, plan_info, block_off, row_token as for the forward.
+ *   d_rows     from moe_dispatch_grad.
+ *   saved      the a_scratch of the forward moe_expert_ffn call made with MOE_FFN_SAVE_Z
+ *              (A and Z of the same rows).
+ *   bwd_scratch moe_workspace_size(cfg, MOE_WS_BWD_SCRATCH) bytes: dZ then counters.
+ *   dx         fp32 [T, d], zeroed by the call.
+ *   dw1        fp32 [E, 2f, d] and dw2 fp32 [E, d, f]: written in full (zero for idle
+ *              experts).
+ * Four persistent kernels (dA + SwiGLU backward, dX, dW2, dW1) of one CTA per SM; every
+ * wait is bounded and sets MOE_STATUS_TIMEOUT instead of hanging.  Needs d % 256 == 0 and
+ * f % 128 == 0. */
+MOE_API int moe_expert_ffn_backward(const moe_cfg* cfg, const uint16_t* xp, const uint16_t* w1,
+                                    const uint16_t* w2, const int32_t* tiles,
+                                    const int32_t* plan_info, const int32_t* block_off,
+                                    const int32_t* row_token, const uint16_t* d_rows,
+                                    const uint16_t* saved, uint16_t* bwd_scratch, float* dx,
+                                    float* dw1, float* dw2, int32_t* status,
+                                    moe_stream_t stream);
 
 /* Static text for a return code (negative) or a status bit mask (positive). */
 MOE_API const char* moe_status_string(int code);

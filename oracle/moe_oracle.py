@@ -66,6 +66,8 @@ Readings where the pages leave a step open (each is also listed in the design no
       with that transpose (dA = D w2, dX = dZ w1, dW2 = D^T A, dW1 = dZ^T X);
       dZ = [dA * U * SiLU'(G), dA * SiLU(G)]; D and dZ are requantized to bf16
       (round to nearest even) before they enter a product, everything else is fp32;
+      with `saved_bf16` the activations the forward keeps for the backward (A, computed
+      from fp32 G and U, and Z = [G, U]) enter it rounded to bf16, as they are stored;
       dx_t = sum_j dX[tok_row[t, j]], j ascending.  The gate gradient (router backward)
       is not part of the expert computation and is left out.
 """
@@ -437,12 +439,14 @@ def expert_ffn(x_rows: np.ndarray, w1: np.ndarray, w2: np.ndarray,
     return A @ np.asarray(w2, dtype=dtype).T
 
 
-def expert_ffn_backward(x_rows, w1, w2, d_rows, dtype=np.float32, requant=True) -> dict:
+def expert_ffn_backward(x_rows, w1, w2, d_rows, dtype=np.float32, requant=True,
+                        saved_bf16=False) -> dict:
     """[MF] "Backward gradients" for the rows of one expert, reading R10.  x_rows [n, d],
     w1 [2f, d], w2 [d, f], d_rows = dL/dO [n, d].  Recomputes Z, G, U, A, then
         dA = D w2,  dG = dA * U * SiLU'(G),  dU = dA * SiLU(G),  dZ = [dG, dU],
         dX = dZ w1,  dW2 = D^T A  [d, f],  dW1 = dZ^T X  [2f, d];
-    with `requant`, D and dZ are rounded to bf16 before their products (fp32 only)."""
+    with `requant`, D and dZ are rounded to bf16 before their products, and with
+    `saved_bf16`, A and Z are taken as bf16-rounded copies (fp32 only)."""
     X = np.asarray(x_rows, dtype=dtype)
     W1 = np.asarray(w1, dtype=dtype)
     W2 = np.asarray(w2, dtype=dtype)
@@ -453,6 +457,10 @@ def expert_ffn_backward(x_rows, w1, w2, d_rows, dtype=np.float32, requant=True) 
     Z = X @ W1.T
     G, U = Z[:, :f], Z[:, f:]
     A = silu(G) * U
+    if saved_bf16:
+        A = round_bf16(A)
+        Z = round_bf16(Z)
+        G, U = Z[:, :f], Z[:, f:]
     dA = D @ W2
     dZ = np.concatenate([dA * U * silu_grad(G), dA * silu(G)], axis=1)
     if requant:
@@ -500,7 +508,7 @@ def moe_forward(logits, x, get_expert, k: int, beta: int, P: int, s: int,
 
 
 def moe_backward(logits, x, get_expert, dy, k: int, beta: int, dtype=np.float32,
-                 requant=True) -> dict:
+                 requant=True, saved_bf16=False) -> dict:
     """Backward of the expert computation for upstream gradient dy = dL/dy [T, d]
     (reading R10): D rows = row_gate * dy[row_token] in the dispatched row order, each
     expert's rows through `expert_ffn_backward`, dx_t = sum_j dX[tok_row[t, j]].  Returns
@@ -529,7 +537,7 @@ def moe_backward(logits, x, get_expert, dy, k: int, beta: int, dtype=np.float32,
         rows = slice(r0, r0 + int(counts[e]))
         w1, w2 = get_expert(e)
         Drows = row_gate[rows, None].astype(dtype) * dy[row_token[rows]]
-        g = expert_ffn_backward(x[row_token[rows]], w1, w2, Drows, dtype, requant)
+        g = expert_ffn_backward(x[row_token[rows]], w1, w2, Drows, dtype, requant, saved_bf16)
         for name in ("D", "Z", "A", "dZ", "dX"):
             out[name][rows] = g[name]
         dW1[e] = g["dW1"]

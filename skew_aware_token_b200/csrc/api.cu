@@ -49,6 +49,8 @@ size_t moe_workspace_size(const moe_cfg* cfg, int which) {
   if (which == MOE_WS_ROWS) return (size_t)max_rows(*cfg);
   if (which == MOE_WS_BLOCKS) return (size_t)max_blocks(*cfg);
   if (which == MOE_WS_FFN_SCRATCH) return (size_t)ffn_scratch_bytes(*cfg);
+  if (which == MOE_WS_FFN_SCRATCH_Z) return (size_t)ffn_scratch_z_bytes(*cfg);
+  if (which == MOE_WS_BWD_SCRATCH) return (size_t)bwd_scratch_bytes(*cfg);
   return 0;
 }
 
@@ -102,6 +104,35 @@ int moe_expert_ffn(const moe_cfg* cfg, const uint16_t* xp, const uint16_t* w1,
   if (rc != MOE_OK) return rc;
   return cuda_result(launch_ffn(*cfg, xp, w1, w2, tiles, plan_info, row_token, row_gate, mode,
                                 a_scratch, out, status, (cudaStream_t)stream));
+}
+
+int moe_dispatch_grad(const moe_cfg* cfg, const float* dy, const int32_t* row_token,
+                      const float* row_gate, const int32_t* plan_info, uint16_t* d_rows,
+                      int32_t* status, moe_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  if (cfg->d % 8) return MOE_ERR_UNSUPPORTED;
+  rc = check_ptrs({dy, row_token, row_gate, plan_info, d_rows, status});
+  if (rc != MOE_OK) return rc;
+  return cuda_result(launch_dispatch_grad(*cfg, dy, row_token, row_gate, plan_info, d_rows,
+                                          status, (cudaStream_t)stream));
+}
+
+int moe_expert_ffn_backward(const moe_cfg* cfg, const uint16_t* xp, const uint16_t* w1,
+                            const uint16_t* w2, const int32_t* tiles, const int32_t* plan_info,
+                            const int32_t* block_off, const int32_t* row_token,
+                            const uint16_t* d_rows, const uint16_t* saved,
+                            uint16_t* bwd_scratch, float* dx, float* dw1, float* dw2,
+                            int32_t* status, moe_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  if (cfg->d % 256 || cfg->f % 128) return MOE_ERR_UNSUPPORTED;
+  rc = check_ptrs({xp, w1, w2, tiles, plan_info, block_off, row_token, d_rows, saved,
+                   bwd_scratch, dx, dw1, dw2, status});
+  if (rc != MOE_OK) return rc;
+  return cuda_result(launch_ffn_backward(*cfg, xp, w1, w2, tiles, plan_info, block_off,
+                                         row_token, d_rows, saved, bwd_scratch, dx, dw1, dw2,
+                                         status, (cudaStream_t)stream));
 }
 
 int moe_combine(const moe_cfg* cfg, const uint16_t* o, const int32_t* tok_row,

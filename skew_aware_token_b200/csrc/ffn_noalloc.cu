@@ -64,7 +64,8 @@ extern "C" MOE_API int moe_expert_ffn_noalloc(const moe_cfg* cfg, const uint16_t
       c.s < 0 || (c.beta != 64 && c.beta != 128) || c.d < 1 || c.f < 1)
     return MOE_ERR_INVALID_ARG;
   if (c.E > kMaxE || (long long)c.T * c.k > kMaxN) return MOE_ERR_UNSUPPORTED;
-  if (mode & ~kFfnModes) return MOE_ERR_INVALID_ARG;
+  // the fixed array holds A only: saving Z for a backward pass needs the caller's scratch
+  if (mode & ~kFfnModes || mode & MOE_FFN_SAVE_Z) return MOE_ERR_INVALID_ARG;
   if (c.d % 256 || c.f % 128) return MOE_ERR_UNSUPPORTED;
   for (const void* p : {(const void*)xp, (const void*)w1, (const void*)w2, (const void*)tiles,
                         (const void*)plan_info, (const void*)row_token, (const void*)row_gate,

@@ -56,13 +56,7 @@
 // Every mbarrier wait is bounded (globaltimer); on expiry the kernel sets
 // MOE_STATUS_TIMEOUT, lets the other roles drop out, waits (bounded) for its own copies
 // and MMAs in flight, frees its TMEM and returns.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-#include <cuda_bf16.h>
-
-#include <mutex>
-
-#include "moe_common.cuh"
+#include "tc_util.cuh"
 
 namespace moe {
 namespace {
@@ -119,232 +113,11 @@ struct FfnArgs {
   int out_ld;    // output row length (elements)
   int write_o;   // FC2: store O (1) or fused combine (0)
   int gather;    // FC1: A rows gathered from x by row_token (tmA maps x [T, d], box 1 row)
+  uint16_t* z;   // FC1 with MOE_FFN_SAVE_Z: Z = [G, U] bf16 [r_max, 2f] (else null)
   const void* x; // the token rows x bf16 [T, d] (gather)
   int strict;
   unsigned long long timeout_ns;
 };
-
-// ------------------------------------------------------------------ PTX wrappers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// address of the same shared variable in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
-  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-// arrive on a barrier in another CTA of the cluster (cluster-mapped address)
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
-               : "memory");
-}
-__device__ __forceinline__ void st_remote_u32(uint32_t cluster_addr, uint32_t v) {
-  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; "
-      "selp.u32 %0, 1, 0, p; }"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-// Bounded wait for the phase of `parity` to complete.  Returns false if another role
-// raised `abort_flag` (when honour_abort) or if the wait ran out (then raises it).
-__device__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                          int32_t* status, unsigned long long timeout_ns, bool honour_abort) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  for (uint32_t spin = 1;; ++spin) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((spin & 31u) == 0) {
-      if (honour_abort && *abort_flag) return false;
-      if (globaltimer() - t0 > timeout_ns) {
-        *abort_flag = 1;
-        set_status(status, MOE_STATUS_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cta.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(map), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-// Copy into this CTA's shared memory whose completion is counted on the barrier of the
-// pair's first CTA (cluster-mapped address `bar`).  No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
-                                                 uint32_t bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(map), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-// Row gather: rows r0..r3 of a 2-D tensor map whose box is one row of 64 columns, columns
-// [x, x + 64), into four consecutive 128-byte rows at dst (the same swizzle as a tile
-// load), completion counted on the pair's first CTA's barrier (cluster address `bar`).
-__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap* map,
-                                                 uint32_t bar, int x, int4 r) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
-      ".mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(map), "r"(x), "r"(r.x), "r"(r.y), "r"(r.z), "r"(r.w), "r"(bar)
-      : "memory");
-}
-// 16-byte copy global -> shared (through L2 only).
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-// Arrive on `bar` once every cp.async this thread issued so far has landed (the barrier's
-// expected count includes this arrival).
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
-}
-// Shared-memory matrix descriptor of a K-major tile written by TMA with the 128-byte
-// swizzle: start address >> 4 (bits 0-13), leading offset unused for this layout (1),
-// stride offset = 1024 bytes between 8-row groups (bits 32-45), descriptor version 1
-// (bit 46), swizzle mode 2 = 128-byte (bits 61-63).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         (1ull << 46) | (2ull << 61);
-}
-template <bool PAIR>
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  if constexpr (PAIR) {
-    asm volatile(
-        "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
-  } else {
-    asm volatile(
-        "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
-  }
-}
-// Arrive on `bar` (same offset in both CTAs of a pair) once this thread's MMAs complete.
-template <bool PAIR>
-__device__ __forceinline__ void umma_commit_all(uint32_t bar) {
-  if constexpr (PAIR) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster"
-        ".b64 [%0], %1;" ::"r"(bar),
-        "h"((uint16_t)3)
-        : "memory");
-  } else {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-        : "memory");
-  }
-}
-// Arrive on this CTA's `bar` once this thread's MMAs complete.
-template <bool PAIR>
-__device__ __forceinline__ void umma_commit_local(uint32_t bar) {
-  if constexpr (PAIR) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-        : "memory");
-  } else {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-        : "memory");
-  }
-}
-template <bool PAIR>
-__device__ __forceinline__ void tmem_alloc(uint32_t slot_addr) {
-  if constexpr (PAIR) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     slot_addr),
-                 "r"(TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
-  } else {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     slot_addr),
-                 "r"(TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
-}
-template <bool PAIR>
-__device__ __forceinline__ void tmem_dealloc(uint32_t base) {
-  if constexpr (PAIR) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(base),
-                 "r"(TMEM_COLS));
-  } else {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(base),
-                 "r"(TMEM_COLS));
-  }
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void red_add_v4(float* addr, float4 v) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(v.x), "f"(v.y),
-               "f"(v.z), "f"(v.w)
-               : "memory");
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
 
 // ------------------------------------------------------------------ work schedule
 // Item L of a unit's range -> tile m, n-tile n and (single SM) the tile half.
@@ -462,7 +235,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     prefetch_tmap(&tmB);
     if (PAIR) prefetch_tmap(&tmA64);
   }
-  if (warp == 1) tmem_alloc<PAIR>(smem_u32(tmem_slot));
+  if (warp == 1) tmem_alloc<PAIR, TMEM_COLS>(smem_u32(tmem_slot));
   tc_fence_before();
   if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
@@ -808,6 +581,23 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 #pragma unroll
             for (int i = 0; i < 4; ++i)
               dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            if (a.z) {  // keep Z = [G, U] for the backward pass
+              uint4* zg = reinterpret_cast<uint4*>(a.z + row * 2 * a.f + n * (BN / 2) + ocol);
+              uint4* zu = reinterpret_cast<uint4*>(a.z + row * 2 * a.f + a.f + n * (BN / 2) + ocol);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                zg[i] = make_uint4(
+                    pack_bf16(__uint_as_float(g[8 * i + 0]), __uint_as_float(g[8 * i + 1])),
+                    pack_bf16(__uint_as_float(g[8 * i + 2]), __uint_as_float(g[8 * i + 3])),
+                    pack_bf16(__uint_as_float(g[8 * i + 4]), __uint_as_float(g[8 * i + 5])),
+                    pack_bf16(__uint_as_float(g[8 * i + 6]), __uint_as_float(g[8 * i + 7])));
+                zu[i] = make_uint4(
+                    pack_bf16(__uint_as_float(u[8 * i + 0]), __uint_as_float(u[8 * i + 1])),
+                    pack_bf16(__uint_as_float(u[8 * i + 2]), __uint_as_float(u[8 * i + 3])),
+                    pack_bf16(__uint_as_float(u[8 * i + 4]), __uint_as_float(u[8 * i + 5])),
+                    pack_bf16(__uint_as_float(u[8 * i + 6]), __uint_as_float(u[8 * i + 7])));
+              }
+            }
           }
         }
       } else if (a.write_o) {
@@ -883,40 +673,11 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
   if constexpr (PAIR) cluster_sync(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc<PAIR>(tmem_base);
+    tmem_dealloc<PAIR, TMEM_COLS>(tmem_base);
   }
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// 2-D bf16 tensor [outer, inner] (inner contiguous), box [box_outer, 64], 128-byte swizzle.
-bool encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-               uint32_t box_outer) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {(cuuint32_t)BK, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int PHASE, bool PAIR>
 cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ta64,
                        const FfnArgs& args, cudaStream_t st) {
@@ -1012,6 +773,11 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   a1.write_o = 0;
   a1.gather = gather;
   a1.x = gather ? xp : nullptr;
+  // Z after A and the scheduler counters in the scratch buffer
+  a1.z = (mode & MOE_FFN_SAVE_Z)
+             ? reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(a_scratch) +
+                                           ffn_a_bytes(c) + kSchedBytes)
+             : nullptr;
   a2.sched = sched + 8;
   a2.out = out;
   a2.n_k = c.f / BK;

@@ -13,8 +13,8 @@ constexpr int kMaxK = 8;
 constexpr int kMaxP = 8;
 constexpr long long kMaxN = 1LL << 22;
 // every flag moe_expert_ffn accepts
-constexpr int kFfnModes =
-    MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR | MOE_FFN_GATHER_X;
+constexpr int kFfnModes = MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR |
+                          MOE_FFN_GATHER_X | MOE_FFN_SAVE_Z;
 
 // Bound on the number of token blocks over every routing of N rows into E experts:
 // sum_e ceil(c_e / beta) <= (N + min(E, N) * (beta - 1)) / beta.
@@ -32,6 +32,16 @@ inline long long ffn_a_bytes(const moe_cfg& c) {
   return (max_rows(c) * c.f * 2 + 255) / 256 * 256;
 }
 inline long long ffn_scratch_bytes(const moe_cfg& c) { return ffn_a_bytes(c) + kSchedBytes; }
+// Z = [G, U] (bf16 [R_max, 2f]) or dZ, rounded up to 256 bytes
+inline long long ffn_z_bytes(const moe_cfg& c) {
+  return (max_rows(c) * 2 * c.f * 2 + 255) / 256 * 256;
+}
+// with MOE_FFN_SAVE_Z: A, the counters, then Z
+inline long long ffn_scratch_z_bytes(const moe_cfg& c) {
+  return ffn_scratch_bytes(c) + ffn_z_bytes(c);
+}
+// backward scratch: dZ, then the counters of its four launches
+inline long long bwd_scratch_bytes(const moe_cfg& c) { return ffn_z_bytes(c) + kSchedBytes; }
 
 __device__ __forceinline__ void set_status(int32_t* status, int bits) {
   atomicOr(status, bits);
@@ -55,6 +65,15 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
                        uint16_t* a_scratch, void* out, int32_t* status, cudaStream_t st);
 cudaError_t launch_combine(const moe_cfg& c, const uint16_t* o, const int32_t* tok_row,
                            const float* gates, float* y, int32_t* status, cudaStream_t st);
+cudaError_t launch_dispatch_grad(const moe_cfg& c, const float* dy, const int32_t* row_token,
+                                 const float* row_gate, const int32_t* plan_info,
+                                 uint16_t* d_rows, int32_t* status, cudaStream_t st);
+cudaError_t launch_ffn_backward(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
+                                const uint16_t* w2, const int32_t* tiles,
+                                const int32_t* plan_info, const int32_t* block_off,
+                                const int32_t* row_token, const uint16_t* d_rows,
+                                const uint16_t* saved, uint16_t* bwd_scratch, float* dx,
+                                float* dw1, float* dw2, int32_t* status, cudaStream_t st);
 
 int num_sms();
 

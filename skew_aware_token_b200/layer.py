@@ -14,12 +14,16 @@ from . import native as N
 
 class MoeLayer:
     def __init__(self, wl, device="cuda", write_o: bool = False, guard: int = 0,
-                 gather_x: bool = False):
+                 gather_x: bool = False, train: bool = False):
         """`guard` adds that many spare elements after every buffer (canary checks).
         `gather_x`: FC1 gathers its rows from x by row_token (MOE_FFN_GATHER_X) and the
         dispatched copy Xp is neither allocated nor written (saves R_max * d * 2 bytes; as
         fast while x stays resident in L2, slower once it does not); False (default)
-        materialises Xp with the dispatch gather."""
+        materialises Xp with the dispatch gather.
+        `train`: the forward keeps Z = [G, U] (MOE_FFN_SAVE_Z) and the layer holds the
+        backward's buffers (D rows, dZ scratch, dx, dW1, dW2); needs the Xp path."""
+        if train and gather_x:
+            raise ValueError("the backward pass reads Xp: train=True needs gather_x=False")
         self.cfg = N.MoeCfg.of(wl)
         self.wl = wl
         dev = torch.device(device)
@@ -50,8 +54,17 @@ class MoeLayer:
         self.row_token = z(max(R, 4))
         self.row_gate = z(max(R, 4), dt=f32)
         self.tok_row = z(max(T * k, 4))
-        ws = N.moe_workspace_size(self.cfg, N.MOE_WS_FFN_SCRATCH)
+        self.train = train
+        ws = N.moe_workspace_size(self.cfg, N.MOE_WS_FFN_SCRATCH_Z if train
+                                  else N.MOE_WS_FFN_SCRATCH)
         self.a_scratch = z(max(ws // 2, 8), dt=torch.bfloat16)
+        if train:
+            self.d_rows = z(max(R * d, 8), dt=torch.bfloat16)
+            bws = N.moe_workspace_size(self.cfg, N.MOE_WS_BWD_SCRATCH)
+            self.bwd_scratch = z(max(bws // 2, 8), dt=torch.bfloat16)
+            self.dx = z(max(T * d, 4), dt=f32)
+            self.dw1 = z(max(E * 2 * f * d, 4), dt=f32)
+            self.dw2 = z(max(E * d * f, 4), dt=f32)
         self.y = z(max(T * d, 4), dt=f32)
         self.o = z(max(R * d, 8), dt=torch.bfloat16) if write_o else None
         self.device = dev
@@ -83,6 +96,8 @@ class MoeLayer:
             src, mode = x, mode | N.MOE_FFN_GATHER_X
         else:
             src = self.xp
+        if self.train:
+            mode |= N.MOE_FFN_SAVE_Z
         N.moe_expert_ffn(self.cfg, src, w1, w2, self.tiles, self.plan_info,
                          self.row_token, self.row_gate, mode, self.a_scratch, out,
                          self.status, stream)
@@ -104,6 +119,19 @@ class MoeLayer:
             self.combine(stream, y)
         out = self.y if y is None else y
         return out[: self.wl.T * self.wl.d].view(self.wl.T, self.wl.d)
+
+    def backward(self, dy, w1, w2, stream=None):
+        """Gradients of the expert computation for dL/dy = dy (fp32 [T, d]) after a forward
+        call of this layer: returns views of dx [T, d], dW1 [E, 2f, d], dW2 [E, d, f]."""
+        if not self.train:
+            raise ValueError("layer built without train=True")
+        N.moe_dispatch_grad(self.cfg, dy, self.row_token, self.row_gate, self.plan_info,
+                            self.d_rows, self.status, stream)
+        N.moe_expert_ffn_backward(self.cfg, self.xp, w1, w2, self.tiles, self.plan_info,
+                                  self.block_off, self.row_token, self.d_rows, self.a_scratch,
+                                  self.bwd_scratch, self.dx, self.dw1, self.dw2, self.status,
+                                  stream)
+        return self.view("dx"), self.view("dw1"), self.view("dw2")
 
     def forward_host(self, logits_h, x_h, w1, w2, y_h, logits_d, x_d, mode=0, stream=None):
         """End to end from pinned host buffers: copies logits and x in, runs the layer,
@@ -140,6 +168,13 @@ class MoeLayer:
             shapes["o"] = (self.o, (R, d))
         if self.xp is not None:
             shapes["xp"] = (self.xp, (R, d))
+        if self.train:
+            f = wl.f
+            z_off = N.moe_workspace_size(self.cfg, N.MOE_WS_FFN_SCRATCH) // 2
+            shapes.update({
+                "z": (self.a_scratch[z_off:], (R, 2 * f)), "d_rows": (self.d_rows, (R, d)),
+                "dz": (self.bwd_scratch, (R, 2 * f)), "dx": (self.dx, (T, d)),
+                "dw1": (self.dw1, (E, 2 * f, d)), "dw2": (self.dw2, (E, d, f))})
         buf, shape = shapes[name]
         n = 1
         for s in shape:

@@ -22,8 +22,10 @@ MOE_NOALLOC_SCRATCH_BYTES = 64 << 20
 MOE_STATUS_BAD_ID, MOE_STATUS_OVERFLOW, MOE_STATUS_NONFINITE = 1, 2, 4
 MOE_STATUS_TIMEOUT, MOE_STATUS_PLAN = 8, 16
 MOE_WS_ROWS, MOE_WS_BLOCKS, MOE_WS_FFN_SCRATCH = 0, 1, 2
+MOE_WS_FFN_SCRATCH_Z, MOE_WS_BWD_SCRATCH = 3, 4
 MOE_FFN_FUSED_COMBINE, MOE_FFN_WRITE_O, MOE_FFN_STRICT_SLOTS, MOE_FFN_SM_PAIR = 0, 1, 2, 4
 MOE_FFN_GATHER_X = 8
+MOE_FFN_SAVE_Z = 16
 PI = dict(B=0, TAU=1, MAKESPAN=2, VARIANT=3, NTILES=4, FIXED_MAKESPAN=5, REPLICAS=6,
           ROUNDS=7, SLOT_TILE_OFF=8, VAR_MAKESPAN=17, VAR_REPLICAS=22, VAR_ROUNDS=27,
           QUOTA_TAU=32, COST=33, VAR_COST=34, LEN=40)
@@ -74,6 +76,8 @@ _SIGNATURES = {
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(MoeCfg)] + [_VP] * 6),
     "moe_expert_ffn_noalloc": (ctypes.c_int, [ctypes.POINTER(MoeCfg)] + [_VP] * 7 +
                                [ctypes.c_int] + [_VP] * 3),
+    "moe_dispatch_grad": (ctypes.c_int, [ctypes.POINTER(MoeCfg)] + [_VP] * 7),
+    "moe_expert_ffn_backward": (ctypes.c_int, [ctypes.POINTER(MoeCfg)] + [_VP] * 15),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
@@ -174,6 +178,26 @@ def moe_expert_ffn(cfg, xp, w1, w2, tiles, plan_info, row_token, row_gate, mode,
         _dev(plan_info, "plan_info"), _dev(row_token, "row_token"), _dev(row_gate, "row_gate"),
         int(mode), _dev(a_scratch, "a_scratch"), _dev(out, "out"), _dev(status, "status"),
         _stream(stream)))
+
+
+def moe_dispatch_grad(cfg, dy, row_token, row_gate, plan_info, d_rows, status,
+                      stream=None) -> None:
+    c = _cfg(cfg)
+    _check("moe_dispatch_grad", lib().moe_dispatch_grad(
+        ctypes.byref(c), _dev(dy, "dy"), _dev(row_token, "row_token"),
+        _dev(row_gate, "row_gate"), _dev(plan_info, "plan_info"), _dev(d_rows, "d_rows"),
+        _dev(status, "status"), _stream(stream)))
+
+
+def moe_expert_ffn_backward(cfg, xp, w1, w2, tiles, plan_info, block_off, row_token, d_rows,
+                            saved, bwd_scratch, dx, dw1, dw2, status, stream=None) -> None:
+    c = _cfg(cfg)
+    _check("moe_expert_ffn_backward", lib().moe_expert_ffn_backward(
+        ctypes.byref(c), _dev(xp, "xp"), _dev(w1, "w1"), _dev(w2, "w2"), _dev(tiles, "tiles"),
+        _dev(plan_info, "plan_info"), _dev(block_off, "block_off"),
+        _dev(row_token, "row_token"), _dev(d_rows, "d_rows"), _dev(saved, "saved"),
+        _dev(bwd_scratch, "bwd_scratch"), _dev(dx, "dx"), _dev(dw1, "dw1"), _dev(dw2, "dw2"),
+        _dev(status, "status"), _stream(stream)))
 
 
 def moe_combine(cfg, o, tok_row, topk_gates, y, status, stream=None) -> None:

@@ -29,6 +29,7 @@ import torch
 
 # Tensor ids that key the per-tensor seed streams.
 TID_LOGITS, TID_X, TID_W1, TID_W2, TID_HOT = 1, 2, 3, 4, 5
+TID_DY = 6  # upstream gradient dL/dy of the backward pass
 HOT_EXPERTS = (0, 1, 2, 3)
 
 
@@ -134,6 +135,12 @@ def make_x(wl: Workload) -> torch.Tensor:
     """Token activations bf16 [T, d] on the host."""
     return torch.randn(wl.T, wl.d, generator=_gen(seed_for(wl.seed, TID_X)),
                        dtype=torch.float32).to(torch.bfloat16)
+
+
+def make_dy(wl: Workload) -> torch.Tensor:
+    """Upstream gradient dL/dy fp32 [T, d] on the host, N(0, 1)."""
+    return torch.randn(wl.T, wl.d, generator=_gen(seed_for(wl.seed, TID_DY)),
+                       dtype=torch.float32)
 
 
 def expert_weights(wl: Workload, e: int, device="cpu") -> tuple[torch.Tensor, torch.Tensor]:

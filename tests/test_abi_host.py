@@ -24,7 +24,8 @@ def test_exports_every_declared_symbol():
     declared = N.declared_symbols()
     assert set(declared) == {"moe_workspace_size", "moe_route_hist", "moe_plan_blocks",
                              "moe_dispatch_permute", "moe_expert_ffn", "moe_combine",
-                             "moe_status_string", "moe_expert_ffn_noalloc"}
+                             "moe_status_string", "moe_expert_ffn_noalloc",
+                             "moe_dispatch_grad", "moe_expert_ffn_backward"}
     out = subprocess.run(["nm", "-D", "--defined-only", N.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
@@ -93,7 +94,7 @@ def test_null_and_misaligned_pointers_rejected():
     assert lib.moe_dispatch_permute(cfg, *disp, None) == N.MOE_ERR_UNSUPPORTED
     for bad_mask in (1 << 6, 1 << 7, 1 << 24, 0xFFFFFFFF):  # bits 6, 7 and 24..31 are unused
         assert lib.moe_plan_blocks(cfg, ok, bad_mask, *[ok] * 8, None) == N.MOE_ERR_INVALID_ARG
-    assert lib.moe_expert_ffn(cfg, *[ok] * 7, 16, *[ok] * 3, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_ffn(cfg, *[ok] * 7, 32, *[ok] * 3, None) == N.MOE_ERR_INVALID_ARG
     bad_d = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(d=320)))
     assert lib.moe_expert_ffn(bad_d, *[ok] * 7, 0, *[ok] * 3, None) == N.MOE_ERR_UNSUPPORTED
     bad_f = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(f=192)))
@@ -132,3 +133,34 @@ def test_header_constants_match_binding():
                  "MOE_FFN_SM_PAIR", "MOE_FFN_GATHER_X", "MOE_ERR_TOO_LARGE"):
         assert enum[name] == getattr(N, name), name
     assert N.variant_mask() == 0 and N.variant_mask([4], u_min=3) == (1 << 4) | (3 << 8)
+
+
+@pytest.mark.skipif(not NO_GPU, reason="fake pointers are only passed where no GPU exists")
+def test_backward_entry_points_reject_bad_arguments():
+    cfg = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"]))
+    lib = N.lib()
+    ok = 1 << 20
+    for i in range(14):
+        args = [ok] * 14
+        args[i] = None
+        assert lib.moe_expert_ffn_backward(cfg, *args, None) == N.MOE_ERR_INVALID_ARG, i
+        args[i] = ok + 8
+        assert lib.moe_expert_ffn_backward(cfg, *args, None) == N.MOE_ERR_UNSUPPORTED, i
+    for i in range(6):
+        args = [ok] * 6
+        args[i] = None
+        assert lib.moe_dispatch_grad(cfg, *args, None) == N.MOE_ERR_INVALID_ARG, i
+    bad_d = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(d=320)))
+    assert lib.moe_expert_ffn_backward(bad_d, *[ok] * 14, None) == N.MOE_ERR_UNSUPPORTED
+    # the allocation-free forward cannot keep Z for a backward pass
+    assert lib.moe_expert_ffn_noalloc(cfg, *[ok] * 7, N.MOE_FFN_SAVE_Z, *[ok] * 2,
+                                      None) == N.MOE_ERR_INVALID_ARG
+
+
+def test_training_workspace_sizes():
+    for wl in (WORKLOADS["tiny"], WORKLOADS["olmoe_a1"], WORKLOADS["dsv3_a1"]):
+        R = N.moe_workspace_size(wl, N.MOE_WS_ROWS)
+        base = N.moe_workspace_size(wl, N.MOE_WS_FFN_SCRATCH)
+        z_bytes = -(-R * 2 * wl.f * 2 // 256) * 256
+        assert N.moe_workspace_size(wl, N.MOE_WS_FFN_SCRATCH_Z) == base + z_bytes
+        assert N.moe_workspace_size(wl, N.MOE_WS_BWD_SCRATCH) == z_bytes + 256
