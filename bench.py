@@ -216,6 +216,44 @@ def run_e2e(layer, logits_h, x_h, w1, w2, mode, wl, args, world, dev):
             "overlap": "H2D of step i+1 and D2H of step i-1 overlap the layer on step i"}
 
 
+def run_backward(layer, w1, w2, wl, args, dev, peak, peak_src):
+    """Times the backward of the expert computation (moe_dispatch_grad, then the four
+    gradient GEMMs of moe_expert_ffn_backward) after the layer's last forward: 12 N d f
+    algorithmic flops per step (twice the forward's)."""
+    dy = synth.make_dy(wl).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(max(args.warmup, 3)):
+        layer.backward(dy, w1, w2)
+    torch.cuda.synchronize(dev)
+    steps = max(1, min(args.steps, 200))
+    marks = [[ev() for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        marks[i][0].record(stream)
+        N.moe_dispatch_grad(layer.cfg, dy, layer.row_token, layer.row_gate, layer.plan_info,
+                            layer.d_rows, layer.status)
+        marks[i][1].record(stream)
+        N.moe_expert_ffn_backward(layer.cfg, layer.xp, w1, w2, layer.tiles, layer.plan_info,
+                                  layer.block_off, layer.row_token, layer.d_rows,
+                                  layer.a_scratch, layer.bwd_scratch, layer.dx, layer.dw1,
+                                  layer.dw2, layer.status)
+        marks[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    status = layer.read_status()
+    if status != 0:
+        raise RuntimeError(f"device status after backward: {N.moe_status_string(status)}")
+    d_ms = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
+    g_ms = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
+    flops = 2 * wl.flops
+    g_tflops = flops / (g_ms / 1e3) / 1e12
+    return {"steps": steps, "ms_per_step": round(d_ms + g_ms, 4),
+            "stages_ms": {"dispatch_grad": round(d_ms, 4), "gemms": round(g_ms, 4)},
+            "flops_per_step": flops, "tokens_per_s": round(wl.T * wl.k / ((d_ms + g_ms) / 1e3), 1),
+            "roofline": {"bound": "tensor", "kernel": "gradient GEMMs (dA+SwiGLU', dX, dW2, dW1)",
+                         "achieved": round(g_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(g_tflops / peak, 4), "peak_source": peak_src}}
+
+
 def run_ours(args, wl, world, rank, local):
     from skew_aware_token_b200.layer import MoeLayer
     dev = torch.device("cuda", local)
@@ -226,7 +264,7 @@ def run_ours(args, wl, world, rank, local):
     logits = logits_h.to(dev)
     x = x_h.to(dev)
     write_o = args.ffn == "write_o"
-    layer = MoeLayer(wl, dev, write_o=write_o, gather_x=args.gather_x)
+    layer = MoeLayer(wl, dev, write_o=write_o, gather_x=args.gather_x, train=args.backward)
     stream = torch.cuda.current_stream(dev)
     mode = ((N.MOE_FFN_STRICT_SLOTS if args.strict else 0) |
             (N.MOE_FFN_WRITE_O if write_o else 0) | (N.MOE_FFN_SM_PAIR if args.sm_pair else 0))
@@ -306,6 +344,9 @@ def run_ours(args, wl, world, rank, local):
         if tr:
             roofline["traffic"] = tr
 
+    backward = run_backward(layer, w1, w2, wl, args, dev, peak, peak_src) if args.backward \
+        else None
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(layer, logits_h, x_h, w1, w2, mode, wl, args, world, dev)
@@ -341,6 +382,7 @@ def run_ours(args, wl, world, rank, local):
         "tflops": round(tflops, 2), "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roofline, "cpu_baseline": cpu,
         "e2e": e2e,
+        "backward": backward,
         "gpu_launches": (LAUNCHES_PER_STEP + int(write_o) - int(args.gather_x)) * args.steps,
         "clocks": clocks.summary(),
         "impl": "ours",
@@ -406,6 +448,9 @@ def main():
     ap.add_argument("--variant-mask", type=lambda v: int(v, 0), default=0,
                     help="planner variants (bits 0..3 bounded greedy, bit 4 quota solver; "
                          "0 = all five) and, in bits 8..15, the quota floor u_min")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the backward of the expert computation (the forward then "
+                         "keeps Z for it)")
     ap.add_argument("--gather-x", action="store_true",
                     help="FC1 gathers its rows from x by row_token (no Xp, no gather kernel)")
     ap.add_argument("--ffn", default="fused", choices=["fused", "write_o"],

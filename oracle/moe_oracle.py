@@ -48,7 +48,7 @@ Readings where the pages leave a step open (each is also listed in the design no
       inside an expert; expert e's i-th row goes to padded row beta*block_off[e] + i.
   R6  the FFN is evaluated in fp32 from the exact bf16 input values; A is kept in fp32.
   R7  the combine sums j = 0..k-1 in ascending order in fp32.
-  R8  the quota solver of `plan_quota` (variant 4) in this block formulation: ranks are
+  R13 the quota solver of `plan_quota` (variant 4) in this block formulation: ranks are
       the P slots, the load of expert e is b_e blocks, N_slot = s; the search runs over
       integer tau in [ceil(B / P), max_r home load] exactly as printed (while lo < hi,
       tau = floor((lo + hi) / 2); the target coefficient beta does not enter the printed
@@ -56,12 +56,12 @@ Readings where the pages leave a step open (each is also listed in the design no
       receivers are ranks other than the donor with slack > 0 and a free replica slot
       (rep_t < s), ties of slack to the lower rank; u_min is counted in blocks (default 1);
       the plan is the oracle's quota table at the tau the search ends on.
-  R9  the reduction-aware variant (C_lambda) keeps each greedy search's moves and returns
+  R14 the reduction-aware variant (C_lambda) keeps each greedy search's moves and returns
       the plan, among the search's start and the plan after each move, of least C_lambda
       (the earliest on ties; n_r grows by one whenever a move opens a copy of one of r's
       experts); the quota solver's plan is scored as it ends; the best variant is then
       the least (C_lambda, makespan, replicas, variant index).
-  R10 backward: D = dL/dO on row r is row_gate[r] * dy[row_token[r]] (zero on padding
+  R15 backward: D = dL/dO on row r is row_gate[r] * dy[row_token[r]] (zero on padding
       rows); the weights are stored w1 [2f, d], w2 [d, f], so each page formula is taken
       with that transpose (dA = D w2, dX = dZ w1, dW2 = D^T A, dW1 = dZ^T X);
       dZ = [dA * U * SiLU'(G), dA * SiLU(G)]; D and dZ are requantized to bf16
@@ -160,7 +160,7 @@ def reduction_cost(q, P: int, lam: int) -> int:
 
 def plan_variant(b, P: int, s: int, v: int, lam: int | None = None) -> dict:
     """One bounded greedy search of [MF] "Bounded Greedy Search"; reading R4 (and with
-    `lam`, the reduction-aware variant of reading R9).
+    `lam`, the reduction-aware variant of reading R14).
 
     Variant v = 2*D + F with donor priority D (0: decreasing total overload l_r,
     1: largest remaining home-expert load max_{h(e)=r} q_er) and fan-out F (0: at most
@@ -194,7 +194,7 @@ def plan_variant(b, P: int, s: int, v: int, lam: int | None = None) -> dict:
     B = sum(b)
     tau = -(-B // P)
     rounds = 0
-    # reading R9: the least C_lambda along the search (start, then after every move)
+    # reading R14: the least C_lambda along the search (start, then after every move)
     best = None
     if lam is not None:
         best = {"cost": reduction_cost(q, P, lam), "q": [row[:] for row in q],
@@ -247,7 +247,7 @@ def plan_variant(b, P: int, s: int, v: int, lam: int | None = None) -> dict:
 
 
 def quota_feasible(b, P: int, s: int, u_min: int, tau: int) -> dict:
-    """[UE] Algorithm 1's greedy feasibility oracle at one threshold tau; reading R8.
+    """[UE] Algorithm 1's greedy feasibility oracle at one threshold tau; reading R13.
 
     Start from the home placement q[e][h(e)] = b_e.  exc_r = max(l_r - tau, 0) and
     slk_r = max(tau - l_r, 0).  Overloaded ranks in order of descending excess (ties to the
@@ -288,7 +288,7 @@ def quota_feasible(b, P: int, s: int, u_min: int, tau: int) -> dict:
 def plan_quota(b, P: int, s: int, u_min: int = 1) -> dict:
     """[UE] Algorithm 1 (joint solving): binary search for the smallest tau that
     `quota_feasible` satisfies, on [ceil(B / P), max_r home load]; the plan is the quota
-    table at that tau.  Reading R8.  'rounds' counts the search iterations."""
+    table at that tau.  Reading R13.  'rounds' counts the search iterations."""
     E = len(b)
     b = [int(x) for x in b]
     u_min = max(int(u_min), 1)
@@ -328,7 +328,7 @@ def plan(b, P: int, s: int, variant_mask: int = GREEDY_VARIANTS, u_min: int = 1,
     """Run the enabled variants (bits 0..3: the greedy searches, bit 4: the quota solver;
     0 means the four greedy searches, the method's planner) and keep the best.  Reading
     R4: the best is the lexicographic minimum of (makespan, total replicas, variant
-    index); with `lam` (reading R9), of (C_lambda, makespan, replicas, variant index)."""
+    index); with `lam` (reading R14), of (C_lambda, makespan, replicas, variant index)."""
     mask = variant_mask & ALL_VARIANTS or GREEDY_VARIANTS
     results = [plan_variant(b, P, s, v, lam) for v in range(4) if mask >> v & 1]
     if mask >> QUOTA_VARIANT & 1:
@@ -441,7 +441,7 @@ def expert_ffn(x_rows: np.ndarray, w1: np.ndarray, w2: np.ndarray,
 
 def expert_ffn_backward(x_rows, w1, w2, d_rows, dtype=np.float32, requant=True,
                         saved_bf16=False) -> dict:
-    """[MF] "Backward gradients" for the rows of one expert, reading R10.  x_rows [n, d],
+    """[MF] "Backward gradients" for the rows of one expert, reading R15.  x_rows [n, d],
     w1 [2f, d], w2 [d, f], d_rows = dL/dO [n, d].  Recomputes Z, G, U, A, then
         dA = D w2,  dG = dA * U * SiLU'(G),  dU = dA * SiLU(G),  dZ = [dG, dU],
         dX = dZ w1,  dW2 = D^T A  [d, f],  dW1 = dZ^T X  [2f, d];
@@ -510,7 +510,7 @@ def moe_forward(logits, x, get_expert, k: int, beta: int, P: int, s: int,
 def moe_backward(logits, x, get_expert, dy, k: int, beta: int, dtype=np.float32,
                  requant=True, saved_bf16=False) -> dict:
     """Backward of the expert computation for upstream gradient dy = dL/dy [T, d]
-    (reading R10): D rows = row_gate * dy[row_token] in the dispatched row order, each
+    (reading R15): D rows = row_gate * dy[row_token] in the dispatched row order, each
     expert's rows through `expert_ffn_backward`, dx_t = sum_j dX[tok_row[t, j]].  Returns
     dx [T, d], per-expert dW1 [E, 2f, d] and dW2 [E, d, f] (zero for idle experts), and
     the row-wise D, Z, A, dZ, dX (zero on padding rows)."""

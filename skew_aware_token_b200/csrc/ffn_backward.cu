@@ -47,7 +47,7 @@ struct BGeo {
   static constexpr int B_BYTES = BN * kBK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = STAGE_BYTES <= 32 * 1024 ? 6 : 4;
-  static constexpr int STG = KIND == DGRAD_X ? 4 * 32 * kStgStride * 4 : 0;
+  static constexpr int STG = 4 * 32 * kStgStride * 4;  // epilogue staging, 32 x 32 per warp
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int NBARS = 2 * STAGES + 5 + 2 * kRing;
   static constexpr int SMEM = STAGES * STAGE_BYTES + STG + kMetaBytes + 1024;
@@ -56,7 +56,7 @@ struct BGeo {
                                     ((A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16) |
                                     ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 };
-static_assert(BGeo<DGRAD_A, 128>::SMEM <= 227 * 1024 && BGeo<DGRAD_X, 256>::SMEM <= 227 * 1024 &&
+static_assert(BGeo<DGRAD_A, 256>::SMEM <= 227 * 1024 && BGeo<DGRAD_X, 256>::SMEM <= 227 * 1024 &&
                   BGeo<WGRAD_2, 256>::SMEM <= 227 * 1024 && BGeo<WGRAD_1, 256>::SMEM <= 227 * 1024,
               "smem");
 static_assert(BGeo<DGRAD_A, 128>::NBARS * 8 + 4 * (2 + kRing) + 4 * 128 <= kMetaBytes, "meta");
@@ -314,11 +314,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       const BItem w = decode_item<KIND, BN>(a, L);
       if (!w.run) continue;
       if (KIND == WGRAD_2 || KIND == WGRAD_1) {
-        float* out = a.dw + ((long long)w.e * a.n_m * kBM + w.m0 + rit) * a.n_out + w.n0;
-        if (w.zero) {  // idle expert: its gradient is zero
+        if (w.zero) {  // idle expert: its gradient is zero (the warp's 32 rows, coalesced)
+          float* out0 =
+              a.dw + ((long long)w.e * a.n_m * kBM + w.m0 + quarter * 32) * a.n_out + w.n0;
           const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-          for (int i = 0; i < BN / 4; ++i) reinterpret_cast<float4*>(out)[i] = z4;
+          for (int r = 0; r < 32; ++r)
+            for (int i = lane; i < BN / 4; i += 32)
+              reinterpret_cast<float4*>(out0 + (long long)r * a.n_out)[i] = z4;
           continue;
         }
       }
@@ -330,45 +332,61 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
       if (KIND == DGRAD_A) {
-        // dZ = [dA * U * SiLU'(G), dA * SiLU(G)] for the n-tile's BN columns of G and U
-        const long long row = (long long)w.row0 + rit;
-        const bool valid = rit < w.nrows && row < a.r_max;
-        const uint16_t* zrow = a.z + row * 2 * a.f;
-        uint16_t* dzrow = a.dz + row * 2 * a.f;
+        // dZ = [dA * U * SiLU'(G), dA * SiLU(G)] for the n-tile's BN columns of G and U.
+        // Each 32 x 32 chunk of dA goes through shared memory; then lanes 8q..8q+7 take
+        // four columns each of one row, so a warp's loads of G and U and stores of dG and
+        // dU each cover four whole 64-byte row segments.
+        float* my_row = stg + (ew * 32 + lane) * kStgStride;
+        const int rq = lane >> 3, cq = 4 * (lane & 7);
+        bool rvalid[8];
+        long long rrow[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = quarter * 32 + 4 * i + rq;
+          rrow[i] = (long long)w.row0 + r;
+          rvalid[i] = r < w.nrows && rrow[i] < a.r_max;
+        }
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(taddr + c * 32, v);
           tmem_wait_ld();
-          if (valid) {
-            const int col = w.n0 + 32 * c;
-            uint4 gz[4], uz[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              gz[i] = __ldg(reinterpret_cast<const uint4*>(zrow + col) + i);
-              uz[i] = __ldg(reinterpret_cast<const uint4*>(zrow + a.f + col) + i);
-            }
-            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gz);
-            const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uz);
-            uint32_t pg[16], pu[16];
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4*>(my_row + 4 * j) =
+                make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                            __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          __syncwarp();
+          const int col = w.n0 + 32 * c + cq;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float2 g = __bfloat1622float2(g2[i]);
-              const float2 u = __bfloat1622float2(u2[i]);
-              const float da0 = __uint_as_float(v[2 * i]), da1 = __uint_as_float(v[2 * i + 1]);
-              const float s0 = 1.0f / (1.0f + __expf(-g.x)), s1 = 1.0f / (1.0f + __expf(-g.y));
-              pg[i] = pack_bf16(da0 * u.x * (s0 * (1.0f + g.x * (1.0f - s0))),
-                                da1 * u.y * (s1 * (1.0f + g.y * (1.0f - s1))));
-              pu[i] = pack_bf16(da0 * g.x * s0, da1 * g.y * s1);
-            }
-            uint4* dg = reinterpret_cast<uint4*>(dzrow + col);
-            uint4* du = reinterpret_cast<uint4*>(dzrow + a.f + col);
+          for (int i = 0; i < 8; ++i) {
+            if (!rvalid[i]) continue;
+            const float4 da = *reinterpret_cast<const float4*>(
+                stg + (ew * 32 + 4 * i + rq) * kStgStride + cq);
+            const uint16_t* zrow = a.z + rrow[i] * 2 * a.f;
+            const uint2 gz = __ldg(reinterpret_cast<const uint2*>(zrow + col));
+            const uint2 uz = __ldg(reinterpret_cast<const uint2*>(zrow + a.f + col));
+            const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gz.x));
+            const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gz.y));
+            const float2 u01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uz.x));
+            const float2 u23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uz.y));
+            const float gs[4] = {g01.x, g01.y, g23.x, g23.y};
+            const float us[4] = {u01.x, u01.y, u23.x, u23.y};
+            const float ds[4] = {da.x, da.y, da.z, da.w};
+            float dg[4], du[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              dg[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
-              du[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+            for (int q = 0; q < 4; ++q) {
+              const float sg = 1.0f / (1.0f + __expf(-gs[q]));
+              dg[q] = ds[q] * us[q] * (sg * (1.0f + gs[q] * (1.0f - sg)));
+              du[q] = ds[q] * gs[q] * sg;
             }
+            uint16_t* dzrow = a.dz + rrow[i] * 2 * a.f;
+            *reinterpret_cast<uint2*>(dzrow + col) =
+                make_uint2(pack_bf16(dg[0], dg[1]), pack_bf16(dg[2], dg[3]));
+            *reinterpret_cast<uint2*>(dzrow + a.f + col) =
+                make_uint2(pack_bf16(du[0], du[1]), pack_bf16(du[2], du[3]));
           }
+          __syncwarp();
         }
       } else if (KIND == DGRAD_X) {
         // dx[token] += dX, staged per 32 x 32 chunk so that one vector reduction of 8 lanes
@@ -405,8 +423,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
           __syncwarp();
         }
       } else {
-        // WGrad: row m0 + rit of expert e's gradient, BN fp32 columns
-        float* out = a.dw + ((long long)w.e * a.n_m * kBM + w.m0 + rit) * a.n_out + w.n0;
+        // WGrad: rows m0 + 32 quarter .. of expert e's gradient, BN fp32 columns; each
+        // 32 x 32 chunk goes through shared memory so that one store instruction writes
+        // four whole 128-byte row segments
+        float* my_row = stg + (ew * 32 + lane) * kStgStride;
+        float* out0 = a.dw + ((long long)w.e * a.n_m * kBM + w.m0 + quarter * 32) * a.n_out +
+                      w.n0 + 4 * (lane & 7);
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
@@ -414,9 +436,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            reinterpret_cast<float4*>(out + 32 * c)[j] =
+            *reinterpret_cast<float4*>(my_row + 4 * j) =
                 make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + (lane >> 3);
+            *reinterpret_cast<float4*>(out0 + (long long)r * a.n_out + 32 * c) =
+                *reinterpret_cast<const float4*>(stg + (ew * 32 + r) * kStgStride +
+                                                 4 * (lane & 7));
+          }
+          __syncwarp();
         }
       }
       tc_fence_before();
@@ -542,15 +573,20 @@ cudaError_t launch_ffn_backward(const moe_cfg& c, const uint16_t* xp, const uint
   base.beta = c.beta;
   base.timeout_ns = kWaitNs;
 
-  // dA = D w2 (N = f in tiles of 128, K = d) with the SwiGLU backward -> dZ
+  // dA = D w2 (N = f in tiles of 256, or 128, K = d) with the SwiGLU backward -> dZ
   BwdArgs g1 = base;
   g1.sched = sched + 0;
   g1.z = z_saved;
   g1.dz = dz;
   g1.n_k = c.d / kBK;
-  g1.n_n = c.f / 128;
   g1.k_rows = c.d;
-  err = launch_bwd<DGRAD_A, 128>(m_d_k, m_w2, g1, st);
+  if (c.f % 256 == 0) {
+    g1.n_n = c.f / 256;
+    err = launch_bwd<DGRAD_A, 256>(m_d_k, m_w2, g1, st);
+  } else {
+    g1.n_n = c.f / 128;
+    err = launch_bwd<DGRAD_A, 128>(m_d_k, m_w2, g1, st);
+  }
   if (err != cudaSuccess) return err;
   // dX = dZ w1 (N = d in tiles of 256, K = 2f), scattered into dx
   BwdArgs g2 = base;
