@@ -501,8 +501,11 @@ template <int KIND, int BN>
 cudaError_t launch_bwd(const CUtensorMap& ta, const CUtensorMap& tb, const BwdArgs& args,
                        cudaStream_t st) {
   auto kern = bwd_kernel<KIND, BN>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         BGeo<KIND, BN>::SMEM);
+  static OncePerDevice attr_once;
+  cudaError_t err = once_per_device(attr_once, [&](int&) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                BGeo<KIND, BN>::SMEM);
+  });
   if (err != cudaSuccess) return err;
   kern<<<num_sms(), kThreads, BGeo<KIND, BN>::SMEM, st>>>(ta, tb, args);
   return cudaGetLastError();

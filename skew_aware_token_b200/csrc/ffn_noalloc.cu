@@ -26,7 +26,6 @@ namespace {
 
 static __device__ __align__(256) uint8_t g_ffn_scratch[MOE_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 

@@ -682,9 +682,11 @@ template <int PHASE, bool PAIR>
 cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ta64,
                        const FfnArgs& args, cudaStream_t st) {
   auto kern = ffn_kernel<PHASE, PAIR>;
-  cudaError_t err =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Geo<PHASE, PAIR>::SMEM);
+  static OncePerDevice attr_once;
+  cudaError_t err = once_per_device(attr_once, [&](int&) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Geo<PHASE, PAIR>::SMEM);
+  });
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -700,7 +702,10 @@ cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUten
     cfg.numAttrs = 1;
     cfg.gridDim = dim3(2);
     int clusters = 0;
-    err = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+    static OncePerDevice occ_once;
+    err = once_per_device(occ_once, [&](int& n) {
+      return cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    }, &clusters);
     if (err != cudaSuccess) return err;
     if (clusters < 1) return cudaErrorInvalidConfiguration;
     cfg.gridDim = dim3(2 * clusters);

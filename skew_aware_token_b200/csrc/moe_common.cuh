@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "moeskew.h"
 
 namespace moe {
@@ -42,6 +44,37 @@ inline long long ffn_scratch_z_bytes(const moe_cfg& c) {
 }
 // backward scratch: dZ, then the counters of its four launches
 inline long long bwd_scratch_bytes(const moe_cfg& c) { return ffn_z_bytes(c) + kSchedBytes; }
+
+// Once per device for one call site: `f(int& value)` runs on the first call made with that
+// device current, and every later call returns its result (and value).  Used for kernel
+// attributes and occupancy queries, so that a launch sequence can be captured into a CUDA
+// graph with nothing but stream work inside it.
+constexpr int kMaxDevices = 64;
+struct OncePerDevice {
+  std::mutex m;
+  bool done[kMaxDevices] = {};
+  cudaError_t err[kMaxDevices] = {};
+  int value[kMaxDevices] = {};
+};
+template <class F>
+cudaError_t once_per_device(OncePerDevice& o, F&& f, int* value = nullptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) {
+    int v = 0;
+    e = f(v);
+    if (value) *value = v;
+    return e;
+  }
+  std::lock_guard<std::mutex> lock(o.m);
+  if (!o.done[dev]) {
+    o.err[dev] = f(o.value[dev]);
+    o.done[dev] = true;
+  }
+  if (value) *value = o.value[dev];
+  return o.err[dev];
+}
 
 __device__ __forceinline__ void set_status(int32_t* status, int bits) {
   atomicOr(status, bits);

@@ -552,12 +552,15 @@ cudaError_t launch_plan(const moe_cfg& c, const int32_t* counts, uint32_t mask,
   const size_t words = (size_t)E + (E + 1) + kVariants * ((size_t)E * P + kMaxP + E + kMaxP) +
                        40 + 40;
   const size_t bytes = words * sizeof(int);
-  if (bytes > 48 * 1024) {
-    cudaError_t err = cudaFuncSetAttribute(plan_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)bytes);
-    if (err != cudaSuccess) return err;
-  }
+  // allow the largest configuration once per device (E = 256 experts, P = 8 slots)
+  static OncePerDevice attr_once;
+  cudaError_t err = once_per_device(attr_once, [](int&) {
+    const size_t most = (size_t)kMaxE + (kMaxE + 1) +
+                        kVariants * ((size_t)kMaxE * kMaxP + kMaxP + kMaxE + kMaxP) + 40 + 40;
+    return cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)(most * sizeof(int)));
+  });
+  if (err != cudaSuccess) return err;
   const unsigned all = (1u << kVariants) - 1u;
   const unsigned m = (mask & all) ? (mask & all) : 0xFu;  // default: the four greedy searches
   const int u_min = (mask >> 8 & 0xFFu) ? (int)(mask >> 8 & 0xFFu) : 1;

@@ -182,6 +182,37 @@ class MoeLayer:
         return buf[:n].view(*shape)
 
 
+class LayerGraph:
+    """One forward of a MoeLayer (route, plan, dispatch, FFN and, unfused, the combine)
+    captured into a CUDA graph: replay() runs it again on whatever `logits` and `x` hold,
+    with one launch from the host.  The layer's own buffers hold the results.
+
+        g = LayerGraph(layer, w1, w2)
+        g.logits.copy_(logits); g.x.copy_(x); g.replay(); y = layer.view("y")
+    """
+
+    def __init__(self, layer: MoeLayer, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, variant_mask=0,
+                 warmup: int = 2):
+        wl, dev = layer.wl, layer.device
+        self.layer = layer
+        self.logits = torch.zeros(wl.T, wl.E, device=dev)
+        self.x = torch.zeros(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
+        run = lambda: layer(self.logits, self.x, w1, w2, mode=mode, variant_mask=variant_mask)
+        # warm up off the capture (the library sets its kernels' attributes on first use)
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            for _ in range(warmup):
+                run()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            run()
+
+    def replay(self):
+        self.graph.replay()
+
+
 class HostPipeline:
     """Runs a MoeLayer over a stream of batches held in pinned host memory, overlapping
     the host-to-device copy of batch i+1 and the device-to-host copy of batch i-1 with the

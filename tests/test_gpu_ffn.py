@@ -155,3 +155,25 @@ def test_host_pipeline_matches_direct_calls():
     for logits_h, x_h, y_h in batches:
         want = layer(logits_h.cuda(), x_h.cuda(), w1, w2).cpu()
         torch.testing.assert_close(y_h, want, rtol=1e-5, atol=1e-6)
+
+
+def test_graph_replay_matches_direct_calls():
+    """The whole layer captured into a CUDA graph gives, batch by batch, what direct calls
+    give (the fused combine's atomics may reorder the last bits)."""
+    from skew_aware_token_b200.layer import LayerGraph
+    wl = FULL_CASES[2]
+    w1, w2 = synth.make_weights(wl, "cuda")
+    layer = MoeLayer(wl, "cuda")
+    g = LayerGraph(layer, w1, w2)
+    direct = MoeLayer(wl, "cuda")
+    for seed in range(3):
+        b = wl.with_(seed=seed)
+        logits, x = synth.make_logits(b).cuda(), synth.make_x(b).cuda()
+        g.logits.copy_(logits)
+        g.x.copy_(x)
+        g.replay()
+        want = direct(logits, x, w1, w2)
+        torch.cuda.synchronize()
+        assert layer.read_status() == 0
+        torch.testing.assert_close(layer.view("y"), want, rtol=1e-5, atol=1e-6)
+        assert torch.equal(layer.view("q"), direct.view("q"))
