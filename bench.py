@@ -169,15 +169,25 @@ def cpu_cores():
 
 def time_oracle(wl, logits_np, x_np, get_expert, budget_s):
     """Times the oracle on the first n tokens, n grown until one run takes about budget_s
-    seconds of CPU work (or covers the whole workload).  Returns (n, seconds)."""
+    seconds of CPU work; when the whole workload runs faster than that, whole-layer runs
+    are repeated until about budget_s has passed.  Returns (n, runs, seconds): `runs` runs
+    over the first n tokens took `seconds` in total."""
     n = min(wl.T, 16)
     oracle_sample(wl, logits_np, x_np, get_expert, n)  # untimed: loads the first experts
     while True:
         t0 = time.perf_counter()
         oracle_sample(wl, logits_np, x_np, get_expert, n)
         dt = time.perf_counter() - t0
-        if n >= wl.T or dt >= 0.5 * budget_s:
-            return n, dt
+        if dt >= 0.5 * budget_s:
+            return n, 1, dt
+        if n >= wl.T:
+            runs, total = 1, dt
+            while total < budget_s:
+                t0 = time.perf_counter()
+                oracle_sample(wl, logits_np, x_np, get_expert, n)
+                total += time.perf_counter() - t0
+                runs += 1
+            return n, runs, total
         grow = budget_s / max(dt, 1e-6)
         n = int(min(wl.T, max(n + 1, n * min(grow, 8.0))))
 
@@ -387,14 +397,13 @@ def run_ours(args, wl, world, rank, local):
         e2e = run_e2e(layer, logits_h, x_h, w1, w2, mode, wl, args, world, dev)
 
     cpu = None
-    cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n, dt = time_oracle(wl, logits_h.numpy(), x_h.float().numpy(),
-                            host_expert_getter(w1, w2), args.cpu_budget)
-        cpu = {"value": n * wl.k / dt, "unit": "tokens/s", "cores": cpu_cores(),
+        n, runs, dt = time_oracle(wl, logits_h.numpy(), x_h.float().numpy(),
+                                  host_expert_getter(w1, w2), args.cpu_budget)
+        cpu = {"value": n * wl.k * runs / dt, "unit": "tokens/s", "cores": cpu_cores(),
                "kind": "oracle",
-               "sample": f"first {n} of {wl.T} tokens of {wl.name}, whole layer, one run "
-                         f"({dt:.1f} s, numpy fp32 + OpenBLAS)"}
+               "sample": f"first {n} of {wl.T} tokens of {wl.name}, whole layer, {runs} "
+                         f"run{'s' if runs > 1 else ''} ({dt:.1f} s, numpy fp32 + OpenBLAS)"}
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -443,7 +452,7 @@ def run_reference(args, wl, world, rank):
 
     logits_np, x_np = logits_h.numpy(), x_h.float().numpy()
     total = args.warmup + args.steps
-    n, dt = time_oracle(wl, logits_np, x_np, get_expert, max(0.05, args.ref_budget / total))
+    n, _, _ = time_oracle(wl, logits_np, x_np, get_expert, max(0.05, args.ref_budget / total))
     for _ in range(args.warmup):
         oracle_sample(wl, logits_np, x_np, get_expert, n)
     t0 = time.perf_counter()
