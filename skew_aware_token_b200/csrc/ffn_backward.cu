@@ -358,14 +358,21 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
           __syncwarp();
           const int col = w.n0 + 32 * c + cq;
+          // all sixteen loads of the chunk in flight at once (rows outside the tile read the
+          // tile's first row and store nothing)
+          uint2 gzs[8], uzs[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint16_t* zrow = a.z + (rvalid[i] ? rrow[i] : (long long)w.row0) * 2 * a.f;
+            gzs[i] = __ldg(reinterpret_cast<const uint2*>(zrow + col));
+            uzs[i] = __ldg(reinterpret_cast<const uint2*>(zrow + a.f + col));
+          }
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             if (!rvalid[i]) continue;
             const float4 da = *reinterpret_cast<const float4*>(
                 stg + (ew * 32 + 4 * i + rq) * kStgStride + cq);
-            const uint16_t* zrow = a.z + rrow[i] * 2 * a.f;
-            const uint2 gz = __ldg(reinterpret_cast<const uint2*>(zrow + col));
-            const uint2 uz = __ldg(reinterpret_cast<const uint2*>(zrow + a.f + col));
+            const uint2 gz = gzs[i], uz = uzs[i];
             const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gz.x));
             const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gz.y));
             const float2 u01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uz.x));
