@@ -252,6 +252,19 @@ def measured_traffic(workload: str):
     return rec["bytes_per_step"]
 
 
+def ffn_one_launch(wl, mode, dev) -> bool:
+    """Whether moe_expert_ffn runs FC1 and FC2 as one launch for this mode (its rule: forced
+    by MOE_FFN_ONE_LAUNCH, else for a fused single-SM Xp call with at most 32 FC1 work items
+    per SM)."""
+    if mode & N.MOE_FFN_ONE_LAUNCH:
+        return True
+    if mode & (N.MOE_FFN_WRITE_O | N.MOE_FFN_STRICT_SLOTS | N.MOE_FFN_SM_PAIR |
+               N.MOE_FFN_GATHER_X | N.MOE_FFN_TWO_LAUNCHES):
+        return False
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    return wl.T * wl.k // 128 * (wl.f // 128) <= 32 * sms
+
+
 def run_backward(layer, w1, w2, wl, args, dev, peak, peak_src):
     """Times the backward of the expert computation (moe_dispatch_grad, then the four
     gradient GEMMs of moe_expert_ffn_backward) after the layer's last forward: 12 N d f
@@ -303,7 +316,9 @@ def run_ours(args, wl, world, rank, local):
     layer = MoeLayer(wl, dev, write_o=write_o, gather_x=args.gather_x, train=args.backward)
     stream = torch.cuda.current_stream(dev)
     mode = ((N.MOE_FFN_STRICT_SLOTS if args.strict else 0) |
-            (N.MOE_FFN_WRITE_O if write_o else 0) | (N.MOE_FFN_SM_PAIR if args.sm_pair else 0))
+            (N.MOE_FFN_WRITE_O if write_o else 0) | (N.MOE_FFN_SM_PAIR if args.sm_pair else 0) |
+            (N.MOE_FFN_ONE_LAUNCH if args.launches == "one" else 0) |
+            (N.MOE_FFN_TWO_LAUNCHES if args.launches == "two" else 0))
     vmask = args.variant_mask
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
@@ -414,6 +429,7 @@ def run_ours(args, wl, world, rank, local):
                 "weights N(0, 1/sqrt(fan_in)), random-init)",
         "config": workload_config(wl, {"kappa": kappa, "strict_slots": bool(args.strict),
                                        "ffn": args.ffn, "sm_pair": bool(args.sm_pair),
+                                       "ffn_launches": args.launches,
                                        "launch": "cuda graph replay" if args.graph else "stream launches",
                                        "fc1_rows": "gathered from x by row_token"
                                        if args.gather_x else "Xp (dispatched copy)",
@@ -428,7 +444,8 @@ def run_ours(args, wl, world, rank, local):
         "roofline": roofline, "cpu_baseline": cpu,
         "e2e": e2e,
         "backward": backward,
-        "gpu_launches": (LAUNCHES_PER_STEP + int(write_o) - int(args.gather_x)) * args.steps,
+        "gpu_launches": (LAUNCHES_PER_STEP + int(write_o) - int(args.gather_x) -
+                         int(ffn_one_launch(wl, mode, dev))) * args.steps,
         "clocks": clocks.summary(),
         "impl": "ours",
     }
@@ -499,6 +516,9 @@ def main():
     ap.add_argument("--backward", action="store_true",
                     help="also time the backward of the expert computation (the forward then "
                          "keeps Z for it)")
+    ap.add_argument("--launches", default="auto", choices=["auto", "one", "two"],
+                    help="FC1 and FC2 in one persistent launch (per-tile-half readiness), two "
+                         "launches, or the library's choice by layer size (default)")
     ap.add_argument("--gather-x", action="store_true",
                     help="FC1 gathers its rows from x by row_token (no Xp, no gather kernel)")
     ap.add_argument("--ffn", default="fused", choices=["fused", "write_o"],

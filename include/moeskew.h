@@ -122,6 +122,16 @@ enum {
                                 A and the counters in a_scratch, which must then hold
                                 moe_workspace_size(cfg, MOE_WS_FFN_SCRATCH_Z) bytes; the
                                 backward pass reads A and Z from there */
+  MOE_FFN_ONE_LAUNCH = 32,   /* flag: FC1 and FC2 in one persistent launch; FC2's work on
+                                a tile half starts once FC1's epilogues have published all
+                                of its A rows (per-half counters, bounded waits).  With the
+                                fused combine, single-SM tiles and Xp only: combined with
+                                WRITE_O, STRICT_SLOTS, SM_PAIR or GATHER_X the call returns
+                                MOE_ERR_INVALID_ARG.  Without this flag or
+                                MOE_FFN_TWO_LAUNCHES, a fused single-SM Xp call takes one
+                                launch when FC1 has at most 32 work items (128 x 128 tiles,
+                                padding aside) per SM, two launches otherwise */
+  MOE_FFN_TWO_LAUNCHES = 64, /* flag: FC1 and FC2 as two launches (never one) */
   MOE_FFN_GATHER_X = 8       /* flag: the `xp` argument is x itself (bf16 [T, d]); FC1
                                 gathers each tile's rows x[row_token[r]] straight into
                                 shared memory (TMA row gather), so the dispatched copy
@@ -133,7 +143,8 @@ enum {
 /* Upper bounds: which = MOE_WS_ROWS -> R_max rows (Xp, A, O, row_token, row_gate);
  * MOE_WS_BLOCKS -> B_max entries (blocks, tiles); MOE_WS_FFN_SCRATCH -> bytes of the
  * a_scratch buffer of moe_expert_ffn (A, bf16 [R_max, f], rounded up to 256 bytes, then
- * 256 bytes of tile-scheduler counters); MOE_WS_FFN_SCRATCH_Z -> the same followed by
+ * 256 bytes of tile-scheduler counters, then 2 * B_max int32 readiness counters rounded
+ * up to 256 bytes); MOE_WS_FFN_SCRATCH_Z -> the same followed by
  * Z (bf16 [R_max, 2f], rounded up to 256 bytes); MOE_WS_BWD_SCRATCH -> bytes of the
  * bwd_scratch buffer of moe_expert_ffn_backward (dZ, bf16 [R_max, 2f], rounded up to 256
  * bytes, then 256 bytes of counters).  Returns 0 for an invalid cfg. */

@@ -90,11 +90,12 @@ struct Geo {
   static constexpr uint32_t IDESC = idesc(M);
   static constexpr uint32_t IDESC_M128 = idesc(BM);  // SM pair: a tile of at most 128 rows
   static constexpr int NBARS = 2 * STAGES + 5 + 2 * RING;
-  static constexpr int STG = PHASE == 2 ? STG_BYTES : 0;  // FC2 combine staging
+  static constexpr int STG = PHASE >= 2 ? STG_BYTES : 0;  // FC2 combine staging
   static constexpr int SMEM = STAGES * STAGE_BYTES + STG + META_BYTES + 1024;
 };
 static_assert(Geo<1, true>::SMEM <= 227 * 1024 && Geo<2, true>::SMEM <= 227 * 1024 &&
-                  Geo<1, false>::SMEM <= 227 * 1024 && Geo<2, false>::SMEM <= 227 * 1024,
+                  Geo<1, false>::SMEM <= 227 * 1024 && Geo<2, false>::SMEM <= 227 * 1024 &&
+                  Geo<3, false>::SMEM <= 227 * 1024,
               "smem");
 static_assert(Geo<1, true>::NBARS * 8 + 4 * (2 + RING) + 4 * 128 <= META_BYTES, "meta");
 
@@ -114,6 +115,12 @@ struct FfnArgs {
   int write_o;   // FC2: store O (1) or fused combine (0)
   uint16_t* z;   // FC1 with MOE_FFN_SAVE_Z: Z = [G, U] bf16 [r_max, 2f] (else null)
   const void* x; // the token rows x bf16 [T, d] (gather)
+  // PHASE 3 (FC1 and FC2 in one launch): FC2's K steps, n-tiles, output and row length,
+  // and the per-(tile, half) readiness counters FC1's epilogue raises to ready_target
+  int n_k2, n_n2, out_ld2;
+  void* out2;
+  int32_t* ready;
+  int ready_target;
   int strict;
   unsigned long long timeout_ns;
 };
@@ -123,12 +130,26 @@ struct FfnArgs {
 struct Sched {
   int32_t* counter;  // global counter this unit draws items from
   long long total;   // items in its range
-  int m_base, n_n, halves;
+  long long total1;  // PHASE 3: the first total1 items are FC1's, the rest FC2's
+  int m_base, n_n, n_n2, halves;
   __device__ void decode(int L, int& m, int& n, int& half) const {
     n = L % n_n;
     const int t = L / n_n;
     m = m_base + t / halves;
     half = t % halves;
+  }
+  // PHASE 3: also which GEMM the item belongs to (1: FC1, 2: FC2)
+  __device__ int decode_phase(int L, int& m, int& n, int& half) const {
+    if (L < total1) {
+      decode(L, m, n, half);
+      return 1;
+    }
+    const int L2 = (int)(L - total1);
+    n = L2 % n_n2;
+    const int t = L2 / n_n2;
+    m = t / halves;
+    half = t % halves;
+    return 2;
   }
 };
 
@@ -139,10 +160,16 @@ __device__ Sched make_sched(const FfnArgs& a) {
   s.halves = PAIR ? 1 : 2;
   const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int* pi = a.plan_info;
+  s.n_n2 = a.n_n2;
+  s.total1 = 1LL << 62;
   if (!a.strict) {
     s.counter = a.sched;
     s.total = (long long)max(pi[MOE_PI_NTILES], 0) * a.n_n * s.halves;
     s.m_base = 0;
+    if (a.n_n2 > 0) {  // PHASE 3: FC2's items after FC1's
+      s.total1 = s.total;
+      s.total += (long long)max(pi[MOE_PI_NTILES], 0) * a.n_n2 * s.halves;
+    }
   } else {
     const int r = unit % a.P;
     const int lo = pi[MOE_PI_SLOT_TILE_OFF + r], hi = pi[MOE_PI_SLOT_TILE_OFF + r + 1];
@@ -183,7 +210,8 @@ __device__ __forceinline__ TileInfo read_tile(const FfnArgs& a, int m, int part)
 template <int PHASE, bool PAIR, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1)
 ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-           const __grid_constant__ CUtensorMap tmA64, const FfnArgs a) {
+           const __grid_constant__ CUtensorMap tmA64, const __grid_constant__ CUtensorMap tmA2,
+           const __grid_constant__ CUtensorMap tmB2, const FfnArgs a) {
   using G = Geo<PHASE, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -235,6 +263,10 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
     if (PAIR) prefetch_tmap(&tmA64);
+    if (PHASE == 3) {
+      prefetch_tmap(&tmA2);
+      prefetch_tmap(&tmB2);
+    }
   }
   if (warp == 1) tmem_alloc<PAIR, TMEM_COLS>(smem_u32(tmem_slot));
   tc_fence_before();
@@ -275,19 +307,29 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         }
         if (L < 0) break;
         int m, n, half;
-        sch.decode(L, m, n, half);
+        const int gp = PHASE == 3 ? sch.decode_phase(L, m, n, half) : (sch.decode(L, m, n, half), PHASE);
         const TileInfo ti = read_tile<PAIR>(a, m, PAIR ? (int)rank : half);
         if (!ti.ok) bad_tile = true;
         if (!ti.run) continue;
         // FC1 B rows: single SM, the n-tile's 128 G rows over its 128 U rows; SM pair, CTA
         // `rank` holds G rows [64 rank, +64) of the n-tile over the matching U rows
         int brow;
-        if (PHASE == 1) brow = ti.e * 2 * a.f + n * (BN / 2) + (PAIR ? (int)rank * (BN / 4) : 0);
+        if (gp == 1) brow = ti.e * 2 * a.f + n * (BN / 2) + (PAIR ? (int)rank * (BN / 4) : 0);
         else brow = ti.e * a.d + n * BN + (PAIR ? (int)rank * (BN / 2) : 0);
         uint32_t tx = G::TX_BYTES;
         if (PAIR && ti.m128) tx = 2 * (A_BYTES / 2 + G::B_BYTES);  // 64 A rows per CTA
+        const CUtensorMap* mapA = (PHASE == 3 && gp == 2) ? &tmA2 : &tmA;
+        const CUtensorMap* mapB = (PHASE == 3 && gp == 2) ? &tmB2 : &tmB;
+        const int nk = (PHASE == 3 && gp == 2) ? a.n_k2 : a.n_k;
+        if (PHASE == 3 && gp == 2) {
+          // FC2 reads A rows of this tile half: wait until FC1 wrote all of them
+          if (!wait_count(a.ready + (2 * m + half), a.ready_target, abort_flag, a.status,
+                          a.timeout_ns))
+            break;
+          fence_proxy_async_global();
+        }
         bool stop = false;
-        for (int kb = 0; kb < a.n_k; ++kb) {
+        for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status, a.timeout_ns,
                          true)) {
             stop = true;
@@ -301,10 +343,10 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             if (PHASE == 1)
               tma_load_2d_pair(sB(stage) + G::B_BYTES / 2, &tmB, fb, kb * BK, brow + a.f);
           } else {
-            tma_load_2d(sA(stage), &tmA, full_bar(stage), kb * BK, ti.a_row);
-            tma_load_2d(sB(stage), &tmB, full_bar(stage), kb * BK, brow);
-            if (PHASE == 1)
-              tma_load_2d(sB(stage) + G::B_BYTES / 2, &tmB, full_bar(stage), kb * BK,
+            tma_load_2d(sA(stage), mapA, full_bar(stage), kb * BK, ti.a_row);
+            tma_load_2d(sB(stage), mapB, full_bar(stage), kb * BK, brow);
+            if (gp == 1)
+              tma_load_2d(sB(stage) + G::B_BYTES / 2, mapB, full_bar(stage), kb * BK,
                           brow + a.f);
           }
           pending |= 1u << stage;
@@ -546,9 +588,10 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         mbar_arrive(iempty_bar(slot));
         if (L < 0) break;
         int m, n, half;
-        sch.decode(L, m, n, half);
+        const int gp = PHASE == 3 ? sch.decode_phase(L, m, n, half) : (sch.decode(L, m, n, half), PHASE);
         const TileInfo ti = read_tile<PAIR>(a, m, PAIR ? 0 : half);
         if (!ti.run) continue;
+        const int nk = (PHASE == 3 && gp == 2) ? a.n_k2 : a.n_k;
         const int buf = acc_it & 1;
         const uint32_t use = (uint32_t)(acc_it >> 1) & 1u;
         if (!mbar_wait(tempty_bar(buf), use ^ 1u, abort_flag, a.status, a.timeout_ns, true))
@@ -557,7 +600,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
         const uint32_t idesc = ti.m128 ? G::IDESC_M128 : G::IDESC;
         bool stop = false;
-        for (int kb = 0; kb < a.n_k; ++kb) {
+        for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, a.status, a.timeout_ns, true)) {
             stop = true;
             break;
@@ -606,9 +649,11 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       }
       if (L < 0) break;
       int m, n, half;
-      sch.decode(L, m, n, half);
+      const int gp = PHASE == 3 ? sch.decode_phase(L, m, n, half) : (sch.decode(L, m, n, half), PHASE);
       const TileInfo ti = read_tile<PAIR>(a, m, PAIR ? (int)rank : half);
       if (!ti.run) continue;
+      void* const outp = (PHASE == 3 && gp == 2) ? a.out2 : a.out;
+      const int out_ld = (PHASE == 3 && gp == 2) ? a.out_ld2 : a.out_ld;
       const int buf = acc_it & 1;
       const uint32_t use = (uint32_t)(acc_it >> 1) & 1u;
       const bool got =
@@ -625,12 +670,12 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       const long long row = (long long)ti.row0 + lrow;
       const bool valid = lrow < ti.nrows && row < a.r_max;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-      if (PHASE == 1) {
+      if (gp == 1) {
         // chunk cc: G at TMEM column gcol, U at ucol, giving A columns [ocol, ocol + 32) of
         // the n-tile.  Single SM: B held the n-tile's 128 G rows over its 128 U rows.  SM
         // pair: CTA r's B half held G rows [64 r, +64) over the matching U rows, so
         // accumulator columns [128 r, +64) are G and [128 r + 64, +64) are U.
-        __nv_bfloat16* A = reinterpret_cast<__nv_bfloat16*>(a.out) + row * a.out_ld + n * (BN / 2);
+        __nv_bfloat16* A = reinterpret_cast<__nv_bfloat16*>(outp) + row * out_ld + n * (BN / 2);
         const int ncc = m128 ? 2 : 4;
 #pragma unroll 1
         for (int cc = 0; cc < ncc; ++cc) {
@@ -683,11 +728,19 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             }
           }
         }
+        if (PHASE == 3) {
+          // publish this warp's A rows of the tile half to FC2's producers (other CTAs
+          // read them with TMA, through the async proxy)
+          fence_proxy_async_global();
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) atomicAdd(a.ready + (2 * m + half), 1);
+        }
       } else if (a.write_o) {
         // chunk c: TMEM columns [32 c, +32) = output columns n BN + ocol0 + 32 c ..
         const int ncc = m128 ? 4 : 8, ocol0 = 128 * chalf;
-        __nv_bfloat16* O = reinterpret_cast<__nv_bfloat16*>(a.out);
-        uint4* dst = reinterpret_cast<uint4*>(O + row * a.out_ld + n * BN + ocol0);
+        __nv_bfloat16* O = reinterpret_cast<__nv_bfloat16*>(outp);
+        uint4* dst = reinterpret_cast<uint4*>(O + row * out_ld + n * BN + ocol0);
 #pragma unroll 1
         for (int c = 0; c < ncc; ++c) {
           uint32_t v[32];
@@ -716,7 +769,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         }
         s_tok[ew * 32 + lane] = tok;
         float* my_row = stg + (ew * 32 + lane) * STG_STRIDE;
-        float* y = reinterpret_cast<float*>(a.out) + n * BN + ocol0 + 4 * (lane & 7);
+        float* y = reinterpret_cast<float*>(outp) + n * BN + ocol0 + 4 * (lane & 7);
         __syncwarp();
 #pragma unroll 1
         for (int c = 0; c < ncc; ++c) {
@@ -736,7 +789,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             if (tk >= 0) {
               const float4 x = *reinterpret_cast<const float4*>(
                   stg + (ew * 32 + r) * STG_STRIDE + 4 * (lane & 7));
-              red_add_v4(y + (long long)tk * a.out_ld + c * 32, x);
+              red_add_v4(y + (long long)tk * out_ld + c * 32, x);
             }
           }
           __syncwarp();
@@ -763,7 +816,8 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 // ------------------------------------------------------------------ host side
 template <int PHASE, bool PAIR, bool GATHER = false>
 cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ta64,
-                       const FfnArgs& args, cudaStream_t st) {
+                       const CUtensorMap& ta2, const CUtensorMap& tb2, const FfnArgs& args,
+                       cudaStream_t st) {
   auto kern = ffn_kernel<PHASE, PAIR, GATHER>;
   static OncePerDevice attr_once;
   cudaError_t err = once_per_device(attr_once, [&](int&) {
@@ -798,7 +852,7 @@ cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUten
   FfnArgs a = args;
   const int units = PAIR ? (int)cfg.gridDim.x / 2 : (int)cfg.gridDim.x;
   a.strict = a.strict && units >= a.P;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, ta64, a);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, ta64, ta2, tb2, a);
 }
 
 }  // namespace
@@ -860,10 +914,10 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   a1.out_ld = c.f;
   a1.write_o = 0;
   a1.x = gather ? xp : nullptr;
-  // Z after A and the scheduler counters in the scratch buffer
+  // Z after A, the scheduler counters and the readiness counters in the scratch buffer
   a1.z = (mode & MOE_FFN_SAVE_Z)
              ? reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(a_scratch) +
-                                           ffn_a_bytes(c) + kSchedBytes)
+                                           ffn_scratch_bytes(c))
              : nullptr;
   a2.sched = sched + 8;
   a2.out = out;
@@ -872,15 +926,38 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   a2.out_ld = c.d;
   a2.write_o = write_o;
 
+  bool one_launch = (mode & MOE_FFN_ONE_LAUNCH) != 0;
+  if (!one_launch && !(mode & kOneLaunchExcludes)) {
+    // small layers: FC1's tail and FC2's ramp-up are a visible share of the time, and one
+    // launch overlaps them (measured about 4 % faster at up to ~20 items per SM, and
+    // slower from ~40 on)
+    const long long fc1_items = (long long)c.T * c.k / BM * (c.f / (BN / 2));
+    one_launch = fc1_items <= 32LL * num_sms();
+  }
+  if (one_launch) {
+    // FC1 items, then FC2 items, in one persistent launch; FC2 waits per tile half
+    int32_t* ready = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(a_scratch) +
+                                                ffn_a_bytes(c) + kSchedBytes);
+    err = cudaMemsetAsync(ready, 0, (size_t)ffn_ready_bytes(c), st);
+    if (err != cudaSuccess) return err;
+    FfnArgs a3 = a1;
+    a3.n_k2 = a2.n_k;
+    a3.n_n2 = a2.n_n;
+    a3.out2 = out;
+    a3.out_ld2 = a2.out_ld;
+    a3.ready = ready;
+    a3.ready_target = 4 * a1.n_n;  // four epilogue warps per FC1 n-tile of the half
+    return launch_one<3, false>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a3, st);
+  }
   if (gather)
-    err = pair ? launch_one<1, true, true>(tm_xp, tm_w1, tm_xp64, a1, st)
-               : launch_one<1, false, true>(tm_xp, tm_w1, tm_xp64, a1, st);
+    err = pair ? launch_one<1, true, true>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a1, st)
+               : launch_one<1, false, true>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a1, st);
   else
-    err = pair ? launch_one<1, true>(tm_xp, tm_w1, tm_xp64, a1, st)
-               : launch_one<1, false>(tm_xp, tm_w1, tm_xp64, a1, st);
+    err = pair ? launch_one<1, true>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a1, st)
+               : launch_one<1, false>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a1, st);
   if (err != cudaSuccess) return err;
-  return pair ? launch_one<2, true>(tm_a, tm_w2, tm_a64, a2, st)
-              : launch_one<2, false>(tm_a, tm_w2, tm_a64, a2, st);
+  return pair ? launch_one<2, true>(tm_a, tm_w2, tm_a64, tm_a, tm_w2, a2, st)
+              : launch_one<2, false>(tm_a, tm_w2, tm_a64, tm_a, tm_w2, a2, st);
 }
 
 }  // namespace moe

@@ -16,7 +16,11 @@ constexpr int kMaxP = 8;
 constexpr long long kMaxN = 1LL << 22;
 // every flag moe_expert_ffn accepts
 constexpr int kFfnModes = MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR |
-                          MOE_FFN_GATHER_X | MOE_FFN_SAVE_Z;
+                          MOE_FFN_GATHER_X | MOE_FFN_SAVE_Z | MOE_FFN_ONE_LAUNCH |
+                          MOE_FFN_TWO_LAUNCHES;
+// flags the one-launch FFN does not combine with
+constexpr int kOneLaunchExcludes = MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR |
+                                   MOE_FFN_GATHER_X | MOE_FFN_TWO_LAUNCHES;
 
 // Bound on the number of token blocks over every routing of N rows into E experts:
 // sum_e ceil(c_e / beta) <= (N + min(E, N) * (beta - 1)) / beta.
@@ -28,12 +32,18 @@ inline long long max_blocks(const moe_cfg& c) {
 inline long long max_rows(const moe_cfg& c) { return max_blocks(c) * c.beta; }
 
 // FFN scratch: A (bf16 [R_max, f]) rounded up to 256 bytes, then the tile-scheduler
-// counters (kSchedBytes).
+// counters (kSchedBytes), then the one-launch FFN's readiness counters.
 constexpr long long kSchedBytes = 256;
 inline long long ffn_a_bytes(const moe_cfg& c) {
   return (max_rows(c) * c.f * 2 + 255) / 256 * 256;
 }
-inline long long ffn_scratch_bytes(const moe_cfg& c) { return ffn_a_bytes(c) + kSchedBytes; }
+// readiness counters of the one-launch FFN: one per (tile, 128-row half), tiles <= B_max
+inline long long ffn_ready_bytes(const moe_cfg& c) {
+  return (2 * max_blocks(c) * 4 + 255) / 256 * 256;
+}
+inline long long ffn_scratch_bytes(const moe_cfg& c) {
+  return ffn_a_bytes(c) + kSchedBytes + ffn_ready_bytes(c);
+}
 // Z = [G, U] (bf16 [R_max, 2f]) or dZ, rounded up to 256 bytes
 inline long long ffn_z_bytes(const moe_cfg& c) {
   return (max_rows(c) * 2 * c.f * 2 + 255) / 256 * 256;

@@ -29,7 +29,9 @@ MODES = [N.MOE_FFN_FUSED_COMBINE, N.MOE_FFN_WRITE_O,
          N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_STRICT_SLOTS,
          N.MOE_FFN_WRITE_O | N.MOE_FFN_STRICT_SLOTS,
          N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_SM_PAIR,
-         N.MOE_FFN_WRITE_O | N.MOE_FFN_SM_PAIR | N.MOE_FFN_STRICT_SLOTS]
+         N.MOE_FFN_WRITE_O | N.MOE_FFN_SM_PAIR | N.MOE_FFN_STRICT_SLOTS,
+         N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_ONE_LAUNCH,
+         N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_TWO_LAUNCHES]
 
 
 _ORACLE = {}
@@ -60,6 +62,8 @@ def test_ffn_every_element(wl, gather_x):
     ref = _oracle_full(wl, w1, w2)
     layer = MoeLayer(wl, "cuda", write_o=True, gather_x=gather_x)
     for mode in MODES:
+        if gather_x and mode & (N.MOE_FFN_ONE_LAUNCH | N.MOE_FFN_TWO_LAUNCHES):
+            continue  # launch-count flags are for the Xp path
         layer.y.fill_(float("nan"))
         run_gpu(wl, w1, w2, mode=mode, layer=layer)
         assert layer.read_status() == 0, (mode, N.moe_status_string(layer.read_status()))
@@ -88,6 +92,34 @@ def test_intermediate_a_matches_swiglu():
         want[sel] = O.silu(Z[:, : wl.f]) * Z[:, wl.f:]
     # A is rounded to bf16 on the GPU: 2^-8 relative plus accumulation-order noise
     check_y(A, want, "A = SiLU(G) * U")
+
+
+@pytest.mark.parametrize("name", ["qwen3_a1.5", "dsv3_a1"])
+def test_one_launch_full_size_sampled_tokens(name):
+    """FC1 and FC2 in one launch at full size: sampled tokens against the oracle, and the
+    whole y against the two-launch FFN (same arithmetic, atomics may reorder last bits)."""
+    wl = WORKLOADS[name]
+    w1, w2 = synth.make_weights(wl, "cuda")
+    layer = run_gpu(wl, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_TWO_LAUNCHES)
+    y2 = layer.view("y").clone()
+    run_gpu(wl, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_ONE_LAUNCH, layer=layer)
+    assert layer.read_status() == 0
+    torch.testing.assert_close(layer.view("y"), y2, rtol=1e-5, atol=1e-5)
+    logits, x = host_inputs(wl)
+    ids_ref, gates_ref = O.route_topk(logits.numpy(), wl.k)
+    rng = np.random.default_rng(1)
+    sample = np.unique(np.concatenate([[0, wl.T - 1], rng.choice(wl.T, 24, replace=False)]))
+    y = f32(layer.view("y")[torch.from_numpy(sample).cuda()])
+    xs = x.float().numpy()
+    cache = {}
+
+    def expert(e):
+        if e not in cache:
+            cache[e] = (f32(w1[e]), f32(w2[e]))
+        return cache[e]
+
+    for i, t in enumerate(sample):
+        check_y(y[i], O.token_output(xs[t], ids_ref[t], gates_ref[t], expert), f"{name} {t}")
 
 
 @pytest.mark.parametrize("name,gather_x", [
