@@ -132,6 +132,12 @@ enum {
                                 launch when FC1 has at most 32 work items (128 x 128 tiles,
                                 padding aside) per SM, two launches otherwise */
   MOE_FFN_TWO_LAUNCHES = 64, /* flag: FC1 and FC2 as two launches (never one) */
+  MOE_FFN_TEST_WAIT_TIMEOUT = 128, /* test hook for failure detection, not for production:
+                                runs the one-launch FFN with FC2's readiness target one
+                                above what FC1's epilogues reach and every wait limited to
+                                10 ms, so FC2's producers give up: the call leaves
+                                MOE_STATUS_TIMEOUT in status (out is then undefined) and
+                                the context stays usable */
   MOE_FFN_GATHER_X = 8       /* flag: the `xp` argument is x itself (bf16 [T, d]); FC1
                                 gathers each tile's rows x[row_token[r]] straight into
                                 shared memory (TMA row gather), so the dispatched copy

@@ -99,7 +99,8 @@ int moe_expert_ffn(const moe_cfg* cfg, const uint16_t* xp, const uint16_t* w1,
   int rc = check_cfg(cfg);
   if (rc != MOE_OK) return rc;
   if (mode & ~kFfnModes) return MOE_ERR_INVALID_ARG;
-  if ((mode & MOE_FFN_ONE_LAUNCH) && (mode & kOneLaunchExcludes)) return MOE_ERR_INVALID_ARG;
+  if ((mode & (MOE_FFN_ONE_LAUNCH | MOE_FFN_TEST_WAIT_TIMEOUT)) && (mode & kOneLaunchExcludes))
+    return MOE_ERR_INVALID_ARG;
   if (cfg->d % 256 || cfg->f % 128) return MOE_ERR_UNSUPPORTED;
   rc = check_ptrs({xp, w1, w2, tiles, plan_info, row_token, row_gate, a_scratch, out, status});
   if (rc != MOE_OK) return rc;

@@ -72,6 +72,7 @@ constexpr int STG_STRIDE = 36;          // floats per staged row of the FC2 comb
 constexpr int STG_BYTES = 4 * 32 * STG_STRIDE * 4;
 constexpr int META_BYTES = 2048;        // barriers, ring, per-row tokens
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per wait
+constexpr unsigned long long kTestTimeoutNs = 10000000ull;  // MOE_FFN_TEST_WAIT_TIMEOUT
 
 template <int PHASE, bool PAIR>
 struct Geo {
@@ -926,7 +927,8 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   a2.out_ld = c.d;
   a2.write_o = write_o;
 
-  bool one_launch = (mode & MOE_FFN_ONE_LAUNCH) != 0;
+  const bool test_timeout = (mode & MOE_FFN_TEST_WAIT_TIMEOUT) != 0;
+  bool one_launch = (mode & (MOE_FFN_ONE_LAUNCH | MOE_FFN_TEST_WAIT_TIMEOUT)) != 0;
   if (!one_launch && !(mode & kOneLaunchExcludes)) {
     // small layers: FC1's tail and FC2's ramp-up are a visible share of the time, and one
     // launch overlaps them (measured about 4 % faster at up to ~20 items per SM, and
@@ -947,6 +949,10 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
     a3.out_ld2 = a2.out_ld;
     a3.ready = ready;
     a3.ready_target = 4 * a1.n_n;  // four epilogue warps per FC1 n-tile of the half
+    if (test_timeout) {            // a target nothing reaches, and short waits
+      a3.ready_target += 1;
+      a3.timeout_ns = kTestTimeoutNs;
+    }
     return launch_one<3, false>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a3, st);
   }
   if (gather)

@@ -17,7 +17,7 @@ constexpr long long kMaxN = 1LL << 22;
 // every flag moe_expert_ffn accepts
 constexpr int kFfnModes = MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR |
                           MOE_FFN_GATHER_X | MOE_FFN_SAVE_Z | MOE_FFN_ONE_LAUNCH |
-                          MOE_FFN_TWO_LAUNCHES;
+                          MOE_FFN_TWO_LAUNCHES | MOE_FFN_TEST_WAIT_TIMEOUT;
 // flags the one-launch FFN does not combine with
 constexpr int kOneLaunchExcludes = MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR |
                                    MOE_FFN_GATHER_X | MOE_FFN_TWO_LAUNCHES;
