@@ -119,6 +119,16 @@ def dist_setup(args):
     return world, rank, local
 
 
+def max_over_ranks(seconds: float, dev) -> float:
+    """The slowest rank's time (each rank passes its own); `dev` holds the reduction's
+    tensor (a GPU for NCCL, the CPU for gloo).  One rank: the value itself."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return seconds
+    t = torch.tensor([seconds], device=dev, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def workload_config(wl, extra=None):
     cfg = {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "f": wl.f,
            "beta": wl.beta, "P": wl.P, "s": wl.s, "alpha": wl.alpha, "hot_p": wl.hot_p,
@@ -215,11 +225,7 @@ def run_e2e(layer, logits_h, x_h, w1, w2, mode, wl, args, world, dev):
         pipe.submit(logits_p, x_p, y_p, w1, w2, mode)
     e1.record(pipe.s_out)
     pipe.drain()
-    t = e0.elapsed_time(e1) / 1e3
-    if world > 1:
-        tt = torch.tensor([t], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        t = float(tt.item())
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
     return {"value": round(wl.T * wl.k * steps * world / t, 1), "unit": "tokens/s",
             "h2d_bytes_per_step": logits_h.numel() * 4 + x_h.numel() * 2,
             "d2h_bytes_per_step": wl.T * wl.d * 4, "steps": steps,
@@ -373,11 +379,7 @@ def run_ours(args, wl, world, rank, local):
         for i in range(args.steps):
             step(recs[i])
         torch.cuda.synchronize(dev)
-    elapsed = start.elapsed_time(stop) / 1e3
-    if world > 1:
-        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(start.elapsed_time(stop) / 1e3, dev)
     stage_ms = {name: statistics.mean(r[i].elapsed_time(r[i + 1]) for r in recs)
                 for i, name in enumerate(["route", "plan", "dispatch", "ffn"])}
     status = layer.read_status()
@@ -509,7 +511,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--variant-mask", type=lambda v: int(v, 0), default=0,
                     help="planner variants (bits 0..3 bounded greedy, bit 4 quota solver; "
-                         "0 = all five) and, in bits 8..15, the quota floor u_min")
+                         "0 = the four greedy searches), bit 5 reduction-aware selection, "
+                         "bits 8..15 the quota floor u_min, bits 16..23 lambda")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch the step's kernels one by one instead of replaying the whole "
                          "layer as one CUDA graph (the default)")
