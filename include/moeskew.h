@@ -171,6 +171,13 @@ MOE_API int moe_route_hist(const moe_cfg* cfg, const float* logits, int32_t* top
                    float* topk_gates, int32_t* counts, int64_t* sumsq, double* kappa,
                    int32_t* status, moe_stream_t stream);
 
+/* Token blocks on their own ("Problem Formulation": b_e = ceil(c_e / beta)) and their
+ * exclusive prefix sum block_off int32 [E+1], from counts int32 [E] (moe_route_hist).
+ * moe_plan_blocks writes the same values; the dispatch needs nothing else from the plan,
+ * so with this call it can run on another stream while the planner searches. */
+MOE_API int moe_block_offsets(const moe_cfg* cfg, const int32_t* counts, int32_t* block_off,
+                              moe_stream_t stream);
+
 /* Token blocks and the block planner ("Problem Formulation", "Bounded Greedy Search").
  *   counts       int32 [E] (from moe_route_hist).
  *   variant_mask bits 0..3 enable greedy variants v = 2*D + F (D donor priority:

@@ -65,6 +65,15 @@ int moe_route_hist(const moe_cfg* cfg, const float* logits, int32_t* topk_ids,
                                        kappa, status, (cudaStream_t)stream));
 }
 
+int moe_block_offsets(const moe_cfg* cfg, const int32_t* counts, int32_t* block_off,
+                      moe_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  rc = check_ptrs({counts, block_off});
+  if (rc != MOE_OK) return rc;
+  return cuda_result(launch_block_offsets(*cfg, counts, block_off, (cudaStream_t)stream));
+}
+
 int moe_plan_blocks(const moe_cfg* cfg, const int32_t* counts, uint32_t variant_mask,
                     int32_t* block_off, int32_t* q, int32_t* slot_load, int32_t* slot_off,
                     int32_t* blocks, int32_t* tiles, int32_t* plan_info, int32_t* status,

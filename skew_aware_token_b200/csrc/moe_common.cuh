@@ -94,6 +94,8 @@ __device__ __forceinline__ void set_status(int32_t* status, int bits) {
 cudaError_t launch_route_hist(const moe_cfg& c, const float* logits, int32_t* ids,
                               float* gates, int32_t* counts, int64_t* sumsq, double* kappa,
                               int32_t* status, cudaStream_t st);
+cudaError_t launch_block_offsets(const moe_cfg& c, const int32_t* counts, int32_t* block_off,
+                                 cudaStream_t st);
 cudaError_t launch_plan(const moe_cfg& c, const int32_t* counts, uint32_t mask,
                         int32_t* block_off, int32_t* q, int32_t* slot_load,
                         int32_t* slot_off, int32_t* blocks, int32_t* tiles,

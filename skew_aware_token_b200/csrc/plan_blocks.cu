@@ -337,6 +337,24 @@ __device__ void quota_variant(int E, int P, int s, int u_min, int B, const int* 
   __syncwarp();
 }
 
+// b_e = ceil(c_e / beta) and the exclusive scan block_off on one warp (lane l owns a
+// contiguous chunk of experts), as the planner's first step computes them.
+__global__ void __launch_bounds__(32, 1)
+block_offsets_kernel(const int32_t* __restrict__ counts, int E, int beta,
+                     int32_t* __restrict__ block_off) {
+  const int lane = threadIdx.x;
+  const int C = (E + 31) / 32;
+  const int e0 = min(lane * C, E), e1 = min(e0 + C, E);
+  int local = 0;
+  for (int e = e0; e < e1; ++e) local += (max(counts[e], 0) + beta - 1) / beta;
+  int run = warp_excl_scan(local, lane);
+  for (int e = e0; e < e1; ++e) {
+    block_off[e] = run;
+    run += (max(counts[e], 0) + beta - 1) / beta;
+  }
+  if (lane == 31) block_off[E] = run;
+}
+
 __global__ void __launch_bounds__(kPlanThreads, 1)
 plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
             unsigned mask, int u_min, int lam, int b_max, int32_t* __restrict__ block_off, int32_t* __restrict__ q_out,
@@ -543,6 +561,12 @@ plan_kernel(const int32_t* __restrict__ counts, int E, int P, int s, int beta,
 }
 
 }  // namespace
+
+cudaError_t launch_block_offsets(const moe_cfg& c, const int32_t* counts, int32_t* block_off,
+                                 cudaStream_t st) {
+  block_offsets_kernel<<<1, 32, 0, st>>>(counts, c.E, c.beta, block_off);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_plan(const moe_cfg& c, const int32_t* counts, uint32_t mask,
                         int32_t* block_off, int32_t* q, int32_t* slot_load,

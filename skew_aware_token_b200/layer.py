@@ -42,7 +42,8 @@ class MoeLayer:
         self.sumsq = z(2, dt=torch.int64)
         self.kappa = z(2, dt=torch.float64)
         self.status = z(4)
-        self.block_off = z(E + 4)
+        self.block_off = z(E + 4)       # written by moe_block_offsets, read by the dispatch
+        self.block_off_plan = z(E + 4)  # the planner's own copy (same values)
         self.q = z(max(E * P, 4))
         self.slot_load = z(8)
         self.slot_off = z(12)
@@ -68,14 +69,23 @@ class MoeLayer:
         self.y = z(max(T * d, 4), dt=f32)
         self.o = z(max(R * d, 8), dt=torch.bfloat16) if write_o else None
         self.device = dev
+        self._side = torch.cuda.Stream(dev) if dev.type == "cuda" else None
 
     # ------------------------------------------------------------------ stages
     def route(self, logits, stream=None):
         N.moe_route_hist(self.cfg, logits, self.topk_ids, self.topk_gates, self.counts,
                          self.sumsq, self.kappa, self.status, stream)
 
+    def block_offsets(self, stream=None):
+        N.moe_block_offsets(self.cfg, self.counts, self.block_off, stream)
+
     def plan(self, variant_mask=0, stream=None):
-        N.moe_plan_blocks(self.cfg, self.counts, variant_mask, self.block_off, self.q,
+        """Block offsets (what the dispatch needs), then the plan."""
+        self.block_offsets(stream)
+        self._search(variant_mask, stream)
+
+    def _search(self, variant_mask, stream):
+        N.moe_plan_blocks(self.cfg, self.counts, variant_mask, self.block_off_plan, self.q,
                           self.slot_load, self.slot_off, self.blocks, self.tiles,
                           self.plan_info, self.status, stream)
 
@@ -110,10 +120,22 @@ class MoeLayer:
     def __call__(self, logits, x, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, variant_mask=0,
                  stream=None, y=None):
         """Route, plan, dispatch, FFN (+ combine): returns y fp32 [T, d], by default a view
-        of the layer's buffer (valid until the next call), or the caller's `y`."""
+        of the layer's buffer (valid until the next call), or the caller's `y`.  The
+        planner's search runs on a side stream while the dispatch runs (the dispatch needs
+        only the block offsets); both join before the FFN."""
         self.route(logits, stream)
-        self.plan(variant_mask, stream)
-        self.dispatch(x, stream)
+        self.block_offsets(stream)
+        main = stream if isinstance(stream, torch.cuda.Stream) else \
+            torch.cuda.current_stream(self.device) if stream is None else None
+        if main is not None:
+            self._side.wait_stream(main)
+            with torch.cuda.stream(self._side):
+                self._search(variant_mask, None)
+            self.dispatch(x, main)
+            main.wait_stream(self._side)
+        else:  # a raw stream handle: one stream
+            self._search(variant_mask, stream)
+            self.dispatch(x, stream)
         self.ffn(w1, w2, mode, stream, y, x)
         if mode & N.MOE_FFN_WRITE_O:
             self.combine(stream, y)

@@ -72,6 +72,7 @@ _VP = ctypes.c_void_p
 _SIGNATURES = {
     "moe_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(MoeCfg), ctypes.c_int]),
     "moe_route_hist": (ctypes.c_int, [ctypes.POINTER(MoeCfg)] + [_VP] * 8),
+    "moe_block_offsets": (ctypes.c_int, [ctypes.POINTER(MoeCfg)] + [_VP] * 3),
     "moe_plan_blocks": (ctypes.c_int, [ctypes.POINTER(MoeCfg), _VP, ctypes.c_uint32] + [_VP] * 9),
     "moe_dispatch_permute": (ctypes.c_int, [ctypes.POINTER(MoeCfg)] + [_VP] * 10),
     "moe_expert_ffn": (ctypes.c_int, [ctypes.POINTER(MoeCfg)] + [_VP] * 7 + [ctypes.c_int] +
@@ -151,6 +152,12 @@ def moe_route_hist(cfg, logits, topk_ids, topk_gates, counts, sumsq, kappa, stat
         ctypes.byref(c), _dev(logits, "logits"), _dev(topk_ids, "topk_ids"),
         _dev(topk_gates, "topk_gates"), _dev(counts, "counts"), _dev(sumsq, "sumsq"),
         _dev(kappa, "kappa"), _dev(status, "status"), _stream(stream)))
+
+
+def moe_block_offsets(cfg, counts, block_off, stream=None) -> None:
+    c = _cfg(cfg)
+    _check("moe_block_offsets", lib().moe_block_offsets(
+        ctypes.byref(c), _dev(counts, "counts"), _dev(block_off, "block_off"), _stream(stream)))
 
 
 def moe_plan_blocks(cfg, counts, variant_mask, block_off, q, slot_load, slot_off, blocks,

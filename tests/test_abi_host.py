@@ -25,7 +25,8 @@ def test_exports_every_declared_symbol():
     assert set(declared) == {"moe_workspace_size", "moe_route_hist", "moe_plan_blocks",
                              "moe_dispatch_permute", "moe_expert_ffn", "moe_combine",
                              "moe_status_string", "moe_expert_ffn_noalloc",
-                             "moe_dispatch_grad", "moe_expert_ffn_backward"}
+                             "moe_dispatch_grad", "moe_expert_ffn_backward",
+                             "moe_block_offsets"}
     out = subprocess.run(["nm", "-D", "--defined-only", N.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}

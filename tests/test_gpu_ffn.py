@@ -156,6 +156,26 @@ def test_full_size_sampled_tokens(name, gather_x):
     assert torch.isfinite(layer.view("y")).all()
 
 
+def test_concurrent_planner_matches_sequential_stages():
+    """The layer call runs the planner's search on a side stream beside the dispatch; the
+    result must be the stage-by-stage one (the same plan, tiles, rows and y)."""
+    wl = FULL_CASES[2]
+    w1, w2 = synth.make_weights(wl, "cuda")
+    logits, x = host_inputs(wl)
+    a = MoeLayer(wl, "cuda")
+    a(logits.cuda(), x.cuda(), w1, w2)
+    b = MoeLayer(wl, "cuda")
+    b.route(logits.cuda())
+    b.plan(0)
+    b.dispatch(x.cuda())
+    b.ffn(w1, w2)
+    torch.cuda.synchronize()
+    assert a.read_status() == 0 and b.read_status() == 0
+    for name in ("block_off", "q", "tiles", "row_token", "tok_row"):
+        assert torch.equal(a.view(name), b.view(name)), name
+    torch.testing.assert_close(a.view("y"), b.view("y"), rtol=1e-5, atol=1e-6)
+
+
 def test_repeated_calls_reuse_buffers():
     wl = FULL_CASES[1]
     w1, w2 = synth.make_weights(wl, "cuda")

@@ -61,6 +61,7 @@ def test_route_hist_and_plan_and_dispatch(case):
     b = O.block_counts(counts_ref, wl.beta)
     boff = O.block_offsets(b)
     assert layer.view("block_off").cpu().tolist() == boff
+    assert layer.block_off_plan[:wl.E + 1].cpu().tolist() == boff  # the planner's copy
     ref = O.plan(b, wl.P, wl.s, variant_mask=ALL5)  # all five variants, best kept
     q = layer.view("q").cpu().numpy()
     assert np.array_equal(q, ref["q"])
