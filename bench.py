@@ -33,7 +33,7 @@ from skew_aware_token_b200 import synth  # noqa: E402
 METRIC = "MoE-layer fwd routed tokens/s and TFLOP/s on 1 B200; % of roofline vs kappa"
 DEFAULT_WORKLOAD = "olmoe_a1"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 7  # route, kappa, plan, rank, gather, fc1, fc2 (+ combine)
+LAUNCHES_PER_STEP = 8  # route, kappa, block offsets, plan, rank, gather, fc1, fc2 (+ combine)
 
 
 def load_peaks():
@@ -257,16 +257,15 @@ def measured_traffic(workload: str):
     return rec["bytes_per_step"]
 
 
-def ffn_one_launch(wl, mode, dev) -> bool:
-    """Whether moe_expert_ffn runs FC1 and FC2 as one launch for this mode (its rule: forced
-    by MOE_FFN_ONE_LAUNCH, else for a fused single-SM Xp call with at most 32 FC1 work items
-    per SM)."""
+def ffn_one_launch(wl, mode, sms: int) -> bool:
+    """Whether moe_expert_ffn runs FC1 and FC2 as one launch for this mode on a GPU with
+    `sms` SMs (its rule: forced by MOE_FFN_ONE_LAUNCH, else for a fused single-SM Xp call
+    with at most 32 FC1 work items per SM)."""
     if mode & N.MOE_FFN_ONE_LAUNCH:
         return True
     if mode & (N.MOE_FFN_WRITE_O | N.MOE_FFN_STRICT_SLOTS | N.MOE_FFN_SM_PAIR |
                N.MOE_FFN_GATHER_X | N.MOE_FFN_TWO_LAUNCHES):
         return False
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     return wl.T * wl.k // 128 * (wl.f // 128) <= 32 * sms
 
 
@@ -311,6 +310,7 @@ def run_backward(layer, w1, w2, wl, args, dev, peak, peak_src):
 def run_ours(args, wl, world, rank, local):
     from skew_aware_token_b200.layer import MoeLayer
     dev = torch.device("cuda", local)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     peaks, peak_src = load_peaks()
     logits_h = synth.make_logits(wl)
     x_h = synth.make_x(wl)
@@ -446,7 +446,8 @@ def run_ours(args, wl, world, rank, local):
         "e2e": e2e,
         "backward": backward,
         "gpu_launches": (LAUNCHES_PER_STEP + int(write_o) - int(args.gather_x) -
-                         int(ffn_one_launch(wl, mode, dev))) * args.steps,
+                         int(ffn_one_launch(wl, mode | (N.MOE_FFN_GATHER_X if args.gather_x
+                                                        else 0), sms))) * args.steps,
         "clocks": clocks.summary(),
         "impl": "ours",
     }

@@ -1,0 +1,58 @@
+"""Host-side helpers of bench.py, on CPU: the FC1/FC2 launch rule it mirrors from
+moe_expert_ffn (one launch when FC1 has at most 32 work items per SM), the committed DRAM
+traffic record and its source digest, and the peak figures."""
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from skew_aware_token_b200 import native as N  # noqa: E402
+from skew_aware_token_b200.synth import WORKLOADS, Workload  # noqa: E402
+
+
+@pytest.mark.parametrize("name,one", [("olmoe_a1", True), ("qwen3_a1.5", True),
+                                      ("sweep_all4_p0_b128", False), ("dsv3_a1", False)])
+def test_one_launch_rule_at_148_sms(name, one):
+    # FC1 items = (T k / 128) (f / 128): OLMoE 2048, Qwen3 3072, sweep 6144, DeepSeek-V3
+    # 16384; the threshold is 32 x 148 = 4736
+    assert bench.ffn_one_launch(WORKLOADS[name], 0, 148) is one
+
+
+def test_one_launch_rule_boundary_and_flags():
+    wl = Workload("edge", T=4736 * 128 // 8, d=256, E=8, k=8, f=128, beta=128, P=1, s=0)
+    assert wl.T * wl.k // 128 * (wl.f // 128) == 32 * 148
+    assert bench.ffn_one_launch(wl, 0, 148)            # at the threshold: one launch
+    assert not bench.ffn_one_launch(wl, 0, 147)        # one item per SM over it: two
+    for flag in (N.MOE_FFN_WRITE_O, N.MOE_FFN_STRICT_SLOTS, N.MOE_FFN_SM_PAIR,
+                 N.MOE_FFN_GATHER_X, N.MOE_FFN_TWO_LAUNCHES):
+        assert not bench.ffn_one_launch(wl, flag, 148), flag
+    assert bench.ffn_one_launch(WORKLOADS["dsv3_a1"], N.MOE_FFN_ONE_LAUNCH, 148)
+
+
+def test_traffic_record_follows_the_ffn_source():
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    for name, r in rec.items():
+        if r["ffn_source_sha1"] == bench.ffn_source_digest():
+            assert bench.measured_traffic(name) == r["bytes_per_step"]
+        else:
+            assert bench.measured_traffic(name) is None
+    assert bench.measured_traffic("no_such_workload") is None
+
+
+def test_traffic_record_is_dropped_when_the_source_changes(monkeypatch):
+    monkeypatch.setattr(bench, "ffn_source_digest", lambda: "0" * 40)
+    assert all(bench.measured_traffic(n) is None for n in WORKLOADS)
+
+
+def test_peaks_come_from_the_measured_file_when_present():
+    peaks, src = bench.load_peaks()
+    if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")):
+        assert src == "of measured"
+        assert peaks["bf16_tflops_sustained"] <= peaks["bf16_tflops"]
+    else:
+        assert src == "of fallback" and peaks == bench.FALLBACK_PEAKS
