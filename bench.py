@@ -243,10 +243,12 @@ def ffn_source_digest() -> str:
     return h.hexdigest()
 
 
-def measured_traffic(workload: str):
-    """DRAM bytes (read + write) of one expert-FFN step (both launches) from the committed
-    ncu capture, or None when there is none for this workload or the FFN source changed
-    since it was taken."""
+def measured_traffic(workload: str, default_ffn: bool = True):
+    """DRAM bytes (read + write) of one expert-FFN step from the committed ncu capture, or
+    None when there is none for this workload, the FFN source changed since it was taken, or
+    the run does not use the library's default FFN configuration (the one captured)."""
+    if not default_ffn:
+        return None
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -403,7 +405,8 @@ def run_ours(args, wl, world, rank, local):
                 "traffic": None, "flops_per_launch": wl.flops,
                 "ms_per_launch": round(stage_ms["ffn"], 4),
                 "frac_of_burst": round(ffn_tflops / burst, 4)}
-    roofline["traffic"] = measured_traffic(wl.name)
+    roofline["traffic"] = measured_traffic(
+        wl.name, default_ffn=mode == 0 and not args.gather_x and args.launches == "auto")
 
     backward = run_backward(layer, w1, w2, wl, args, dev, peak, peak_src) if args.backward \
         else None

@@ -56,3 +56,8 @@ def test_peaks_come_from_the_measured_file_when_present():
         assert peaks["bf16_tflops_sustained"] <= peaks["bf16_tflops"]
     else:
         assert src == "of fallback" and peaks == bench.FALLBACK_PEAKS
+
+
+def test_traffic_record_only_for_the_captured_configuration():
+    for name in WORKLOADS:
+        assert bench.measured_traffic(name, default_ffn=False) is None
