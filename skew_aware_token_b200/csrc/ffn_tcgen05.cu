@@ -4,9 +4,9 @@
 //   Z_e = X_e W1_e,  Z_e = [G_e, U_e],  A_e = SiLU(G_e) * U_e,  O_e = A_e W2_e,
 //   y_t = sum_{e in S_t} p_{t,e} O_e[t].
 // The pages' forward megakernel runs FC1, then FC2 on each token block ("Executor:
-// Pipelined Expert Replication", Forward); here the blocks are grouped into the planner's
-// execution tiles (up to 256 rows of one expert) and the two GEMMs are two persistent
-// launches over the same tile list.
+// Pipelined Expert Replication", Forward); here the blocks form the planner's tiles (up to
+// 256 rows of one expert), and the GEMMs run as two persistent launches over the tile list,
+// or as one (FC2 on a tile half starts once FC1 wrote its rows) for small layers.
 //
 // Two variants of one kernel template:
 //   single SM (default): one CTA runs one 128-row half of a tile with
