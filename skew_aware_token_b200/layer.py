@@ -1,5 +1,7 @@
 """The forward MoE layer as one call: owns the device buffers of one configuration and
-strings the five C-ABI calls together on the current CUDA stream.
+strings the C-ABI calls together (route + histogram, block offsets, plan, dispatch, expert
+FFN, and the combine when the FFN writes O) on the current CUDA stream, the planner's search
+on a second stream beside the dispatch.
 
     layer = MoeLayer(workload, device="cuda")
     y = layer(logits, x, w1, w2)          # device tensors in, y fp32 [T, d] out
