@@ -8,7 +8,7 @@
 // (section 4, Algorithm 1); that solver is also a one-SM kernel with its load matrix in
 // shared memory.  Plans are deterministic (TopoEP: bitwise-identical plans).
 //
-// The greedy rule (shared word for word with the CPU statement of the method):
+// The greedy rule (the same rule the CPU oracle states; no code is shared):
 //   start  q[e][h(e)] = b_e, h(e) = floor(e P / E); loads l_r; replicas rep_r = 0.
 //   round  while max_r l_r > tau: donors = {r : l_r > tau} ordered by (key desc, r asc)
 //          with key = l_r (variant D = 0) or max_{h(e)=r} q[e][r] (D = 1), taken at the
