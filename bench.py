@@ -262,13 +262,13 @@ def measured_traffic(workload: str, default_ffn: bool = True):
 def ffn_one_launch(wl, mode, sms: int) -> bool:
     """Whether moe_expert_ffn runs FC1 and FC2 as one launch for this mode on a GPU with
     `sms` SMs (its rule: forced by MOE_FFN_ONE_LAUNCH, else for a fused single-SM Xp call
-    with at most 32 FC1 work items per SM)."""
+    with at most 2 FC1 work items per SM)."""
     if mode & N.MOE_FFN_ONE_LAUNCH:
         return True
     if mode & (N.MOE_FFN_WRITE_O | N.MOE_FFN_STRICT_SLOTS | N.MOE_FFN_SM_PAIR |
                N.MOE_FFN_GATHER_X | N.MOE_FFN_TWO_LAUNCHES):
         return False
-    return wl.T * wl.k // 128 * (wl.f // 128) <= 32 * sms
+    return wl.T * wl.k // 128 * (wl.f // 128) <= 2 * sms
 
 
 def run_backward(layer, w1, w2, wl, args, dev, peak, peak_src):

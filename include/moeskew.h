@@ -114,7 +114,8 @@ enum {
   MOE_FFN_STRICT_SLOTS = 2,  /* flag: execution unit u (an SM pair, or an SM) only runs
                                 slot (u mod P)'s tiles, so the layer time follows the
                                 plan's makespan (one GPU standing in for P); without it
-                                every unit takes tiles of any slot */
+                                every unit takes tiles of any slot.  The call returns
+                                MOE_ERR_UNSUPPORTED when the GPU has fewer than P units */
   MOE_FFN_SM_PAIR = 4,       /* flag: run each tile on a pair of SMs (a cluster of two
                                 CTAs, tcgen05 cta_group::2, M = 256) instead of each
                                 128-row half on one SM (cta_group::1, the default) */
@@ -129,7 +130,7 @@ enum {
                                 WRITE_O, STRICT_SLOTS, SM_PAIR or GATHER_X the call returns
                                 MOE_ERR_INVALID_ARG.  Without this flag or
                                 MOE_FFN_TWO_LAUNCHES, a fused single-SM Xp call takes one
-                                launch when FC1 has at most 32 work items (128 x 128 tiles,
+                                launch when FC1 has at most 2 work items (128 x 128 tiles,
                                 padding aside) per SM, two launches otherwise */
   MOE_FFN_TWO_LAUNCHES = 64, /* flag: FC1 and FC2 as two launches (never one) */
   MOE_FFN_TEST_WAIT_TIMEOUT = 128, /* test hook for failure detection, not for production:
@@ -138,6 +139,11 @@ enum {
                                 10 ms, so FC2's producers give up: the call leaves
                                 MOE_STATUS_TIMEOUT in status (out is then undefined) and
                                 the context stays usable */
+  MOE_FFN_FC1_M128 = 256,    /* flag: run FC1 on 128-row halves of the tiles (the tile-half
+                                kernel, M = 128 per SM) instead of on whole tiles of up to
+                                256 rows (two M = 128 MMAs sharing each weight stage, the
+                                two-launch default).  The one-launch FFN, SM pairs, rows
+                                gathered from x and MOE_FFN_SAVE_Z always use tile halves */
   MOE_FFN_GATHER_X = 8       /* flag: the `xp` argument is x itself (bf16 [T, d]); FC1
                                 gathers each tile's rows x[row_token[r]] straight into
                                 shared memory (TMA row gather), so the dispatched copy

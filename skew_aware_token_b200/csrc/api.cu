@@ -113,6 +113,7 @@ int moe_expert_ffn(const moe_cfg* cfg, const uint16_t* xp, const uint16_t* w1,
   if (cfg->d % 256 || cfg->f % 128) return MOE_ERR_UNSUPPORTED;
   rc = check_ptrs({xp, w1, w2, tiles, plan_info, row_token, row_gate, a_scratch, out, status});
   if (rc != MOE_OK) return rc;
+  if ((mode & MOE_FFN_STRICT_SLOTS) && ffn_units(mode) < cfg->P) return MOE_ERR_UNSUPPORTED;
   return cuda_result(launch_ffn(*cfg, xp, w1, w2, tiles, plan_info, row_token, row_gate, mode,
                                 a_scratch, out, status, (cudaStream_t)stream));
 }

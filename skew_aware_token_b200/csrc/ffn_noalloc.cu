@@ -68,6 +68,7 @@ extern "C" MOE_API int moe_expert_ffn_noalloc(const moe_cfg* cfg, const uint16_t
   if ((mode & (MOE_FFN_ONE_LAUNCH | MOE_FFN_TEST_WAIT_TIMEOUT)) && (mode & kOneLaunchExcludes))
     return MOE_ERR_INVALID_ARG;
   if (c.d % 256 || c.f % 128) return MOE_ERR_UNSUPPORTED;
+  if ((mode & MOE_FFN_STRICT_SLOTS) && ffn_units(mode) < c.P) return MOE_ERR_UNSUPPORTED;
   for (const void* p : {(const void*)xp, (const void*)w1, (const void*)w2, (const void*)tiles,
                         (const void*)plan_info, (const void*)row_token, (const void*)row_gate,
                         (const void*)out, (const void*)status}) {

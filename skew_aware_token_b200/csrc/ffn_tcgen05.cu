@@ -850,10 +850,11 @@ cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUten
   } else {
     cfg.gridDim = dim3(num_sms());
   }
-  FfnArgs a = args;
+  // strict slots need one unit per slot at least (checked by the caller before anything is
+  // enqueued; a unit u >= units would never exist to run slot u's tiles)
   const int units = PAIR ? (int)cfg.gridDim.x / 2 : (int)cfg.gridDim.x;
-  a.strict = a.strict && units >= a.P;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, ta64, ta2, tb2, a);
+  if (args.strict && units < args.P) return cudaErrorInvalidConfiguration;
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, ta64, ta2, tb2, args);
 }
 
 }  // namespace
@@ -930,11 +931,11 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   const bool test_timeout = (mode & MOE_FFN_TEST_WAIT_TIMEOUT) != 0;
   bool one_launch = (mode & (MOE_FFN_ONE_LAUNCH | MOE_FFN_TEST_WAIT_TIMEOUT)) != 0;
   if (!one_launch && !(mode & kOneLaunchExcludes)) {
-    // small layers: FC1's tail and FC2's ramp-up are a visible share of the time, and one
-    // launch overlaps them (measured about 4 % faster at up to ~20 items per SM, and
-    // slower from ~40 on)
+    // tiny layers: one launch saves a launch and overlaps FC1's tail with FC2's start.  From
+    // a few items per SM on, two launches with FC1 on whole 256-row tiles are faster (about
+    // 10 % on the 4096-token layer with 14 FC1 half-tile items per SM)
     const long long fc1_items = (long long)c.T * c.k / BM * (c.f / (BN / 2));
-    one_launch = fc1_items <= 32LL * num_sms();
+    one_launch = fc1_items <= 2LL * num_sms();
   }
   if (one_launch) {
     // FC1 items, then FC2 items, in one persistent launch; FC2 waits per tile half
@@ -955,7 +956,10 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
     }
     return launch_one<3, false>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a3, st);
   }
-  if (gather)
+  if (fc1_wide_supported(mode))
+    err = launch_fc1_wide(c, xp, w1, tiles, plan_info, a_scratch, sched, status, a1.strict != 0,
+                          st);
+  else if (gather)
     err = pair ? launch_one<1, true, true>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a1, st)
                : launch_one<1, false, true>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a1, st);
   else
@@ -964,6 +968,32 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   if (err != cudaSuccess) return err;
   return pair ? launch_one<2, true>(tm_a, tm_w2, tm_a64, tm_a, tm_w2, a2, st)
               : launch_one<2, false>(tm_a, tm_w2, tm_a64, tm_a, tm_w2, a2, st);
+}
+
+int ffn_units(int mode) {
+  if (!(mode & MOE_FFN_SM_PAIR)) return num_sms();
+  // clusters of two CTAs that fit at once (the pair launches' grid)
+  auto kern = ffn_kernel<2, true, false>;
+  static OncePerDevice occ_once;
+  int clusters = 0;
+  cudaError_t err = once_per_device(occ_once, [&](int& n) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Geo<2, true>::SMEM);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = Geo<2, true>::SMEM;
+    return cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+  }, &clusters);
+  return err == cudaSuccess ? clusters : 0;
 }
 
 }  // namespace moe

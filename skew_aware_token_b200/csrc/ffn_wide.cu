@@ -1,0 +1,489 @@
+// FC1 + SwiGLU of the grouped expert FFN on whole 256-row tiles (tcgen05 + TMEM, TMA in
+// and out), the default FC1 of the two-launch FFN.
+//
+// "MegaFlux" summary, Methodology 2, expert-computation equation: Z_e = X_e W1_e,
+// Z_e = [G_e, U_e], A_e = SiLU(G_e) * U_e.  A work item is one planner tile (up to 256 rows
+// of one expert) times one n-tile of 128 output columns of A.
+//
+// Why a 256-row tile on one SM: a K step of 64 then moves A (256 rows, 32 KB) and B (the
+// n-tile's 128 G rows over its 128 U rows, 32 KB) for 2 x 128x256x64 MMAs, i.e. 64 bytes
+// per tensor-core clock of the SM, where a 128-row tile moves 48 KB per 128x256x64 MMA
+// (96 B/clk).  On B200 an SM takes in about 69 B/clk from L2 (copies from L2 plus, for a
+// cta_group::2 pair, the partner's B half), so the 128-row tile is capped near 0.73 of the
+// tensor rate and the 256-row tile is not (0.98 measured with operands in L2).  The price:
+// the two 128x256 fp32 accumulators fill all 512 TMEM columns, so the epilogue of an item
+// does not overlap the next item's MMAs.  The epilogue is kept short:
+//   - SiLU(g) = g/2 + (g/2) tanh(g/2) with the tanh.approx instruction (one MUFU op);
+//   - the warps that read TMEM never touch global memory (a thread's global stores held up
+//     its later tcgen05.ld waits): they write A, rounded to bf16, into a shared-memory
+//     staging buffer laid out as 32-row x 64-column boxes with the 128-byte swizzle, and a
+//     store warp writes the boxes to A with TMA (cp.async.bulk.tensor, shared -> global).
+//
+// Roles (352 threads, one CTA per SM, persistent):
+//   warp 0      TMA producer: draws items from the global (or, strict slots, the slot's)
+//               counter, passes them through a ring in shared memory, loads A rows
+//               [row0, row0 + 256) of Xp (the second 128-row box only when the tile has
+//               more than 128 rows) and the n-tile's G and U rows of W1_e per K step into a
+//               3-stage ring (128-byte swizzle).
+//   warp 1      MMA issuer: per K step tcgen05.mma.cta_group::1.kind::f16 M=128 N=256 for
+//               rows 0..127 into TMEM columns [0, 256), and for rows 128..255 into
+//               [256, 512); commit frees the stage; after the last K step the accumulators
+//               go to the epilogue.
+//   warps 2..9  epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (32 rows of each half)
+//               and 64 of the n-tile's 128 output columns ((w - 2) / 4 picks which),
+//               A = SiLU(G) * U -> bf16 -> staging (one half at a time).
+//   warp 10     store warp: TMA stores of the staged boxes whose rows are in the tile (tile
+//               sizes are multiples of 64 rows), then frees the staging buffer once the
+//               copies have read it.
+// Every wait is bounded (globaltimer); on expiry the kernel sets MOE_STATUS_TIMEOUT, the
+// other roles drop out, copies and MMAs in flight are waited for, TMEM is freed.
+#include "tc_util.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int WM = 256;                 // rows per item
+constexpr int HM = 128;                 // rows per MMA (TMEM lanes)
+constexpr int WK = 64;                  // K per stage: one 128-byte swizzle span of bf16
+constexpr int WN = 256;                 // MMA N: 128 G + 128 U columns
+constexpr int W_ST = 3;                 // stages
+constexpr int W_A_BYTES = WM * WK * 2;  // 32 KB
+constexpr int W_B_BYTES = WN * WK * 2;  // 32 KB
+constexpr int W_STAGE = W_A_BYTES + W_B_BYTES;
+constexpr int W_HALF_A = HM * WK * 2;   // one 128-row A box
+constexpr int W_STG_BYTES = HM * 128 * 2;  // one half of the item's A: 128 rows x 128 cols
+constexpr int W_RING = 8;
+constexpr int W_EPI_WARPS = 8;          // two per TMEM lane quadrant
+constexpr int W_THREADS = 32 * (3 + W_EPI_WARPS);
+// full[ST], empty[ST], drain, tfull, tempty, staged, stgfree, ifull[RING], iempty[RING]
+constexpr int W_NBARS = 2 * W_ST + 5 + 2 * W_RING;
+constexpr int W_META = 512;
+constexpr int W_SMEM = W_ST * W_STAGE + W_STG_BYTES + W_META + 1024;
+static_assert(W_SMEM <= 227 * 1024, "shared memory");
+static_assert(W_NBARS * 8 + 4 * (2 + W_RING) <= W_META, "meta");
+// kind::f16: D fp32, A and B bf16, both K-major, N = 256, M = 128
+constexpr uint32_t W_IDESC =
+    (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(WN >> 3) << 17) | ((uint32_t)(HM >> 4) << 24);
+
+struct WideArgs {
+  int32_t* sched;  // item counters: [0], or [slot] with strict slots; zeroed by the host
+  const int32_t* tiles;
+  const int32_t* plan_info;
+  int32_t* status;
+  long long r_max;
+  int E, P, f, n_k, n_n;
+  int strict;
+  unsigned long long timeout_ns;
+};
+
+struct WideSched {
+  int32_t* counter;
+  long long total;
+  int m_base, n_n;
+};
+
+__device__ WideSched wide_sched(const WideArgs& a) {
+  WideSched s;
+  s.n_n = a.n_n;
+  const int* pi = a.plan_info;
+  if (!a.strict) {
+    s.counter = a.sched;
+    s.total = (long long)max(pi[MOE_PI_NTILES], 0) * a.n_n;
+    s.m_base = 0;
+  } else {
+    const int r = (int)blockIdx.x % a.P;
+    const int lo = pi[MOE_PI_SLOT_TILE_OFF + r], hi = pi[MOE_PI_SLOT_TILE_OFF + r + 1];
+    s.counter = a.sched + r;
+    s.total = (long long)max(hi - lo, 0) * a.n_n;
+    s.m_base = lo;
+  }
+  return s;
+}
+
+struct WideTile {
+  int e, row0, nrows, n;
+  bool ok;
+};
+__device__ __forceinline__ WideTile wide_tile(const WideArgs& a, const WideSched& s, int L) {
+  WideTile t;
+  t.n = L % s.n_n;
+  const int m = s.m_base + L / s.n_n;
+  const int4 v = __ldg(reinterpret_cast<const int4*>(a.tiles) + m);
+  t.e = v.x;
+  t.row0 = v.y;
+  t.nrows = v.z;
+  // tiles hold whole 64-row blocks; a 32-row store box is then all in the tile or all out
+  t.ok = v.x >= 0 && v.x < a.E && v.y >= 0 && (long long)v.y < a.r_max && v.z > 0 &&
+         v.z <= WM && (v.z & 31) == 0;
+  return t;
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   map),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// The bounded mbarrier wait of tc_util.cuh, inlined: the epilogue keeps its packed A values
+// in registers across the wait for the staging buffer, and a call would save them to the
+// stack (local-memory stores that hold up the thread's next tcgen05.ld wait).
+__device__ __forceinline__ bool wait_inl(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         int32_t* status, unsigned long long timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t spin = 1;; ++spin) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((spin & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > timeout_ns) {
+        *abort_flag = 1;
+        set_status(status, MOE_STATUS_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// SiLU(g) = g * sigmoid(g) = g/2 + (g/2) tanh(g/2)
+__device__ __forceinline__ float silu_tanh(float g) {
+  const float h = 0.5f * g;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+  return fmaf(h, t, h);
+}
+
+__global__ void __launch_bounds__(W_THREADS, 1)
+fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                const __grid_constant__ CUtensorMap tmA, const WideArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stg = smem + W_ST * W_STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + W_STG_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + W_NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + W_ST + s); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * W_ST);
+  const uint32_t tfull_bar = smem_u32(bars + 2 * W_ST + 1);
+  const uint32_t tempty_bar = smem_u32(bars + 2 * W_ST + 2);
+  const uint32_t staged_bar = smem_u32(bars + 2 * W_ST + 3);
+  const uint32_t stgfree_bar = smem_u32(bars + 2 * W_ST + 4);
+  auto ifull_bar = [&](int i) { return smem_u32(bars + 2 * W_ST + 5 + i); };
+  auto iempty_bar = [&](int i) { return smem_u32(bars + 2 * W_ST + 5 + W_RING + i); };
+  auto sA = [&](int s) { return smem_u32(smem + s * W_STAGE); };
+  auto sB = [&](int s) { return smem_u32(smem + s * W_STAGE + W_A_BYTES); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < W_ST; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(drain_bar, 1);
+    mbar_init(tfull_bar, 1);
+    mbar_init(tempty_bar, W_EPI_WARPS);
+    mbar_init(staged_bar, W_EPI_WARPS);
+    mbar_init(stgfree_bar, 1);  // the store thread
+    for (int i = 0; i < W_RING; ++i) {
+      mbar_init(ifull_bar(i), 1);
+      mbar_init(iempty_bar(i), 2 + W_EPI_WARPS);  // MMA thread, epilogue warps, store thread
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmA);
+  }
+  if (warp == 1) tmem_alloc<false, 512>(smem_u32(tmem_slot));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WideSched sch = wide_sched(a);
+
+  // consumers: the item of ring position `it`, or -1 when the work is done or a wait gave up
+  auto take_item = [&](int it, bool honour) -> int {
+    const int slot = it % W_RING;
+    if (!mbar_wait(ifull_bar(slot), (uint32_t)(it / W_RING) & 1u, abort_flag, a.status,
+                   a.timeout_ns, honour))
+      return -2;
+    return ring[slot];
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, pending = 0, pend_parity = 0;
+      bool bad_tile = false;
+      for (int it = 0;; ++it) {
+        const int slot = it % W_RING;
+        if (!mbar_wait(iempty_bar(slot), ((uint32_t)(it / W_RING) & 1u) ^ 1u, abort_flag,
+                       a.status, a.timeout_ns, true))
+          break;
+        const long long v = atomicAdd(sch.counter, 1);
+        const int L = v < sch.total ? (int)v : -1;
+        ring[slot] = L;
+        mbar_arrive(ifull_bar(slot));
+        if (L < 0) break;
+        const WideTile t = wide_tile(a, sch, L);
+        if (!t.ok) {
+          bad_tile = true;
+          continue;
+        }
+        const bool two = t.nrows > HM;
+        const int brow = t.e * 2 * a.f + t.n * (WN / 2);
+        const uint32_t tx = (two ? 2 : 1) * W_HALF_A + W_B_BYTES;
+        bool stop = false;
+        for (int kb = 0; kb < a.n_k; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status, a.timeout_ns,
+                         true)) {
+            stop = true;
+            break;
+          }
+          mbar_expect_tx(full_bar(stage), tx);
+          // B first: the weights come from the farthest memory
+          tma_load_2d(sB(stage), &tmW, full_bar(stage), kb * WK, brow);
+          tma_load_2d(sB(stage) + W_B_BYTES / 2, &tmW, full_bar(stage), kb * WK, brow + a.f);
+          tma_load_2d(sA(stage), &tmX, full_bar(stage), kb * WK, t.row0);
+          if (two) tma_load_2d(sA(stage) + W_HALF_A, &tmX, full_bar(stage), kb * WK, t.row0 + HM);
+          pending |= 1u << stage;
+          pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == W_ST) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (stop) break;
+      }
+      if (bad_tile) set_status(a.status, MOE_STATUS_PLAN);
+      if (*abort_flag) {
+        // let the copies already armed land before shared memory goes away
+        for (int s = 0; s < W_ST; ++s)
+          if (pending >> s & 1u)
+            mbar_wait(full_bar(s), pend_parity >> s & 1u, abort_flag, a.status, a.timeout_ns,
+                      false);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc_it = 0;
+      bool issued = false;
+      for (int it = 0;; ++it) {
+        const int L = take_item(it, true);
+        if (L == -2) break;
+        mbar_arrive(iempty_bar(it % W_RING));
+        if (L < 0) break;
+        const WideTile t = wide_tile(a, sch, L);
+        if (!t.ok) continue;
+        const bool two = t.nrows > HM;
+        // the previous item's accumulators have been read out
+        if (!mbar_wait(tempty_bar, ((uint32_t)acc_it & 1u) ^ 1u, abort_flag, a.status,
+                       a.timeout_ns, true))
+          break;
+        tc_fence_after();
+        bool stop = false;
+        for (int kb = 0; kb < a.n_k; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, a.status, a.timeout_ns, true)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = sA(stage), b0 = sB(stage);
+#pragma unroll
+          for (int kk = 0; kk < WK / 16; ++kk) {
+            const uint32_t acc = (kb | kk) != 0;
+            umma_bf16<false>(tmem_base, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32),
+                             W_IDESC, acc);
+            if (two)
+              umma_bf16<false>(tmem_base + WN, sw128_desc(a0 + W_HALF_A + kk * 32),
+                               sw128_desc(b0 + kk * 32), W_IDESC, acc);
+          }
+          issued = true;
+          umma_commit_all<false>(empty_bar(stage));
+          if (++stage == W_ST) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (stop) break;
+        umma_commit_all<false>(tfull_bar);
+        ++acc_it;
+      }
+      if (issued) {
+        umma_commit_local<false>(drain_bar);
+        mbar_wait(drain_bar, 0, abort_flag, a.status, a.timeout_ns, false);
+      }
+    }
+  } else if (warp < 2 + W_EPI_WARPS) {
+    // ------------------------------------------------------------ epilogue (warps 2..9)
+    const int quarter = warp & 3;  // TMEM lanes 32 quarter .. +31 = rows of each half
+    const int ch = (warp - 2) >> 2;  // output columns [64 ch, +64) of the n-tile
+    // staging: quarter q's rows hold two 32-row x 128-byte boxes (columns 0..63, 64..127)
+    uint8_t* my_box = stg + quarter * 8192 + ch * 4096 + lane * 128;
+    int acc_it = 0, staged_n = 0;
+    for (int it = 0;; ++it) {
+      const int L = take_item(it, true);
+      if (!__all_sync(0xffffffffu, L != -2)) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(iempty_bar(it % W_RING));
+      if (L < 0) break;
+      const WideTile t = wide_tile(a, sch, L);
+      if (!t.ok) continue;
+      const int halves = t.nrows > HM ? 2 : 1;
+      const bool got = wait_inl(tfull_bar, (uint32_t)acc_it & 1u, abort_flag, a.status,
+                                a.timeout_ns);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      bool ok = true;
+#pragma unroll 1
+      for (int h = 0; h < halves; ++h) {
+        // the staging buffer is free once the store warp's copies have read the last half
+        const bool fr = wait_inl(stgfree_bar, ((uint32_t)staged_n & 1u) ^ 1u, abort_flag,
+                                 a.status, a.timeout_ns);
+        if (!__all_sync(0xffffffffu, fr)) {
+          ok = false;
+          break;
+        }
+        // accumulator columns of half h: G at [256 h, +128), U at [256 h + 128, +128); this
+        // warp takes G and U columns [64 ch, +64) in two chunks of 32, each written to its
+        // box row as soon as it is converted: 16-byte chunk c of the 128-byte row sits at
+        // chunk position c ^ (row & 7) (128-byte swizzle; row = lane)
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t g[32], u[32];
+          const int col = 64 * ch + 32 * cc;
+          tmem_ld32(taddr + h * WN + col, g);
+          tmem_ld32(taddr + h * WN + WN / 2 + col, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t p[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int c = 8 * i + 2 * j;
+              p[j] = pack_bf16(silu_tanh(__uint_as_float(g[c])) * __uint_as_float(u[c]),
+                               silu_tanh(__uint_as_float(g[c + 1])) * __uint_as_float(u[c + 1]));
+            }
+            const int chunk = cc * 4 + i;
+            *reinterpret_cast<uint4*>(my_box + ((chunk ^ (lane & 7)) << 4)) =
+                make_uint4(p[0], p[1], p[2], p[3]);
+          }
+        }
+        if (h == halves - 1) {
+          // every accumulator column of this item has been read: the next item may start
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar);
+        }
+        fence_proxy_async();  // make the staging writes visible to the TMA engine
+        __syncwarp();
+        if (lane == 0) mbar_arrive(staged_bar);
+        ++staged_n;
+      }
+      if (!ok) break;
+      ++acc_it;
+    }
+  } else {
+    // ------------------------------------------------------------ store warp (warp 10)
+    if (lane == 0) {
+      int staged_n = 0;
+      for (int it = 0;; ++it) {
+        const int L = take_item(it, true);
+        if (L == -2) break;
+        mbar_arrive(iempty_bar(it % W_RING));
+        if (L < 0) break;
+        const WideTile t = wide_tile(a, sch, L);
+        if (!t.ok) continue;
+        const int halves = t.nrows > HM ? 2 : 1;
+        bool stop = false;
+        for (int h = 0; h < halves; ++h) {
+          if (!mbar_wait(staged_bar, (uint32_t)staged_n & 1u, abort_flag, a.status,
+                         a.timeout_ns, true)) {
+            stop = true;
+            break;
+          }
+          const int rows = min(t.nrows - HM * h, HM);
+          for (int q = 0; q < 4; ++q) {
+            if (32 * q >= rows) break;
+            const uint32_t src = smem_u32(stg + q * 8192);
+            const int y = t.row0 + HM * h + 32 * q;
+            tma_store_2d(&tmA, src, t.n * 128, y);
+            tma_store_2d(&tmA, src + 4096, t.n * 128 + 64, y);
+          }
+          bulk_commit();
+          bulk_wait_read();  // the copies have read the staging buffer
+          mbar_arrive(stgfree_bar);
+          ++staged_n;
+        }
+        if (stop) break;
+      }
+      bulk_wait_all();  // A is written before the CTA's shared memory goes away
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<false, 512>(tmem_base);
+  }
+}
+
+}  // namespace
+
+bool fc1_wide_supported(int mode) {
+  return !(mode & (MOE_FFN_SM_PAIR | MOE_FFN_GATHER_X | MOE_FFN_SAVE_Z | MOE_FFN_FC1_M128));
+}
+
+cudaError_t launch_fc1_wide(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
+                            const int32_t* tiles, const int32_t* plan_info, uint16_t* a_out,
+                            int32_t* sched, int32_t* status, bool strict, cudaStream_t st) {
+  const long long r_max = max_rows(c);
+  CUtensorMap tm_x, tm_w, tm_a;
+  // Xp: 128-row boxes; W1: the n-tile's 128 G (or U) rows; A: 32-row store boxes
+  if (!encode_2d(&tm_x, xp, c.d, r_max, HM) ||
+      !encode_2d(&tm_w, w1, c.d, (uint64_t)c.E * 2 * c.f, WN / 2) ||
+      !encode_2d(&tm_a, a_out, c.f, r_max, 32))
+    return cudaErrorInvalidValue;
+  static OncePerDevice attr_once;
+  cudaError_t err = once_per_device(attr_once, [&](int&) {
+    return cudaFuncSetAttribute(fc1_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                W_SMEM);
+  });
+  if (err != cudaSuccess) return err;
+  WideArgs a{};
+  a.sched = sched;
+  a.tiles = tiles;
+  a.plan_info = plan_info;
+  a.status = status;
+  a.r_max = r_max;
+  a.E = c.E;
+  a.P = c.P;
+  a.f = c.f;
+  a.n_k = c.d / WK;
+  a.n_n = c.f / 128;
+  a.strict = strict ? 1 : 0;
+  a.timeout_ns = 2000000000ull;
+  fc1_wide_kernel<<<num_sms(), W_THREADS, W_SMEM, st>>>(tm_x, tm_w, tm_a, a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

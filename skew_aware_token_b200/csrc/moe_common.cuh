@@ -17,7 +17,8 @@ constexpr long long kMaxN = 1LL << 22;
 // every flag moe_expert_ffn accepts
 constexpr int kFfnModes = MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR |
                           MOE_FFN_GATHER_X | MOE_FFN_SAVE_Z | MOE_FFN_ONE_LAUNCH |
-                          MOE_FFN_TWO_LAUNCHES | MOE_FFN_TEST_WAIT_TIMEOUT;
+                          MOE_FFN_TWO_LAUNCHES | MOE_FFN_TEST_WAIT_TIMEOUT |
+                          MOE_FFN_FC1_M128;
 // flags the one-launch FFN does not combine with
 constexpr int kOneLaunchExcludes = MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR |
                                    MOE_FFN_GATHER_X | MOE_FFN_TWO_LAUNCHES;
@@ -108,6 +109,15 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
                        const uint16_t* w2, const int32_t* tiles, const int32_t* plan_info,
                        const int32_t* row_token, const float* row_gate, int mode,
                        uint16_t* a_scratch, void* out, int32_t* status, cudaStream_t st);
+// FC1 on whole 256-row tiles (ffn_wide.cu): the two-launch FFN's FC1 unless the mode asks
+// for SM pairs, rows gathered from x, Z kept for the backward, or 128-row halves
+bool fc1_wide_supported(int mode);
+cudaError_t launch_fc1_wide(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
+                            const int32_t* tiles, const int32_t* plan_info, uint16_t* a_out,
+                            int32_t* sched, int32_t* status, bool strict, cudaStream_t st);
+// execution units of the FFN launches for this mode (SMs, or SM pairs): strict slots need
+// at least P of them
+int ffn_units(int mode);
 cudaError_t launch_combine(const moe_cfg& c, const uint16_t* o, const int32_t* tok_row,
                            const float* gates, float* y, int32_t* status, cudaStream_t st);
 cudaError_t launch_dispatch_grad(const moe_cfg& c, const float* dy, const int32_t* row_token,

@@ -1,5 +1,5 @@
 """Host-side helpers of bench.py, on CPU: the FC1/FC2 launch rule it mirrors from
-moe_expert_ffn (one launch when FC1 has at most 32 work items per SM), the committed DRAM
+moe_expert_ffn (one launch when FC1 has at most 2 work items per SM), the committed DRAM
 traffic record and its source digest, and the peak figures."""
 import json
 import os
@@ -15,19 +15,19 @@ from skew_aware_token_b200 import native as N  # noqa: E402
 from skew_aware_token_b200.synth import WORKLOADS, Workload  # noqa: E402
 
 
-@pytest.mark.parametrize("name,one", [("olmoe_a1", True), ("qwen3_a1.5", True),
+@pytest.mark.parametrize("name,one", [("tiny", True), ("olmoe_a1", False), ("qwen3_a1.5", False),
                                       ("sweep_all4_p0_b128", False), ("dsv3_a1", False)])
 def test_one_launch_rule_at_148_sms(name, one):
-    # FC1 items = (T k / 128) (f / 128): OLMoE 2048, Qwen3 3072, sweep 6144, DeepSeek-V3
-    # 16384; the threshold is 32 x 148 = 4736
+    # FC1 items = (T k / 128) (f / 128): tiny 32, OLMoE 2048, Qwen3 3072, sweep 6144,
+    # DeepSeek-V3 16384; the threshold is 2 x 148 = 296
     assert bench.ffn_one_launch(WORKLOADS[name], 0, 148) is one
 
 
 def test_one_launch_rule_boundary_and_flags():
-    wl = Workload("edge", T=4736 * 128 // 8, d=256, E=8, k=8, f=128, beta=128, P=1, s=0)
-    assert wl.T * wl.k // 128 * (wl.f // 128) == 32 * 148
+    wl = Workload("edge", T=296 * 128 // 8, d=256, E=8, k=8, f=128, beta=128, P=1, s=0)
+    assert wl.T * wl.k // 128 * (wl.f // 128) == 2 * 148
     assert bench.ffn_one_launch(wl, 0, 148)            # at the threshold: one launch
-    assert not bench.ffn_one_launch(wl, 0, 147)        # one item per SM over it: two
+    assert not bench.ffn_one_launch(wl, 0, 147)        # over the threshold: two
     for flag in (N.MOE_FFN_WRITE_O, N.MOE_FFN_STRICT_SLOTS, N.MOE_FFN_SM_PAIR,
                  N.MOE_FFN_GATHER_X, N.MOE_FFN_TWO_LAUNCHES):
         assert not bench.ffn_one_launch(wl, flag, 148), flag

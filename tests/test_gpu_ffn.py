@@ -31,7 +31,9 @@ MODES = [N.MOE_FFN_FUSED_COMBINE, N.MOE_FFN_WRITE_O,
          N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_SM_PAIR,
          N.MOE_FFN_WRITE_O | N.MOE_FFN_SM_PAIR | N.MOE_FFN_STRICT_SLOTS,
          N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_ONE_LAUNCH,
-         N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_TWO_LAUNCHES]
+         N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_TWO_LAUNCHES,
+         N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_TWO_LAUNCHES | N.MOE_FFN_FC1_M128,
+         N.MOE_FFN_WRITE_O | N.MOE_FFN_FC1_M128 | N.MOE_FFN_STRICT_SLOTS]
 
 
 _ORACLE = {}
@@ -62,8 +64,9 @@ def test_ffn_every_element(wl, gather_x):
     ref = _oracle_full(wl, w1, w2)
     layer = MoeLayer(wl, "cuda", write_o=True, gather_x=gather_x)
     for mode in MODES:
-        if gather_x and mode & (N.MOE_FFN_ONE_LAUNCH | N.MOE_FFN_TWO_LAUNCHES):
-            continue  # launch-count flags are for the Xp path
+        if gather_x and mode & (N.MOE_FFN_ONE_LAUNCH | N.MOE_FFN_TWO_LAUNCHES |
+                                N.MOE_FFN_FC1_M128):
+            continue  # launch-count and FC1 tile flags are for the Xp path
         layer.y.fill_(float("nan"))
         run_gpu(wl, w1, w2, mode=mode, layer=layer)
         assert layer.read_status() == 0, (mode, N.moe_status_string(layer.read_status()))
@@ -75,11 +78,16 @@ def test_ffn_every_element(wl, gather_x):
             check_y(o[rows], ref["O"][rows], f"{wl.name} O rows")
 
 
-def test_intermediate_a_matches_swiglu():
-    wl = FULL_CASES[2]
+@pytest.mark.parametrize("mode", [N.MOE_FFN_ONE_LAUNCH, N.MOE_FFN_TWO_LAUNCHES,
+                                  N.MOE_FFN_TWO_LAUNCHES | N.MOE_FFN_FC1_M128],
+                         ids=["one_launch", "fc1_whole_tiles", "fc1_tile_halves"])
+@pytest.mark.parametrize("wl", [FULL_CASES[1], FULL_CASES[2]], ids=lambda w: w.name)
+def test_intermediate_a_matches_swiglu(wl, mode):
+    """FC1's output A on every valid row, for each FC1 kernel (tile halves in one launch or
+    two, whole 256-row tiles)."""
     w1, w2 = synth.make_weights(wl, "cuda")
     ref = _oracle_full(wl, w1, w2)
-    layer = run_gpu(wl, w1, w2)
+    layer = run_gpu(wl, w1, w2, mode=mode)
     rows = np.nonzero(ref["row_token"] >= 0)[0]
     A = f32(layer.view("a_scratch"))[rows]
     _, x = host_inputs(wl)
@@ -97,10 +105,12 @@ def test_intermediate_a_matches_swiglu():
 @pytest.mark.parametrize("name", ["qwen3_a1.5", "dsv3_a1"])
 def test_one_launch_full_size_sampled_tokens(name):
     """FC1 and FC2 in one launch at full size: sampled tokens against the oracle, and the
-    whole y against the two-launch FFN (same arithmetic, atomics may reorder last bits)."""
+    whole y against the two-launch FFN on the same 128-row FC1 tiles (same arithmetic,
+    atomics may reorder last bits)."""
     wl = WORKLOADS[name]
     w1, w2 = synth.make_weights(wl, "cuda")
-    layer = run_gpu(wl, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_TWO_LAUNCHES)
+    layer = run_gpu(wl, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_TWO_LAUNCHES |
+                    N.MOE_FFN_FC1_M128)
     y2 = layer.view("y").clone()
     run_gpu(wl, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_ONE_LAUNCH, layer=layer)
     assert layer.read_status() == 0
