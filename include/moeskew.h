@@ -144,6 +144,16 @@ enum {
                                 256 rows (two M = 128 MMAs sharing each weight stage, the
                                 two-launch default).  The one-launch FFN, SM pairs, rows
                                 gathered from x and MOE_FFN_SAVE_Z always use tile halves */
+  MOE_FFN_FC2_WHOLE = 512,   /* flag: run the fused-combine FC2 on whole tiles (two M = 128
+                                MMAs sharing each weight stage) instead of on tile halves.
+                                Whole tiles need a third less L2 traffic per MMA, but both
+                                256-column accumulators then fill TMEM and the fp32
+                                reductions of an item no longer overlap the next item's
+                                MMAs; on the layers measured halves are as fast or faster,
+                                so this is off by default.  With MOE_FFN_WRITE_O the
+                                two-launch FFN's FC2 always runs whole tiles (its O rows
+                                leave through TMA stores); SM pairs and the one-launch FFN
+                                always use tile halves */
   MOE_FFN_GATHER_X = 8       /* flag: the `xp` argument is x itself (bf16 [T, d]); FC1
                                 gathers each tile's rows x[row_token[r]] straight into
                                 shared memory (TMA row gather), so the dispatched copy

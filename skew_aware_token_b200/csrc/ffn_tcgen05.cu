@@ -123,19 +123,29 @@ struct FfnArgs {
   int32_t* ready;
   int ready_target;
   int strict;
+  int n_group;   // n-tiles per group of the item order (see Sched); n_n: no grouping
   unsigned long long timeout_ns;
 };
 
 // ------------------------------------------------------------------ work schedule
-// Item L of a unit's range -> tile m, n-tile n and (single SM) the tile half.
+// Item L of a unit's range -> tile m, n-tile n and (single SM) the tile half.  Items come in
+// groups of n_group n-tiles (column stripes of the output): group by group, within a group
+// row by row (a row = a tile half, or a tile), within a row its n-tiles.  With
+// n_group = n_n that is row by row with all n-tiles of a row together.
 struct Sched {
   int32_t* counter;  // global counter this unit draws items from
   long long total;   // items in its range
   long long total1;  // PHASE 3: the first total1 items are FC1's, the rest FC2's
   int m_base, n_n, n_n2, halves;
+  int rows;          // rows (tile halves, or tiles) in the unit's range
+  int n_group;
   __device__ void decode(int L, int& m, int& n, int& half) const {
-    n = L % n_n;
-    const int t = L / n_n;
+    const int per_group = rows * n_group;
+    const int g = L / per_group;
+    const int r = L - g * per_group;
+    const int width = min(n_group, n_n - g * n_group);  // the last group may be narrower
+    const int t = r / width;
+    n = g * n_group + (r - t * width);
     m = m_base + t / halves;
     half = t % halves;
   }
@@ -163,9 +173,12 @@ __device__ Sched make_sched(const FfnArgs& a) {
   const int* pi = a.plan_info;
   s.n_n2 = a.n_n2;
   s.total1 = 1LL << 62;
+  // grouping only for a plain FC2 launch (PHASE 3 decodes its FC2 items separately)
+  s.n_group = (a.n_group > 0 && a.n_group < a.n_n && a.n_n2 == 0) ? a.n_group : a.n_n;
   if (!a.strict) {
     s.counter = a.sched;
-    s.total = (long long)max(pi[MOE_PI_NTILES], 0) * a.n_n * s.halves;
+    s.rows = max(pi[MOE_PI_NTILES], 0) * s.halves;
+    s.total = (long long)s.rows * a.n_n;
     s.m_base = 0;
     if (a.n_n2 > 0) {  // PHASE 3: FC2's items after FC1's
       s.total1 = s.total;
@@ -175,7 +188,8 @@ __device__ Sched make_sched(const FfnArgs& a) {
     const int r = unit % a.P;
     const int lo = pi[MOE_PI_SLOT_TILE_OFF + r], hi = pi[MOE_PI_SLOT_TILE_OFF + r + 1];
     s.counter = a.sched + r;
-    s.total = (long long)max(hi - lo, 0) * a.n_n * s.halves;
+    s.rows = max(hi - lo, 0) * s.halves;
+    s.total = (long long)s.rows * a.n_n;
     s.m_base = lo;
   }
   return s;
@@ -908,6 +922,7 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   a1.strict = (mode & MOE_FFN_STRICT_SLOTS) != 0;
   a1.timeout_ns = kTimeoutNs;
 
+  a1.n_group = 0;  // FC1: no grouping
   FfnArgs a2 = a1;
   a1.sched = sched;
   a1.out = a_scratch;
@@ -925,6 +940,7 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   a2.out = out;
   a2.n_k = c.f / BK;
   a2.n_n = c.d / BN;
+  a2.n_group = write_o ? a2.n_n : fc2_n_group(c);
   a2.out_ld = c.d;
   a2.write_o = write_o;
 
@@ -966,8 +982,38 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
     err = pair ? launch_one<1, true>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a1, st)
                : launch_one<1, false>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a1, st);
   if (err != cudaSuccess) return err;
+  if (fc2_wide_supported(mode))
+    return launch_fc2_wide(c, a_scratch, w2, tiles, plan_info, row_token, row_gate, out,
+                           write_o, a2.sched, status, a2.strict != 0, st);
   return pair ? launch_one<2, true>(tm_a, tm_w2, tm_a64, tm_a, tm_w2, a2, st)
               : launch_one<2, false>(tm_a, tm_w2, tm_a64, tm_a, tm_w2, a2, st);
+}
+
+int fc2_n_group(const moe_cfg& c) {
+  // FC2's fused combine adds into y (T x d fp32).  When y is larger than what stays in L2,
+  // its lines are written back and fetched again between a token's k contributions (the
+  // sweep layer's 134 MB y cost 2 GB of DRAM traffic in FC2, about 10 y).  Items taken in
+  // groups of n-tiles keep only the group's y columns live (T x 256 x 4 bytes per n-tile),
+  // at the price of reading A once per group.  Estimated DRAM bytes: A x groups, plus y x 2
+  // when the group's columns fit in 64 MB of L2 and y x 10 when they do not; the group
+  // count with the least estimate wins (ties: fewer groups), groups of equal width.
+  const int n_n = c.d / BN;
+  const double stripe = (double)c.T * BN * 4;
+  const double y_bytes = stripe * n_n;
+  const double a_bytes = (double)max_rows(c) * c.f * 2;
+  const double live_cap = 64.0 * 1024 * 1024;
+  int best = n_n;
+  double best_cost = 0;
+  for (int groups = 1; groups <= n_n; ++groups) {
+    const int width = (n_n + groups - 1) / groups;
+    if ((n_n + width - 1) / width != groups) continue;  // same as a smaller group count
+    const double cost = a_bytes * groups + (stripe * width <= live_cap ? 2.0 : 10.0) * y_bytes;
+    if (groups == 1 || cost < best_cost) {
+      best_cost = cost;
+      best = width;
+    }
+  }
+  return best;
 }
 
 int ffn_units(int mode) {

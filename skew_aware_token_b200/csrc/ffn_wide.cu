@@ -1,40 +1,53 @@
-// FC1 + SwiGLU of the grouped expert FFN on whole 256-row tiles (tcgen05 + TMEM, TMA in
-// and out), the default FC1 of the two-launch FFN.
+// The grouped expert FFN on whole 256-row tiles (tcgen05 + TMEM, fed by TMA): FC1 + SwiGLU,
+// and FC2 with the gate-weighted combine fused into its epilogue.  These are the two-launch
+// FFN's default kernels.
 //
-// "MegaFlux" summary, Methodology 2, expert-computation equation: Z_e = X_e W1_e,
-// Z_e = [G_e, U_e], A_e = SiLU(G_e) * U_e.  A work item is one planner tile (up to 256 rows
-// of one expert) times one n-tile of 128 output columns of A.
+// "MegaFlux" summary, Methodology 2, expert-computation equation:
+//   Z_e = X_e W1_e,  Z_e = [G_e, U_e],  A_e = SiLU(G_e) * U_e,  O_e = A_e W2_e,
+//   y_t = sum_{e in S_t} p_{t,e} O_e[t].
+// A work item is one planner tile (up to 256 rows of one expert) times one n-tile: 128
+// output columns of A for FC1 (the B tile stacks the n-tile's 128 G rows of W1_e over its
+// 128 U rows), 256 output columns of y for FC2.
 //
-// Why a 256-row tile on one SM: a K step of 64 then moves A (256 rows, 32 KB) and B (the
-// n-tile's 128 G rows over its 128 U rows, 32 KB) for 2 x 128x256x64 MMAs, i.e. 64 bytes
-// per tensor-core clock of the SM, where a 128-row tile moves 48 KB per 128x256x64 MMA
-// (96 B/clk).  On B200 an SM takes in about 69 B/clk from L2 (copies from L2 plus, for a
-// cta_group::2 pair, the partner's B half), so the 128-row tile is capped near 0.73 of the
-// tensor rate and the 256-row tile is not (0.98 measured with operands in L2).  The price:
-// the two 128x256 fp32 accumulators fill all 512 TMEM columns, so the epilogue of an item
-// does not overlap the next item's MMAs.  The epilogue is kept short:
-//   - SiLU(g) = g/2 + (g/2) tanh(g/2) with the tanh.approx instruction (one MUFU op);
-//   - the warps that read TMEM never touch global memory (a thread's global stores held up
-//     its later tcgen05.ld waits): they write A, rounded to bf16, into a shared-memory
-//     staging buffer laid out as 32-row x 64-column boxes with the 128-byte swizzle, and a
-//     store warp writes the boxes to A with TMA (cp.async.bulk.tensor, shared -> global).
+// Why a 256-row tile on one SM: a K step of 64 then moves A (256 rows, 32 KB) and B (256
+// rows, 32 KB) for 2 x 128x256x64 MMAs, i.e. 64 bytes per tensor-core clock of the SM, where
+// a 128-row tile moves 48 KB per 128x256x64 MMA (96 B/clk).  On B200 an SM takes in about
+// 69 B/clk from L2 (copies from L2 plus, for a cta_group::2 pair, the partner's B half), so
+// the 128-row tile is capped near 0.73 of the tensor rate and the 256-row tile is not (0.98
+// measured with operands in L2).  The price: the two 128x256 fp32 accumulators fill all 512
+// TMEM columns, so an item's epilogue does not overlap the next item's MMAs, and it is kept
+// short:
+//   FC1: SiLU(g) = g/2 + (g/2) tanh(g/2) with the tanh.approx instruction (one MUFU op); the
+//        warps that read TMEM never touch global memory (a warp's pending global stores
+//        hold up its later instructions, TMEM loads included): they write A, rounded to
+//        bf16, into a shared-memory staging buffer laid out as 32-row x 64-column boxes with
+//        the 128-byte swizzle, and a store warp writes the boxes to A with TMA stores.
+//   FC2, fused combine: each warp scales its 32 rows by the gates, transposes 32 x 32 chunks
+//        through a swizzled 4 KB shared-memory slot and adds them into y with 16-byte vector
+//        reductions, each instruction covering four whole 128-byte row segments.
+//   FC2, O rows (MOE_FFN_WRITE_O): O rounded to bf16 leaves like FC1's A, through the
+//        staging buffer and TMA stores (256 columns per item: two 128-column rounds per half);
+//        moe_combine then adds each token's k rows in order.
+// The fused-combine FC2 on whole tiles is an option (MOE_FFN_FC2_WHOLE): its reductions,
+// about 2 TB/s of fp32 adds into y competing with the operand copies for L2, cannot overlap
+// the next item's MMAs here, and the tile-half FC2 (double-buffered accumulators) is as fast
+// or faster on the layers measured.
 //
 // Roles (352 threads, one CTA per SM, persistent):
 //   warp 0      TMA producer: draws items from the global (or, strict slots, the slot's)
-//               counter, passes them through a ring in shared memory, loads A rows
-//               [row0, row0 + 256) of Xp (the second 128-row box only when the tile has
-//               more than 128 rows) and the n-tile's G and U rows of W1_e per K step into a
-//               3-stage ring (128-byte swizzle).
+//               counter, passes them through a ring in shared memory, and loads per K step
+//               the A rows [row0, row0 + 256) (the second 128-row box only when the tile
+//               has more than 128 rows) and the item's 256 B rows into a 3-stage ring
+//               (128-byte swizzle).
 //   warp 1      MMA issuer: per K step tcgen05.mma.cta_group::1.kind::f16 M=128 N=256 for
 //               rows 0..127 into TMEM columns [0, 256), and for rows 128..255 into
 //               [256, 512); commit frees the stage; after the last K step the accumulators
 //               go to the epilogue.
 //   warps 2..9  epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (32 rows of each half)
-//               and 64 of the n-tile's 128 output columns ((w - 2) / 4 picks which),
-//               A = SiLU(G) * U -> bf16 -> staging (one half at a time).
-//   warp 10     store warp: TMA stores of the staged boxes whose rows are in the tile (tile
-//               sizes are multiples of 64 rows), then frees the staging buffer once the
-//               copies have read it.
+//               and half of the accumulator columns ((w - 2) / 4 picks which).
+//   warp 10     store warp (FC1, and FC2 with O rows): TMA stores of the staged boxes whose
+//               rows are in the tile (tile sizes are multiples of 64 rows), then frees the
+//               staging buffer once the copies have read it.  Idle in the fused combine.
 // Every wait is bounded (globaltimer); on expiry the kernel sets MOE_STATUS_TIMEOUT, the
 // other roles drop out, copies and MMAs in flight are waited for, TMEM is freed.
 #include "tc_util.cuh"
@@ -45,13 +58,13 @@ namespace {
 constexpr int WM = 256;                 // rows per item
 constexpr int HM = 128;                 // rows per MMA (TMEM lanes)
 constexpr int WK = 64;                  // K per stage: one 128-byte swizzle span of bf16
-constexpr int WN = 256;                 // MMA N: 128 G + 128 U columns
+constexpr int WN = 256;                 // MMA N (FC1: 128 G + 128 U columns)
 constexpr int W_ST = 3;                 // stages
 constexpr int W_A_BYTES = WM * WK * 2;  // 32 KB
 constexpr int W_B_BYTES = WN * WK * 2;  // 32 KB
 constexpr int W_STAGE = W_A_BYTES + W_B_BYTES;
-constexpr int W_HALF_A = HM * WK * 2;   // one 128-row A box
-constexpr int W_STG_BYTES = HM * 128 * 2;  // one half of the item's A: 128 rows x 128 cols
+constexpr int W_HALF_A = HM * WK * 2;   // one 128-row box
+constexpr int W_STG_BYTES = 32768;      // 128 rows x 128 bf16 (one store round); FC2 fused: 8 x 4 KB
 constexpr int W_RING = 8;
 constexpr int W_EPI_WARPS = 8;          // two per TMEM lane quadrant
 constexpr int W_THREADS = 32 * (3 + W_EPI_WARPS);
@@ -61,6 +74,7 @@ constexpr int W_META = 512;
 constexpr int W_SMEM = W_ST * W_STAGE + W_STG_BYTES + W_META + 1024;
 static_assert(W_SMEM <= 227 * 1024, "shared memory");
 static_assert(W_NBARS * 8 + 4 * (2 + W_RING) <= W_META, "meta");
+static_assert(W_EPI_WARPS * 4096 <= W_STG_BYTES, "FC2 transpose slots");
 // kind::f16: D fp32, A and B bf16, both K-major, N = 256, M = 128
 constexpr uint32_t W_IDESC =
     (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(WN >> 3) << 17) | ((uint32_t)(HM >> 4) << 24);
@@ -69,34 +83,44 @@ struct WideArgs {
   int32_t* sched;  // item counters: [0], or [slot] with strict slots; zeroed by the host
   const int32_t* tiles;
   const int32_t* plan_info;
+  const int32_t* row_token;  // FC2
+  const float* row_gate;     // FC2
+  float* y;                  // FC2: y fp32 [T, d], zeroed by the host
   int32_t* status;
   long long r_max;
-  int E, P, f, n_k, n_n;
+  int T, d, E, P, f;
+  int n_k, n_n;     // K steps of 64, n-tiles per tile
+  int n_group;      // n-tiles per group of the item order (n_n: no grouping)
+  int brows_per_e;  // B rows per expert: FC1 2f, FC2 d
   int strict;
   unsigned long long timeout_ns;
 };
 
+// Items come in groups of n_group n-tiles (column stripes of the output): group by group,
+// within a group tile by tile, within a tile its n-tiles.
 struct WideSched {
   int32_t* counter;
   long long total;
-  int m_base, n_n;
+  int m_base, n_n, n_group, tiles;
 };
 
 __device__ WideSched wide_sched(const WideArgs& a) {
   WideSched s;
   s.n_n = a.n_n;
+  s.n_group = (a.n_group > 0 && a.n_group < a.n_n) ? a.n_group : a.n_n;
   const int* pi = a.plan_info;
   if (!a.strict) {
     s.counter = a.sched;
-    s.total = (long long)max(pi[MOE_PI_NTILES], 0) * a.n_n;
+    s.tiles = max(pi[MOE_PI_NTILES], 0);
     s.m_base = 0;
   } else {
     const int r = (int)blockIdx.x % a.P;
     const int lo = pi[MOE_PI_SLOT_TILE_OFF + r], hi = pi[MOE_PI_SLOT_TILE_OFF + r + 1];
     s.counter = a.sched + r;
-    s.total = (long long)max(hi - lo, 0) * a.n_n;
+    s.tiles = max(hi - lo, 0);
     s.m_base = lo;
   }
+  s.total = (long long)s.tiles * a.n_n;
   return s;
 }
 
@@ -106,8 +130,13 @@ struct WideTile {
 };
 __device__ __forceinline__ WideTile wide_tile(const WideArgs& a, const WideSched& s, int L) {
   WideTile t;
-  t.n = L % s.n_n;
-  const int m = s.m_base + L / s.n_n;
+  const int per_group = s.tiles * s.n_group;
+  const int g = L / per_group;
+  const int r = L - g * per_group;
+  const int width = min(s.n_group, s.n_n - g * s.n_group);  // the last group may be narrower
+  const int mt = r / width;
+  t.n = g * s.n_group + (r - mt * width);
+  const int m = s.m_base + mt;
   const int4 v = __ldg(reinterpret_cast<const int4*>(a.tiles) + m);
   t.e = v.x;
   t.row0 = v.y;
@@ -133,9 +162,9 @@ __device__ __forceinline__ void bulk_wait_read() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
-// The bounded mbarrier wait of tc_util.cuh, inlined: the epilogue keeps its packed A values
-// in registers across the wait for the staging buffer, and a call would save them to the
-// stack (local-memory stores that hold up the thread's next tcgen05.ld wait).
+// The bounded mbarrier wait of tc_util.cuh, inlined: the epilogue keeps values in registers
+// across its waits, and a call would save them to the stack (local-memory stores, which
+// hold up the warp like any other pending global store).
 __device__ __forceinline__ bool wait_inl(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          int32_t* status, unsigned long long timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -161,9 +190,15 @@ __device__ __forceinline__ float silu_tanh(float g) {
   return fmaf(h, t, h);
 }
 
+// What an item's epilogue produces
+enum { EPI_SWIGLU = 1, EPI_COMBINE = 2, EPI_STORE_O = 3 };
+
+// KIND EPI_SWIGLU: FC1 + SwiGLU -> A (tmO = A's store map); EPI_COMBINE: FC2 + fused
+// combine -> y; EPI_STORE_O: FC2 -> O bf16 (tmO = O's store map)
+template <int KIND>
 __global__ void __launch_bounds__(W_THREADS, 1)
-fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                const __grid_constant__ CUtensorMap tmA, const WideArgs a) {
+wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+            const __grid_constant__ CUtensorMap tmO, const WideArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -185,6 +220,8 @@ fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   auto iempty_bar = [&](int i) { return smem_u32(bars + 2 * W_ST + 5 + W_RING + i); };
   auto sA = [&](int s) { return smem_u32(smem + s * W_STAGE); };
   auto sB = [&](int s) { return smem_u32(smem + s * W_STAGE + W_A_BYTES); };
+  constexpr int PHASE = KIND == EPI_SWIGLU ? 1 : 2;
+  constexpr bool STORE_WARP = KIND != EPI_COMBINE;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < W_ST; ++s) {
@@ -195,17 +232,18 @@ fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     mbar_init(tfull_bar, 1);
     mbar_init(tempty_bar, W_EPI_WARPS);
     mbar_init(staged_bar, W_EPI_WARPS);
-    mbar_init(stgfree_bar, 1);  // the store thread
+    mbar_init(stgfree_bar, 1);
     for (int i = 0; i < W_RING; ++i) {
       mbar_init(ifull_bar(i), 1);
-      mbar_init(iempty_bar(i), 2 + W_EPI_WARPS);  // MMA thread, epilogue warps, store thread
+      // MMA thread, epilogue warps (and the store thread)
+      mbar_init(iempty_bar(i), 1 + W_EPI_WARPS + (STORE_WARP ? 1 : 0));
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     prefetch_tmap(&tmX);
     prefetch_tmap(&tmW);
-    prefetch_tmap(&tmA);
+    if (STORE_WARP) prefetch_tmap(&tmO);
   }
   if (warp == 1) tmem_alloc<false, 512>(smem_u32(tmem_slot));
   tc_fence_before();
@@ -214,11 +252,12 @@ fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   const uint32_t tmem_base = *tmem_slot;
   const WideSched sch = wide_sched(a);
 
-  // consumers: the item of ring position `it`, or -1 when the work is done or a wait gave up
-  auto take_item = [&](int it, bool honour) -> int {
+  // consumers: the item of ring position `it`, -1 when the work is done, -2 when the wait
+  // gave up
+  auto take_item = [&](int it) -> int {
     const int slot = it % W_RING;
     if (!mbar_wait(ifull_bar(slot), (uint32_t)(it / W_RING) & 1u, abort_flag, a.status,
-                   a.timeout_ns, honour))
+                   a.timeout_ns, true))
       return -2;
     return ring[slot];
   };
@@ -245,7 +284,9 @@ fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
           continue;
         }
         const bool two = t.nrows > HM;
-        const int brow = t.e * 2 * a.f + t.n * (WN / 2);
+        // B rows: FC1 the n-tile's G rows (its U rows f further on), FC2 256 rows of W2_e
+        const int brow = t.e * a.brows_per_e + t.n * (PHASE == 1 ? WN / 2 : WN);
+        const int brow2 = PHASE == 1 ? brow + a.f : brow + WN / 2;
         const uint32_t tx = (two ? 2 : 1) * W_HALF_A + W_B_BYTES;
         bool stop = false;
         for (int kb = 0; kb < a.n_k; ++kb) {
@@ -257,7 +298,7 @@ fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
           mbar_expect_tx(full_bar(stage), tx);
           // B first: the weights come from the farthest memory
           tma_load_2d(sB(stage), &tmW, full_bar(stage), kb * WK, brow);
-          tma_load_2d(sB(stage) + W_B_BYTES / 2, &tmW, full_bar(stage), kb * WK, brow + a.f);
+          tma_load_2d(sB(stage) + W_B_BYTES / 2, &tmW, full_bar(stage), kb * WK, brow2);
           tma_load_2d(sA(stage), &tmX, full_bar(stage), kb * WK, t.row0);
           if (two) tma_load_2d(sA(stage) + W_HALF_A, &tmX, full_bar(stage), kb * WK, t.row0 + HM);
           pending |= 1u << stage;
@@ -286,7 +327,7 @@ fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
       int acc_it = 0;
       bool issued = false;
       for (int it = 0;; ++it) {
-        const int L = take_item(it, true);
+        const int L = take_item(it);
         if (L == -2) break;
         mbar_arrive(iempty_bar(it % W_RING));
         if (L < 0) break;
@@ -333,13 +374,11 @@ fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     }
   } else if (warp < 2 + W_EPI_WARPS) {
     // ------------------------------------------------------------ epilogue (warps 2..9)
-    const int quarter = warp & 3;  // TMEM lanes 32 quarter .. +31 = rows of each half
-    const int ch = (warp - 2) >> 2;  // output columns [64 ch, +64) of the n-tile
-    // staging: quarter q's rows hold two 32-row x 128-byte boxes (columns 0..63, 64..127)
-    uint8_t* my_box = stg + quarter * 8192 + ch * 4096 + lane * 128;
+    const int quarter = warp & 3;    // TMEM lanes 32 quarter .. +31 = rows of each half
+    const int ch = (warp - 2) >> 2;  // accumulator column half (FC1: of G and of U)
     int acc_it = 0, staged_n = 0;
     for (int it = 0;; ++it) {
-      const int L = take_item(it, true);
+      const int L = take_item(it);
       if (!__all_sync(0xffffffffu, L != -2)) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(iempty_bar(it % W_RING));
@@ -353,60 +392,128 @@ fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
       bool ok = true;
+      if constexpr (KIND != EPI_COMBINE) {
+        // staging: quarter q's rows hold two 32-row x 128-byte boxes (columns 0..63, 64..127)
+        // of one round: 128 output columns of one half (FC1: the item's A columns; O rows:
+        // rounds 0 and 1 take accumulator columns [0, 128) and [128, 256) of the half)
+        uint8_t* my_box = stg + quarter * 8192 + ch * 4096 + lane * 128;
+        constexpr int ROUNDS = KIND == EPI_SWIGLU ? 1 : 2;
 #pragma unroll 1
-      for (int h = 0; h < halves; ++h) {
-        // the staging buffer is free once the store warp's copies have read the last half
-        const bool fr = wait_inl(stgfree_bar, ((uint32_t)staged_n & 1u) ^ 1u, abort_flag,
-                                 a.status, a.timeout_ns);
-        if (!__all_sync(0xffffffffu, fr)) {
-          ok = false;
-          break;
-        }
-        // accumulator columns of half h: G at [256 h, +128), U at [256 h + 128, +128); this
-        // warp takes G and U columns [64 ch, +64) in two chunks of 32, each written to its
-        // box row as soon as it is converted: 16-byte chunk c of the 128-byte row sits at
-        // chunk position c ^ (row & 7) (128-byte swizzle; row = lane)
+        for (int hr = 0; hr < halves * ROUNDS; ++hr) {
+          const int h = hr / ROUNDS, rnd = hr % ROUNDS;
+          // the staging buffer is free once the store warp's copies have read the last round
+          const bool fr = wait_inl(stgfree_bar, ((uint32_t)staged_n & 1u) ^ 1u, abort_flag,
+                                   a.status, a.timeout_ns);
+          if (!__all_sync(0xffffffffu, fr)) {
+            ok = false;
+            break;
+          }
+          // this warp converts 64 output columns in two chunks of 32, each written to its
+          // box row as soon as it is converted: 16-byte chunk c of the 128-byte row sits at
+          // chunk position c ^ (row & 7) (128-byte swizzle; row = lane)
 #pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t g[32], u[32];
-          const int col = 64 * ch + 32 * cc;
-          tmem_ld32(taddr + h * WN + col, g);
-          tmem_ld32(taddr + h * WN + WN / 2 + col, u);
-          tmem_wait_ld();
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t p[16];
+            if constexpr (KIND == EPI_SWIGLU) {
+              // accumulator columns of half h: G at [256 h, +128), U at [256 h + 128, +128)
+              uint32_t g[32], u[32];
+              const int col = 64 * ch + 32 * cc;
+              tmem_ld32(taddr + h * WN + col, g);
+              tmem_ld32(taddr + h * WN + WN / 2 + col, u);
+              tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t p[4];
+              for (int i = 0; i < 16; ++i)
+                p[i] = pack_bf16(silu_tanh(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]),
+                                 silu_tanh(__uint_as_float(g[2 * i + 1])) *
+                                     __uint_as_float(u[2 * i + 1]));
+            } else {
+              uint32_t v[32];
+              tmem_ld32(taddr + h * WN + 128 * rnd + 64 * ch + 32 * cc, v);
+              tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int c = 8 * i + 2 * j;
-              p[j] = pack_bf16(silu_tanh(__uint_as_float(g[c])) * __uint_as_float(u[c]),
-                               silu_tanh(__uint_as_float(g[c + 1])) * __uint_as_float(u[c + 1]));
+              for (int i = 0; i < 16; ++i)
+                p[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
             }
-            const int chunk = cc * 4 + i;
-            *reinterpret_cast<uint4*>(my_box + ((chunk ^ (lane & 7)) << 4)) =
-                make_uint4(p[0], p[1], p[2], p[3]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int chunk = cc * 4 + i;
+              *reinterpret_cast<uint4*>(my_box + ((chunk ^ (lane & 7)) << 4)) =
+                  make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            }
+          }
+          if (hr == halves * ROUNDS - 1) {
+            // every accumulator column of this item has been read: the next item may start
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar);
+          }
+          fence_proxy_async();  // make the staging writes visible to the TMA engine
+          __syncwarp();
+          if (lane == 0) mbar_arrive(staged_bar);
+          ++staged_n;
+        }
+      } else {
+        // fused combine: y[token] += gate * O over columns [256 n + 128 ch, +128) for this
+        // warp's 32 rows of each half.  Each 32 x 32 chunk is staged in this warp's 4 KB slot
+        // (row r's 16-byte group j at position j ^ (r & 7)); then lanes 8q..8q+7 of a vector
+        // reduction take one 128-byte row segment.
+        float* slot_f = reinterpret_cast<float*>(stg + (warp - 2) * 4096);
+#pragma unroll 1
+        for (int h = 0; h < halves; ++h) {
+          const int rit = HM * h + 32 * quarter + lane;  // row inside the tile
+          const long long row = (long long)t.row0 + rit;
+          int tok = -1;
+          float gate = 0.f;
+          if (rit < t.nrows && row < a.r_max) {
+            tok = __ldg(a.row_token + row);
+            gate = __ldg(a.row_gate + row);
+            if (tok >= a.T) tok = -1;
+          }
+          float* ybase = a.y + (long long)t.n * WN + 128 * ch + 4 * (lane & 7);
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            tmem_ld32(taddr + h * WN + 128 * ch + 32 * c, v);
+            tmem_wait_ld();
+            if (h == halves - 1 && c == 3) {
+              // every accumulator column of this item has been read
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(tempty_bar);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<float4*>(slot_f + 32 * lane + 4 * (j ^ (lane & 7))) =
+                  make_float4(gate * __uint_as_float(v[4 * j]),
+                              gate * __uint_as_float(v[4 * j + 1]),
+                              gate * __uint_as_float(v[4 * j + 2]),
+                              gate * __uint_as_float(v[4 * j + 3]));
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int r = 4 * i + (lane >> 3);
+              const int tk = __shfl_sync(0xffffffffu, tok, r);
+              if (tk >= 0) {
+                const float4 x = *reinterpret_cast<const float4*>(
+                    slot_f + 32 * r + 4 * ((lane & 7) ^ (r & 7)));
+                red_add_v4(ybase + (long long)tk * a.d + 32 * c, x);
+              }
+            }
+            __syncwarp();
           }
         }
-        if (h == halves - 1) {
-          // every accumulator column of this item has been read: the next item may start
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tempty_bar);
-        }
-        fence_proxy_async();  // make the staging writes visible to the TMA engine
-        __syncwarp();
-        if (lane == 0) mbar_arrive(staged_bar);
-        ++staged_n;
       }
       if (!ok) break;
       ++acc_it;
     }
-  } else {
+  } else if (STORE_WARP) {
     // ------------------------------------------------------------ store warp (warp 10)
     if (lane == 0) {
+      constexpr int ROUNDS = KIND == EPI_SWIGLU ? 1 : 2;
+      constexpr int OCOLS = 128 * ROUNDS;  // output columns per item
       int staged_n = 0;
       for (int it = 0;; ++it) {
-        const int L = take_item(it, true);
+        const int L = take_item(it);
         if (L == -2) break;
         mbar_arrive(iempty_bar(it % W_RING));
         if (L < 0) break;
@@ -414,19 +521,21 @@ fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         if (!t.ok) continue;
         const int halves = t.nrows > HM ? 2 : 1;
         bool stop = false;
-        for (int h = 0; h < halves; ++h) {
+        for (int hr = 0; hr < halves * ROUNDS; ++hr) {
+          const int h = hr / ROUNDS, rnd = hr % ROUNDS;
           if (!mbar_wait(staged_bar, (uint32_t)staged_n & 1u, abort_flag, a.status,
                          a.timeout_ns, true)) {
             stop = true;
             break;
           }
           const int rows = min(t.nrows - HM * h, HM);
+          const int x0 = t.n * OCOLS + 128 * rnd;
           for (int q = 0; q < 4; ++q) {
             if (32 * q >= rows) break;
             const uint32_t src = smem_u32(stg + q * 8192);
             const int y = t.row0 + HM * h + 32 * q;
-            tma_store_2d(&tmA, src, t.n * 128, y);
-            tma_store_2d(&tmA, src + 4096, t.n * 128 + 64, y);
+            tma_store_2d(&tmO, src, x0, y);
+            tma_store_2d(&tmO, src + 4096, x0 + 64, y);
           }
           bulk_commit();
           bulk_wait_read();  // the copies have read the staging buffer
@@ -435,7 +544,7 @@ fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         }
         if (stop) break;
       }
-      bulk_wait_all();  // A is written before the CTA's shared memory goes away
+      bulk_wait_all();  // the output is written before the CTA's shared memory goes away
     }
   }
 
@@ -447,10 +556,45 @@ fc1_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   }
 }
 
+template <int KIND>
+cudaError_t launch_wide(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& to,
+                        const WideArgs& a, cudaStream_t st) {
+  static OncePerDevice attr_once;
+  cudaError_t err = once_per_device(attr_once, [&](int&) {
+    return cudaFuncSetAttribute(wide_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                W_SMEM);
+  });
+  if (err != cudaSuccess) return err;
+  wide_kernel<KIND><<<num_sms(), W_THREADS, W_SMEM, st>>>(tx, tw, to, a);
+  return cudaGetLastError();
+}
+
+WideArgs wide_args(const moe_cfg& c, const int32_t* tiles, const int32_t* plan_info,
+                   int32_t* sched, int32_t* status, bool strict) {
+  WideArgs a{};
+  a.sched = sched;
+  a.tiles = tiles;
+  a.plan_info = plan_info;
+  a.status = status;
+  a.r_max = max_rows(c);
+  a.T = c.T;
+  a.d = c.d;
+  a.E = c.E;
+  a.P = c.P;
+  a.f = c.f;
+  a.strict = strict ? 1 : 0;
+  a.timeout_ns = 2000000000ull;
+  return a;
+}
+
 }  // namespace
 
 bool fc1_wide_supported(int mode) {
   return !(mode & (MOE_FFN_SM_PAIR | MOE_FFN_GATHER_X | MOE_FFN_SAVE_Z | MOE_FFN_FC1_M128));
+}
+bool fc2_wide_supported(int mode) {
+  if (mode & MOE_FFN_SM_PAIR) return false;
+  return (mode & (MOE_FFN_WRITE_O | MOE_FFN_FC2_WHOLE)) != 0;
 }
 
 cudaError_t launch_fc1_wide(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
@@ -463,27 +607,39 @@ cudaError_t launch_fc1_wide(const moe_cfg& c, const uint16_t* xp, const uint16_t
       !encode_2d(&tm_w, w1, c.d, (uint64_t)c.E * 2 * c.f, WN / 2) ||
       !encode_2d(&tm_a, a_out, c.f, r_max, 32))
     return cudaErrorInvalidValue;
-  static OncePerDevice attr_once;
-  cudaError_t err = once_per_device(attr_once, [&](int&) {
-    return cudaFuncSetAttribute(fc1_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                W_SMEM);
-  });
-  if (err != cudaSuccess) return err;
-  WideArgs a{};
-  a.sched = sched;
-  a.tiles = tiles;
-  a.plan_info = plan_info;
-  a.status = status;
-  a.r_max = r_max;
-  a.E = c.E;
-  a.P = c.P;
-  a.f = c.f;
+  WideArgs a = wide_args(c, tiles, plan_info, sched, status, strict);
   a.n_k = c.d / WK;
   a.n_n = c.f / 128;
-  a.strict = strict ? 1 : 0;
-  a.timeout_ns = 2000000000ull;
-  fc1_wide_kernel<<<num_sms(), W_THREADS, W_SMEM, st>>>(tm_x, tm_w, tm_a, a);
-  return cudaGetLastError();
+  a.n_group = a.n_n;
+  a.brows_per_e = 2 * c.f;
+  return launch_wide<EPI_SWIGLU>(tm_x, tm_w, tm_a, a, st);
+}
+
+cudaError_t launch_fc2_wide(const moe_cfg& c, const uint16_t* a_in, const uint16_t* w2,
+                            const int32_t* tiles, const int32_t* plan_info,
+                            const int32_t* row_token, const float* row_gate, void* out,
+                            bool write_o, int32_t* sched, int32_t* status, bool strict,
+                            cudaStream_t st) {
+  const long long r_max = max_rows(c);
+  CUtensorMap tm_a, tm_w, tm_o;
+  // A: 128-row boxes; W2: 128-row boxes (two per 256-row n-tile); O: 32-row store boxes
+  if (!encode_2d(&tm_a, a_in, c.f, r_max, HM) ||
+      !encode_2d(&tm_w, w2, c.f, (uint64_t)c.E * c.d, WN / 2) ||
+      (write_o && !encode_2d(&tm_o, out, c.d, r_max, 32)))
+    return cudaErrorInvalidValue;
+  WideArgs a = wide_args(c, tiles, plan_info, sched, status, strict);
+  a.row_token = row_token;
+  a.row_gate = row_gate;
+  a.n_k = c.f / WK;
+  a.n_n = c.d / WN;
+  a.brows_per_e = c.d;
+  if (write_o) {
+    a.n_group = a.n_n;
+    return launch_wide<EPI_STORE_O>(tm_a, tm_w, tm_o, a, st);
+  }
+  a.y = static_cast<float*>(out);
+  a.n_group = fc2_n_group(c);
+  return launch_wide<EPI_COMBINE>(tm_a, tm_w, tm_a, a, st);
 }
 
 }  // namespace moe

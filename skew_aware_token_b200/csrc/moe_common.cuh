@@ -18,7 +18,7 @@ constexpr long long kMaxN = 1LL << 22;
 constexpr int kFfnModes = MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR |
                           MOE_FFN_GATHER_X | MOE_FFN_SAVE_Z | MOE_FFN_ONE_LAUNCH |
                           MOE_FFN_TWO_LAUNCHES | MOE_FFN_TEST_WAIT_TIMEOUT |
-                          MOE_FFN_FC1_M128;
+                          MOE_FFN_FC1_M128 | MOE_FFN_FC2_WHOLE;
 // flags the one-launch FFN does not combine with
 constexpr int kOneLaunchExcludes = MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR |
                                    MOE_FFN_GATHER_X | MOE_FFN_TWO_LAUNCHES;
@@ -109,12 +109,22 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
                        const uint16_t* w2, const int32_t* tiles, const int32_t* plan_info,
                        const int32_t* row_token, const float* row_gate, int mode,
                        uint16_t* a_scratch, void* out, int32_t* status, cudaStream_t st);
-// FC1 on whole 256-row tiles (ffn_wide.cu): the two-launch FFN's FC1 unless the mode asks
-// for SM pairs, rows gathered from x, Z kept for the backward, or 128-row halves
+// FC1 + SwiGLU on whole 256-row tiles (ffn_wide.cu): the two-launch FFN's FC1 unless the
+// mode asks for SM pairs, rows gathered from x, Z kept for the backward, or 128-row halves
 bool fc1_wide_supported(int mode);
 cudaError_t launch_fc1_wide(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
                             const int32_t* tiles, const int32_t* plan_info, uint16_t* a_out,
                             int32_t* sched, int32_t* status, bool strict, cudaStream_t st);
+// FC2 on whole 256-row tiles: the two-launch FFN's FC2 with O rows (unless on SM pairs), and
+// with the fused combine when the mode asks for MOE_FFN_FC2_WHOLE
+bool fc2_wide_supported(int mode);
+cudaError_t launch_fc2_wide(const moe_cfg& c, const uint16_t* a_in, const uint16_t* w2,
+                            const int32_t* tiles, const int32_t* plan_info,
+                            const int32_t* row_token, const float* row_gate, void* out,
+                            bool write_o, int32_t* sched, int32_t* status, bool strict,
+                            cudaStream_t st);
+// n-tiles of 256 output columns per group of FC2's item order (ffn_tcgen05.cu)
+int fc2_n_group(const moe_cfg& c);
 // execution units of the FFN launches for this mode (SMs, or SM pairs): strict slots need
 // at least P of them
 int ffn_units(int mode);

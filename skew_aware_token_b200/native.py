@@ -30,6 +30,7 @@ MOE_FFN_ONE_LAUNCH = 32
 MOE_FFN_TWO_LAUNCHES = 64
 MOE_FFN_TEST_WAIT_TIMEOUT = 128
 MOE_FFN_FC1_M128 = 256
+MOE_FFN_FC2_WHOLE = 512
 PI = dict(B=0, TAU=1, MAKESPAN=2, VARIANT=3, NTILES=4, FIXED_MAKESPAN=5, REPLICAS=6,
           ROUNDS=7, SLOT_TILE_OFF=8, VAR_MAKESPAN=17, VAR_REPLICAS=22, VAR_ROUNDS=27,
           QUOTA_TAU=32, COST=33, VAR_COST=34, LEN=40)

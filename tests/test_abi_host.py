@@ -96,7 +96,7 @@ def test_null_and_misaligned_pointers_rejected():
     assert lib.moe_dispatch_permute(cfg, *disp, None) == N.MOE_ERR_UNSUPPORTED
     for bad_mask in (1 << 6, 1 << 7, 1 << 24, 0xFFFFFFFF):  # bits 6, 7 and 24..31 are unused
         assert lib.moe_plan_blocks(cfg, ok, bad_mask, *[ok] * 8, None) == N.MOE_ERR_INVALID_ARG
-    assert lib.moe_expert_ffn(cfg, *[ok] * 7, 512, *[ok] * 3, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_ffn(cfg, *[ok] * 7, 1024, *[ok] * 3, None) == N.MOE_ERR_INVALID_ARG
     bad_d = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(d=320)))
     assert lib.moe_expert_ffn(bad_d, *[ok] * 7, 0, *[ok] * 3, None) == N.MOE_ERR_UNSUPPORTED
     bad_f = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(f=192)))

@@ -33,6 +33,9 @@ MODES = [N.MOE_FFN_FUSED_COMBINE, N.MOE_FFN_WRITE_O,
          N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_ONE_LAUNCH,
          N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_TWO_LAUNCHES,
          N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_TWO_LAUNCHES | N.MOE_FFN_FC1_M128,
+         N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_TWO_LAUNCHES | N.MOE_FFN_FC2_WHOLE,
+         N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_FC2_WHOLE | N.MOE_FFN_STRICT_SLOTS,
+         N.MOE_FFN_FUSED_COMBINE | N.MOE_FFN_FC1_M128 | N.MOE_FFN_STRICT_SLOTS,
          N.MOE_FFN_WRITE_O | N.MOE_FFN_FC1_M128 | N.MOE_FFN_STRICT_SLOTS]
 
 
@@ -65,7 +68,7 @@ def test_ffn_every_element(wl, gather_x):
     layer = MoeLayer(wl, "cuda", write_o=True, gather_x=gather_x)
     for mode in MODES:
         if gather_x and mode & (N.MOE_FFN_ONE_LAUNCH | N.MOE_FFN_TWO_LAUNCHES |
-                                N.MOE_FFN_FC1_M128):
+                                N.MOE_FFN_FC1_M128 | N.MOE_FFN_FC2_WHOLE):
             continue  # launch-count and FC1 tile flags are for the Xp path
         layer.y.fill_(float("nan"))
         run_gpu(wl, w1, w2, mode=mode, layer=layer)
