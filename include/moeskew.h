@@ -82,7 +82,9 @@ enum {
   MOE_WS_BLOCKS = 1,
   MOE_WS_FFN_SCRATCH = 2,
   MOE_WS_FFN_SCRATCH_Z = 3,  /* a_scratch of moe_expert_ffn with MOE_FFN_SAVE_Z */
-  MOE_WS_BWD_SCRATCH = 4     /* bwd_scratch of moe_expert_ffn_backward */
+  MOE_WS_BWD_SCRATCH = 4,    /* bwd_scratch of moe_expert_ffn_backward */
+  MOE_WS_FFN_RECORD = 5      /* byte offset in a_scratch of the slot record written with
+                                MOE_FFN_RECORD_SLOTS (int32 [B_max]) */
 };
 
 /* plan_info layout (int32[MOE_PI_LEN]) written by moe_plan_blocks */
@@ -154,6 +156,14 @@ enum {
                                 two-launch FFN's FC2 always runs whole tiles (its O rows
                                 leave through TMA stores); SM pairs and the one-launch FFN
                                 always use tile halves */
+  MOE_FFN_RECORD_SLOTS = 1024, /* diagnostic flag: the call also records which virtual
+                                slots' execution units ran each execution tile: int32 word
+                                m of the slot record (at byte offset
+                                moe_workspace_size(cfg, MOE_WS_FFN_RECORD) of a_scratch,
+                                zeroed by the call) gets bit (u mod P) when unit u (an SM,
+                                or an SM pair) ran one of tile m's FC1 items and bit
+                                8 + (u mod P) for FC2.  With MOE_FFN_STRICT_SLOTS tile m
+                                then holds exactly its slot's two bits */
   MOE_FFN_GATHER_X = 8       /* flag: the `xp` argument is x itself (bf16 [T, d]); FC1
                                 gathers each tile's rows x[row_token[r]] straight into
                                 shared memory (TMA row gather), so the dispatched copy
@@ -166,7 +176,9 @@ enum {
  * MOE_WS_BLOCKS -> B_max entries (blocks, tiles); MOE_WS_FFN_SCRATCH -> bytes of the
  * a_scratch buffer of moe_expert_ffn (A, bf16 [R_max, f], rounded up to 256 bytes, then
  * 256 bytes of tile-scheduler counters, then 2 * B_max int32 readiness counters rounded
- * up to 256 bytes); MOE_WS_FFN_SCRATCH_Z -> the same followed by
+ * up to 256 bytes, then the B_max int32 slot record rounded up to 256 bytes);
+ * MOE_WS_FFN_RECORD -> the byte offset of that slot record; MOE_WS_FFN_SCRATCH_Z -> the
+ * same scratch followed by
  * Z (bf16 [R_max, 2f], rounded up to 256 bytes); MOE_WS_BWD_SCRATCH -> bytes of the
  * bwd_scratch buffer of moe_expert_ffn_backward (dZ, bf16 [R_max, 2f], rounded up to 256
  * bytes, then 256 bytes of counters).  Returns 0 for an invalid cfg. */

@@ -51,6 +51,7 @@ size_t moe_workspace_size(const moe_cfg* cfg, int which) {
   if (which == MOE_WS_FFN_SCRATCH) return (size_t)ffn_scratch_bytes(*cfg);
   if (which == MOE_WS_FFN_SCRATCH_Z) return (size_t)ffn_scratch_z_bytes(*cfg);
   if (which == MOE_WS_BWD_SCRATCH) return (size_t)bwd_scratch_bytes(*cfg);
+  if (which == MOE_WS_FFN_RECORD) return (size_t)ffn_record_offset(*cfg);
   return 0;
 }
 

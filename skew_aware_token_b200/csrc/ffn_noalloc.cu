@@ -63,8 +63,10 @@ extern "C" MOE_API int moe_expert_ffn_noalloc(const moe_cfg* cfg, const uint16_t
       c.s < 0 || (c.beta != 64 && c.beta != 128) || c.d < 1 || c.f < 1)
     return MOE_ERR_INVALID_ARG;
   if (c.E > kMaxE || (long long)c.T * c.k > kMaxN) return MOE_ERR_UNSUPPORTED;
-  // the fixed array holds A only: saving Z for a backward pass needs the caller's scratch
-  if (mode & ~kFfnModes || mode & MOE_FFN_SAVE_Z) return MOE_ERR_INVALID_ARG;
+  // the fixed array holds A and counters only: Z for a backward pass needs the caller's
+  // scratch, and a slot record there could not be read back by the caller
+  if (mode & ~kFfnModes || mode & (MOE_FFN_SAVE_Z | MOE_FFN_RECORD_SLOTS))
+    return MOE_ERR_INVALID_ARG;
   if ((mode & (MOE_FFN_ONE_LAUNCH | MOE_FFN_TEST_WAIT_TIMEOUT)) && (mode & kOneLaunchExcludes))
     return MOE_ERR_INVALID_ARG;
   if (c.d % 256 || c.f % 128) return MOE_ERR_UNSUPPORTED;

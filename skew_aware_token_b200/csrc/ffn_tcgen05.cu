@@ -124,8 +124,15 @@ struct FfnArgs {
   int ready_target;
   int strict;
   int n_group;   // n-tiles per group of the item order (see Sched); n_n: no grouping
+  int32_t* slot_rec;  // MOE_FFN_RECORD_SLOTS: per tile, bit (u mod P) [+ 8 for FC2] of every
+                      // unit u that ran one of its items; else null
   unsigned long long timeout_ns;
 };
+
+// the slot record: unit u (an SM, or an SM pair) ran an item of tile m of GEMM gp
+__device__ __forceinline__ void record_slot(const FfnArgs& a, int m, int gp, int unit) {
+  if (a.slot_rec) atomicOr(a.slot_rec + m, 1 << ((unit % a.P) + (gp == 2 ? 8 : 0)));
+}
 
 // ------------------------------------------------------------------ work schedule
 // Item L of a unit's range -> tile m, n-tile n and (single SM) the tile half.  Items come in
@@ -326,6 +333,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         const TileInfo ti = read_tile<PAIR>(a, m, PAIR ? (int)rank : half);
         if (!ti.ok) bad_tile = true;
         if (!ti.run) continue;
+        if (mma_cta) record_slot(a, m, gp, PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x);
         // FC1 B rows: single SM, the n-tile's 128 G rows over its 128 U rows; SM pair, CTA
         // `rank` holds G rows [64 rank, +64) of the n-tile over the matching U rows
         int brow;
@@ -428,6 +436,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     };
     struct Item {
       int L;        // item number, -1: none
+      int m;        // tile
       int brow;     // first B row
       TileInfo ti;
       int mt[4];    // cp.async gather: tokens of rows lane + 32q (padding rows: token 0)
@@ -436,6 +445,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     auto locate = [&](Item& w) {
       int m, n, half;
       sch.decode(w.L, m, n, half);
+      w.m = m;
       w.ti = read_tile<PAIR>(a, m, PAIR ? (int)rank : half);
       // FC1 B rows: single SM, the n-tile's 128 G rows over its 128 U rows; SM pair, CTA
       // `rank` holds G rows [64 rank, +64) of the n-tile over the matching U rows, so that
@@ -485,6 +495,8 @@ ffn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     }
     for (int it = 0; cur.L >= 0; ++it) {
       if (!cur.ti.ok) bad_tile = true;
+      if (cur.ti.run && lane == 0 && mma_cta)
+        record_slot(a, cur.m, PHASE, PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x);
       bool drew = false, located = false, loaded = false;
       took = true;
       nxt.L = -1;
@@ -891,6 +903,13 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
                                               ffn_a_bytes(c));
   err = cudaMemsetAsync(sched, 0, 16 * sizeof(int32_t), st);
   if (err != cudaSuccess) return err;
+  int32_t* slot_rec = nullptr;
+  if (mode & MOE_FFN_RECORD_SLOTS) {
+    slot_rec = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(a_scratch) +
+                                          ffn_record_offset(c));
+    err = cudaMemsetAsync(slot_rec, 0, (size_t)ffn_record_bytes(c), st);
+    if (err != cudaSuccess) return err;
+  }
 
   const bool gather = (mode & MOE_FFN_GATHER_X) != 0;
   // A maps: boxes of 128 rows, and of 64 rows for the SM pair's tiles of at most 128 rows;
@@ -920,6 +939,7 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   a1.E = c.E;
   a1.P = c.P;
   a1.strict = (mode & MOE_FFN_STRICT_SLOTS) != 0;
+  a1.slot_rec = slot_rec;
   a1.timeout_ns = kTimeoutNs;
 
   a1.n_group = 0;  // FC1: no grouping
@@ -974,7 +994,7 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   }
   if (fc1_wide_supported(mode))
     err = launch_fc1_wide(c, xp, w1, tiles, plan_info, a_scratch, sched, status, a1.strict != 0,
-                          st);
+                          slot_rec, st);
   else if (gather)
     err = pair ? launch_one<1, true, true>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a1, st)
                : launch_one<1, false, true>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a1, st);
@@ -984,7 +1004,7 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   if (err != cudaSuccess) return err;
   if (fc2_wide_supported(mode))
     return launch_fc2_wide(c, a_scratch, w2, tiles, plan_info, row_token, row_gate, out,
-                           write_o, a2.sched, status, a2.strict != 0, st);
+                           write_o, a2.sched, status, a2.strict != 0, slot_rec, st);
   return pair ? launch_one<2, true>(tm_a, tm_w2, tm_a64, tm_a, tm_w2, a2, st)
               : launch_one<2, false>(tm_a, tm_w2, tm_a64, tm_a, tm_w2, a2, st);
 }

@@ -93,6 +93,7 @@ struct WideArgs {
   int n_group;      // n-tiles per group of the item order (n_n: no grouping)
   int brows_per_e;  // B rows per expert: FC1 2f, FC2 d
   int strict;
+  int32_t* slot_rec;  // MOE_FFN_RECORD_SLOTS: per tile, bit (unit mod P) [+ 8 for FC2]
   unsigned long long timeout_ns;
 };
 
@@ -125,7 +126,7 @@ __device__ WideSched wide_sched(const WideArgs& a) {
 }
 
 struct WideTile {
-  int e, row0, nrows, n;
+  int m, e, row0, nrows, n;
   bool ok;
 };
 __device__ __forceinline__ WideTile wide_tile(const WideArgs& a, const WideSched& s, int L) {
@@ -137,6 +138,7 @@ __device__ __forceinline__ WideTile wide_tile(const WideArgs& a, const WideSched
   const int mt = r / width;
   t.n = g * s.n_group + (r - mt * width);
   const int m = s.m_base + mt;
+  t.m = m;
   const int4 v = __ldg(reinterpret_cast<const int4*>(a.tiles) + m);
   t.e = v.x;
   t.row0 = v.y;
@@ -283,6 +285,8 @@ wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           bad_tile = true;
           continue;
         }
+        if (a.slot_rec)
+          atomicOr(a.slot_rec + t.m, 1 << ((int)(blockIdx.x % a.P) + (PHASE == 2 ? 8 : 0)));
         const bool two = t.nrows > HM;
         // B rows: FC1 the n-tile's G rows (its U rows f further on), FC2 256 rows of W2_e
         const int brow = t.e * a.brows_per_e + t.n * (PHASE == 1 ? WN / 2 : WN);
@@ -570,7 +574,7 @@ cudaError_t launch_wide(const CUtensorMap& tx, const CUtensorMap& tw, const CUte
 }
 
 WideArgs wide_args(const moe_cfg& c, const int32_t* tiles, const int32_t* plan_info,
-                   int32_t* sched, int32_t* status, bool strict) {
+                   int32_t* sched, int32_t* status, bool strict, int32_t* slot_rec) {
   WideArgs a{};
   a.sched = sched;
   a.tiles = tiles;
@@ -583,6 +587,7 @@ WideArgs wide_args(const moe_cfg& c, const int32_t* tiles, const int32_t* plan_i
   a.P = c.P;
   a.f = c.f;
   a.strict = strict ? 1 : 0;
+  a.slot_rec = slot_rec;
   a.timeout_ns = 2000000000ull;
   return a;
 }
@@ -599,7 +604,8 @@ bool fc2_wide_supported(int mode) {
 
 cudaError_t launch_fc1_wide(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
                             const int32_t* tiles, const int32_t* plan_info, uint16_t* a_out,
-                            int32_t* sched, int32_t* status, bool strict, cudaStream_t st) {
+                            int32_t* sched, int32_t* status, bool strict, int32_t* slot_rec,
+                            cudaStream_t st) {
   const long long r_max = max_rows(c);
   CUtensorMap tm_x, tm_w, tm_a;
   // Xp: 128-row boxes; W1: the n-tile's 128 G (or U) rows; A: 32-row store boxes
@@ -607,7 +613,7 @@ cudaError_t launch_fc1_wide(const moe_cfg& c, const uint16_t* xp, const uint16_t
       !encode_2d(&tm_w, w1, c.d, (uint64_t)c.E * 2 * c.f, WN / 2) ||
       !encode_2d(&tm_a, a_out, c.f, r_max, 32))
     return cudaErrorInvalidValue;
-  WideArgs a = wide_args(c, tiles, plan_info, sched, status, strict);
+  WideArgs a = wide_args(c, tiles, plan_info, sched, status, strict, slot_rec);
   a.n_k = c.d / WK;
   a.n_n = c.f / 128;
   a.n_group = a.n_n;
@@ -619,7 +625,7 @@ cudaError_t launch_fc2_wide(const moe_cfg& c, const uint16_t* a_in, const uint16
                             const int32_t* tiles, const int32_t* plan_info,
                             const int32_t* row_token, const float* row_gate, void* out,
                             bool write_o, int32_t* sched, int32_t* status, bool strict,
-                            cudaStream_t st) {
+                            int32_t* slot_rec, cudaStream_t st) {
   const long long r_max = max_rows(c);
   CUtensorMap tm_a, tm_w, tm_o;
   // A: 128-row boxes; W2: 128-row boxes (two per 256-row n-tile); O: 32-row store boxes
@@ -627,7 +633,7 @@ cudaError_t launch_fc2_wide(const moe_cfg& c, const uint16_t* a_in, const uint16
       !encode_2d(&tm_w, w2, c.f, (uint64_t)c.E * c.d, WN / 2) ||
       (write_o && !encode_2d(&tm_o, out, c.d, r_max, 32)))
     return cudaErrorInvalidValue;
-  WideArgs a = wide_args(c, tiles, plan_info, sched, status, strict);
+  WideArgs a = wide_args(c, tiles, plan_info, sched, status, strict, slot_rec);
   a.row_token = row_token;
   a.row_gate = row_gate;
   a.n_k = c.f / WK;

@@ -18,7 +18,7 @@ constexpr long long kMaxN = 1LL << 22;
 constexpr int kFfnModes = MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR |
                           MOE_FFN_GATHER_X | MOE_FFN_SAVE_Z | MOE_FFN_ONE_LAUNCH |
                           MOE_FFN_TWO_LAUNCHES | MOE_FFN_TEST_WAIT_TIMEOUT |
-                          MOE_FFN_FC1_M128 | MOE_FFN_FC2_WHOLE;
+                          MOE_FFN_FC1_M128 | MOE_FFN_FC2_WHOLE | MOE_FFN_RECORD_SLOTS;
 // flags the one-launch FFN does not combine with
 constexpr int kOneLaunchExcludes = MOE_FFN_WRITE_O | MOE_FFN_STRICT_SLOTS | MOE_FFN_SM_PAIR |
                                    MOE_FFN_GATHER_X | MOE_FFN_TWO_LAUNCHES;
@@ -33,7 +33,7 @@ inline long long max_blocks(const moe_cfg& c) {
 inline long long max_rows(const moe_cfg& c) { return max_blocks(c) * c.beta; }
 
 // FFN scratch: A (bf16 [R_max, f]) rounded up to 256 bytes, then the tile-scheduler
-// counters (kSchedBytes), then the one-launch FFN's readiness counters.
+// counters (kSchedBytes), then the one-launch FFN's readiness counters, then the slot record.
 constexpr long long kSchedBytes = 256;
 inline long long ffn_a_bytes(const moe_cfg& c) {
   return (max_rows(c) * c.f * 2 + 255) / 256 * 256;
@@ -42,8 +42,15 @@ inline long long ffn_a_bytes(const moe_cfg& c) {
 inline long long ffn_ready_bytes(const moe_cfg& c) {
   return (2 * max_blocks(c) * 4 + 255) / 256 * 256;
 }
-inline long long ffn_scratch_bytes(const moe_cfg& c) {
+// slot record of MOE_FFN_RECORD_SLOTS: one int32 per execution tile (tiles <= B_max)
+inline long long ffn_record_bytes(const moe_cfg& c) {
+  return (max_blocks(c) * 4 + 255) / 256 * 256;
+}
+inline long long ffn_record_offset(const moe_cfg& c) {
   return ffn_a_bytes(c) + kSchedBytes + ffn_ready_bytes(c);
+}
+inline long long ffn_scratch_bytes(const moe_cfg& c) {
+  return ffn_record_offset(c) + ffn_record_bytes(c);
 }
 // Z = [G, U] (bf16 [R_max, 2f]) or dZ, rounded up to 256 bytes
 inline long long ffn_z_bytes(const moe_cfg& c) {
@@ -114,7 +121,8 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
 bool fc1_wide_supported(int mode);
 cudaError_t launch_fc1_wide(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
                             const int32_t* tiles, const int32_t* plan_info, uint16_t* a_out,
-                            int32_t* sched, int32_t* status, bool strict, cudaStream_t st);
+                            int32_t* sched, int32_t* status, bool strict, int32_t* slot_rec,
+                            cudaStream_t st);
 // FC2 on whole 256-row tiles: the two-launch FFN's FC2 with O rows (unless on SM pairs), and
 // with the fused combine when the mode asks for MOE_FFN_FC2_WHOLE
 bool fc2_wide_supported(int mode);
@@ -122,7 +130,7 @@ cudaError_t launch_fc2_wide(const moe_cfg& c, const uint16_t* a_in, const uint16
                             const int32_t* tiles, const int32_t* plan_info,
                             const int32_t* row_token, const float* row_gate, void* out,
                             bool write_o, int32_t* sched, int32_t* status, bool strict,
-                            cudaStream_t st);
+                            int32_t* slot_rec, cudaStream_t st);
 // n-tiles of 256 output columns per group of FC2's item order (ffn_tcgen05.cu)
 int fc2_n_group(const moe_cfg& c);
 // execution units of the FFN launches for this mode (SMs, or SM pairs): strict slots need

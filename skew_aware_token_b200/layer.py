@@ -122,9 +122,18 @@ class MoeLayer:
     def __call__(self, logits, x, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, variant_mask=0,
                  stream=None, y=None):
         """Route, plan, dispatch, FFN (+ combine): returns y fp32 [T, d], by default a view
-        of the layer's buffer (valid until the next call), or the caller's `y`.  The
-        planner's search runs on a side stream while the dispatch runs (the dispatch needs
-        only the block offsets); both join before the FFN."""
+        of the layer's buffer (valid until the next call), or the caller's `y`."""
+        self.pre_ffn(logits, x, variant_mask, stream)
+        self.ffn(w1, w2, mode, stream, y, x)
+        if mode & N.MOE_FFN_WRITE_O:
+            self.combine(stream, y)
+        out = self.y if y is None else y
+        return out[: self.wl.T * self.wl.d].view(self.wl.T, self.wl.d)
+
+    def pre_ffn(self, logits, x, variant_mask=0, stream=None):
+        """The stages before the FFN: route + histogram, block offsets, then the planner's
+        search on a side stream while the dispatch runs (the dispatch needs only the block
+        offsets); both join on the main stream."""
         self.route(logits, stream)
         self.block_offsets(stream)
         main = stream if isinstance(stream, torch.cuda.Stream) else \
@@ -138,11 +147,6 @@ class MoeLayer:
         else:  # a raw stream handle: one stream
             self._search(variant_mask, stream)
             self.dispatch(x, stream)
-        self.ffn(w1, w2, mode, stream, y, x)
-        if mode & N.MOE_FFN_WRITE_O:
-            self.combine(stream, y)
-        out = self.y if y is None else y
-        return out[: self.wl.T * self.wl.d].view(self.wl.T, self.wl.d)
 
     def backward(self, dy, w1, w2, stream=None):
         """Gradients of the expert computation for dL/dy = dy (fp32 [T, d]) after a forward
@@ -199,6 +203,10 @@ class MoeLayer:
                 "z": (self.a_scratch[z_off:], (R, 2 * f)), "d_rows": (self.d_rows, (R, d)),
                 "dz": (self.bwd_scratch, (R, 2 * f)), "dx": (self.dx, (T, d)),
                 "dw1": (self.dw1, (E, 2 * f, d)), "dw2": (self.dw2, (E, d, f))})
+        if name == "slot_record":
+            # int32 [B_max] at a byte offset of the FFN scratch (MOE_FFN_RECORD_SLOTS)
+            off = N.moe_workspace_size(self.cfg, N.MOE_WS_FFN_RECORD) // 2
+            return self.a_scratch[off: off + 2 * Bm].view(torch.int32)
         buf, shape = shapes[name]
         n = 1
         for s in shape:

@@ -22,7 +22,7 @@ MOE_NOALLOC_SCRATCH_BYTES = 64 << 20
 MOE_STATUS_BAD_ID, MOE_STATUS_OVERFLOW, MOE_STATUS_NONFINITE = 1, 2, 4
 MOE_STATUS_TIMEOUT, MOE_STATUS_PLAN = 8, 16
 MOE_WS_ROWS, MOE_WS_BLOCKS, MOE_WS_FFN_SCRATCH = 0, 1, 2
-MOE_WS_FFN_SCRATCH_Z, MOE_WS_BWD_SCRATCH = 3, 4
+MOE_WS_FFN_SCRATCH_Z, MOE_WS_BWD_SCRATCH, MOE_WS_FFN_RECORD = 3, 4, 5
 MOE_FFN_FUSED_COMBINE, MOE_FFN_WRITE_O, MOE_FFN_STRICT_SLOTS, MOE_FFN_SM_PAIR = 0, 1, 2, 4
 MOE_FFN_GATHER_X = 8
 MOE_FFN_SAVE_Z = 16
@@ -31,6 +31,7 @@ MOE_FFN_TWO_LAUNCHES = 64
 MOE_FFN_TEST_WAIT_TIMEOUT = 128
 MOE_FFN_FC1_M128 = 256
 MOE_FFN_FC2_WHOLE = 512
+MOE_FFN_RECORD_SLOTS = 1024
 PI = dict(B=0, TAU=1, MAKESPAN=2, VARIANT=3, NTILES=4, FIXED_MAKESPAN=5, REPLICAS=6,
           ROUNDS=7, SLOT_TILE_OFF=8, VAR_MAKESPAN=17, VAR_REPLICAS=22, VAR_ROUNDS=27,
           QUOTA_TAU=32, COST=33, VAR_COST=34, LEN=40)

@@ -45,7 +45,10 @@ def test_workspace_sizes_follow_the_block_bound():
         assert N.moe_workspace_size(wl, N.MOE_WS_ROWS) == b_max * wl.beta
         a_bytes = (b_max * wl.beta * wl.f * 2 + 255) // 256 * 256
         ready_bytes = (2 * b_max * 4 + 255) // 256 * 256  # one-launch readiness counters
-        assert N.moe_workspace_size(wl, N.MOE_WS_FFN_SCRATCH) == a_bytes + 256 + ready_bytes
+        record_bytes = (b_max * 4 + 255) // 256 * 256     # slot record
+        assert N.moe_workspace_size(wl, N.MOE_WS_FFN_RECORD) == a_bytes + 256 + ready_bytes
+        assert N.moe_workspace_size(wl, N.MOE_WS_FFN_SCRATCH) == (a_bytes + 256 + ready_bytes +
+                                                                   record_bytes)
         # the bound holds for the worst routing: every expert one row past a block
         worst = [wl.beta + 1] * wl.E
         if sum(worst) <= Nr:
@@ -96,7 +99,7 @@ def test_null_and_misaligned_pointers_rejected():
     assert lib.moe_dispatch_permute(cfg, *disp, None) == N.MOE_ERR_UNSUPPORTED
     for bad_mask in (1 << 6, 1 << 7, 1 << 24, 0xFFFFFFFF):  # bits 6, 7 and 24..31 are unused
         assert lib.moe_plan_blocks(cfg, ok, bad_mask, *[ok] * 8, None) == N.MOE_ERR_INVALID_ARG
-    assert lib.moe_expert_ffn(cfg, *[ok] * 7, 1024, *[ok] * 3, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_ffn(cfg, *[ok] * 7, 2048, *[ok] * 3, None) == N.MOE_ERR_INVALID_ARG
     bad_d = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(d=320)))
     assert lib.moe_expert_ffn(bad_d, *[ok] * 7, 0, *[ok] * 3, None) == N.MOE_ERR_UNSUPPORTED
     bad_f = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"].with_(f=192)))

@@ -61,3 +61,38 @@ def test_peaks_come_from_the_measured_file_when_present():
 def test_traffic_record_only_for_the_captured_configuration():
     for name in WORKLOADS:
         assert bench.measured_traffic(name, default_ffn=False) is None
+
+
+def test_peak_follows_the_timed_region_length():
+    peaks = {"bf16_tflops": 1612.8, "bf16_tflops_sustained": 1367.4}
+    assert bench.pick_peak(peaks, 0.3) == (1612.8, "burst")
+    assert bench.pick_peak(peaks, bench.SUSTAINED_AFTER_S) == (1367.4, "sustained")
+
+
+def test_roofline_fraction_is_algorithmic_flops_over_time():
+    wl = WORKLOADS["dsv3_a1"]
+    peaks = {"bf16_tflops": 1612.8, "bf16_tflops_sustained": 1367.4}
+    rl = bench.roofline(wl, 12.0, 0.24, peaks, "of measured")
+    achieved = 6 * wl.T * wl.k * wl.d * wl.f / 12e-3 / 1e12
+    assert rl["achieved"] == round(achieved, 2)
+    assert rl["frac"] == round(achieved / 1612.8, 4) and rl["peak"] == 1612.8
+    assert rl["frac_of_sustained"] == round(achieved / 1367.4, 4)
+
+
+def test_launch_count_per_step():
+    wl = WORKLOADS["dsv3_a1"]
+    assert bench.gpu_launches_per_step(wl, 0, 148) == 8
+    assert bench.gpu_launches_per_step(wl, N.MOE_FFN_WRITE_O, 148) == 9
+    assert bench.gpu_launches_per_step(wl, N.MOE_FFN_GATHER_X, 148) == 7
+    assert bench.gpu_launches_per_step(WORKLOADS["tiny"], 0, 148) == 7  # one FFN launch
+
+
+def test_oracle_sample_fits_its_memory_bound():
+    wl = WORKLOADS["dsv3_a1"]
+    logits = bench.synth.make_logits(wl).numpy()
+    n = bench.sample_size(wl, logits, max_bytes=4e9)
+    experts = bench.sample_experts(wl, logits, n)
+    assert 1 <= n < wl.T
+    assert len(experts) * 3 * wl.d * wl.f * 4 <= 4e9
+    # the next doubling would not fit
+    assert len(bench.sample_experts(wl, logits, 2 * n)) * 3 * wl.d * wl.f * 4 > 4e9
