@@ -57,8 +57,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 SUSTAINED_AFTER_S = 2.0
 FLUSH_BYTES = 256 << 20
 # kernels of one step: route + histogram, kappa, block offsets, plan, dispatch rank and
-# gather, FC1, FC2 (the unfused combine adds one)
+# gather, FC1, FC2; the dispatch adds its count and prefix kernels when the pairs span more
+# than one chunk, and O rows add the combine
 LAUNCHES_PER_STEP = 8
+DISPATCH_CHUNK = 1024  # pairs per chunk of the dispatch's counting sort
 
 
 def load_peaks():
@@ -184,7 +186,8 @@ def rmax_rows(wl) -> int:
 
 def gpu_launches_per_step(wl, mode, sms: int) -> int:
     """Kernels of this library launched per step for an FFN mode (see LAUNCHES_PER_STEP)."""
-    return (LAUNCHES_PER_STEP + int(bool(mode & N.MOE_FFN_WRITE_O)) -
+    chunks = wl.T * wl.k // DISPATCH_CHUNK
+    return (LAUNCHES_PER_STEP + 2 * int(chunks > 1) + int(bool(mode & N.MOE_FFN_WRITE_O)) -
             int(bool(mode & N.MOE_FFN_GATHER_X)) - int(ffn_one_launch(wl, mode, sms)))
 
 
@@ -289,8 +292,9 @@ def time_layer(layer, logits, x, w1, w2, mode, vmask, steps, warmup, dev, world,
     flush outside its events.  Per step, events on the launching stream mark the start, the
     end of the stages before the FFN (route, block offsets, plan beside the dispatch) and
     the end of the FFN (and the combine, with O rows).  Returns per-stage mean ms, the sum
-    of step times (max over ranks) and the wall region."""
+    of step times (max over ranks), the wall region and the FFN mode that ran."""
     stream = torch.cuda.current_stream(dev)
+    eff = layer.ffn_mode(mode)  # the layer may run a fused-combine call with O rows
     layer.clear_status()
     for _ in range(warmup):
         flush()
@@ -313,8 +317,8 @@ def time_layer(layer, logits, x, w1, w2, mode, vmask, steps, warmup, dev, world,
             marks[i][0].record(stream)
             layer.pre_ffn(logits, x, vmask)
             marks[i][1].record(stream)
-            layer.ffn(w1, w2, mode, x=x)
-            if mode & N.MOE_FFN_WRITE_O:
+            layer.ffn(w1, w2, eff, x=x)
+            if eff & N.MOE_FFN_WRITE_O:
                 layer.combine()
             marks[i][2].record(stream)
         stop.record(stream)
@@ -330,7 +334,7 @@ def time_layer(layer, logits, x, w1, w2, mode, vmask, steps, warmup, dev, world,
             "ffn_ms_median": statistics.median(ffn),
             "steps_s": max_over_ranks(step_s, dev),
             "ffn_s": max_over_ranks(sum(ffn) / 1e3, dev),
-            "region_s": start.elapsed_time(stop) / 1e3, "wall_s": t_wall}
+            "region_s": start.elapsed_time(stop) / 1e3, "wall_s": t_wall, "mode": eff}
 
 
 class _NullCtx:
@@ -581,7 +585,8 @@ def run_ours(args, wl, world, rank, local):
     logits = logits_h.to(dev)
     x = x_h.to(dev)
     write_o = args.ffn == "write_o"
-    layer = MoeLayer(wl, dev, write_o=True, gather_x=args.gather_x)
+    layer = MoeLayer(wl, dev, write_o=True, gather_x=args.gather_x,
+                     o_rows=None if args.ffn == "auto" else write_o)
     mode = ((N.MOE_FFN_STRICT_SLOTS if args.strict else 0) |
             (N.MOE_FFN_WRITE_O if write_o else 0) | (N.MOE_FFN_SM_PAIR if args.sm_pair else 0) |
             (N.MOE_FFN_ONE_LAUNCH if args.launches == "one" else 0) |
@@ -625,7 +630,9 @@ def run_ours(args, wl, world, rank, local):
         "data": "synthetic (seeded; router logits N(0,1) + Zipf bias, x N(0,1), "
                 "weights N(0, 1/sqrt(fan_in)), random-init)",
         "config": workload_config(wl, {
-            "kappa": kappa, "strict_slots": bool(args.strict), "ffn": args.ffn,
+            "kappa": kappa, "strict_slots": bool(args.strict),
+            "ffn": "O rows + ordered combine" if r["mode"] & N.MOE_FFN_WRITE_O
+            else "FC2 with fused combine",
             "sm_pair": bool(args.sm_pair), "ffn_launches": args.launches,
             "launch": "stream launches, per-step CUDA events",
             "fc1_rows": "gathered from x by row_token" if args.gather_x
@@ -643,8 +650,9 @@ def run_ours(args, wl, world, rank, local):
                        "the timed steps",
         "timed_region_s": round(r["region_s"], 4),
         "roofline": rl, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": gpu_launches_per_step(wl, mode | (N.MOE_FFN_GATHER_X if args.gather_x
-                                                          else 0), sms) * args.steps,
+        "gpu_launches": gpu_launches_per_step(wl, r["mode"] | (N.MOE_FFN_GATHER_X
+                                                               if args.gather_x else 0),
+                                              sms) * args.steps,
         "clocks": clocks.summary(),
         "impl": "ours",
     }
@@ -726,8 +734,9 @@ def main():
                          "launches, or the library's choice by layer size (default)")
     ap.add_argument("--gather-x", action="store_true",
                     help="FC1 gathers its rows from x by row_token (no Xp, no gather kernel)")
-    ap.add_argument("--ffn", default="fused", choices=["fused", "write_o"],
-                    help="fused: FC2 adds gate*O into y; write_o: FC2 stores O, then moe_combine")
+    ap.add_argument("--ffn", default="auto", choices=["auto", "fused", "write_o"],
+                    help="fused: FC2 adds gate*O into y; write_o: FC2 stores O, then "
+                         "moe_combine; auto: the layer's choice by the size of y (default)")
     ap.add_argument("--sm-pair", action="store_true",
                     help="run the FFN on SM pairs (tcgen05 cta_group::2) instead of single SMs")
     ap.add_argument("--strict", action="store_true",

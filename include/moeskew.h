@@ -295,17 +295,23 @@ MOE_API int moe_combine(const moe_cfg* cfg, const uint16_t* o, const int32_t* to
  * device memory (a plugin or custom operator that its host framework hands only inputs
  * and outputs, or a deployment that forbids cudaMalloc after start-up).  The pages have no
  * counterpart: this is a deployment variant of the FFN entry point above.
- *   Arguments, modes, outputs and device status are those of moe_expert_ffn, without
- *   a_scratch: its contents (A and the tile-scheduler counters, together
- *   moe_workspace_size(cfg, MOE_WS_FFN_SCRATCH) bytes) live in a library-owned array of
- *   MOE_NOALLOC_SCRATCH_BYTES, which they must not exceed, else the call returns
- *   MOE_ERR_TOO_LARGE and enqueues nothing.
+ *   Arguments, outputs and device status are those of moe_expert_ffn, without a_scratch:
+ *   its contents (A, the tile-scheduler counters, the one-launch FFN's readiness counters
+ *   and the slot record, together moe_workspace_size(cfg, MOE_WS_FFN_SCRATCH) bytes) live
+ *   in a library-owned array of MOE_NOALLOC_SCRATCH_BYTES, which they must not exceed, else
+ *   the call returns MOE_ERR_TOO_LARGE and enqueues nothing.  The modes are those of
+ *   moe_expert_ffn except MOE_FFN_SAVE_Z (Z for a backward pass needs the caller's
+ *   scratch) and MOE_FFN_RECORD_SLOTS (the caller could not read the record back): both
+ *   return MOE_ERR_INVALID_ARG.
  *   The call allocates nothing.  The array is reserved on every GPU where the library's
  *   device code is loaded, until the process exits.  The first call on a device looks up
  *   the array's device address (cudaGetSymbolAddress, with that device current) and caches
- *   it, so make that first call before any stream capture.
- *   All calls share the array and it keeps the last call's contents; calls whose kernels
- *   overlap on the GPU (e.g. on two streams) race on it and must be serialised. */
+ *   it with the current CUDA context, so make that first call before any stream capture; a
+ *   call under a different context of the device (after cudaDeviceReset) looks it up
+ *   again, so it too must come before any capture.
+ *   All calls share the array and it keeps the last call's contents; every call zeroes the
+ *   counters that must start at zero.  Calls whose kernels overlap on the GPU (e.g. on two
+ *   streams) race on the array and must be serialised. */
 MOE_API int moe_expert_ffn_noalloc(const moe_cfg* cfg, const uint16_t* xp, const uint16_t* w1,
                                    const uint16_t* w2, const int32_t* tiles,
                                    const int32_t* plan_info, const int32_t* row_token,

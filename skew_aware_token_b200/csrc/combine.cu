@@ -5,8 +5,10 @@
 // j = 0..k-1 in fp32, so the result does not depend on scheduling.
 //
 // One warp per token; each lane owns 8-column groups of the row (16-byte bf16 loads of
-// the k expert rows, two 16-byte fp32 stores).  Rows outside the caller's O buffer are
-// skipped and reported (MOE_STATUS_BAD_ID), never read.
+// the k expert rows, two 16-byte fp32 stores), two groups per iteration so that 2k loads
+// are in flight per lane before the first add.  O rows are read once, so the loads bypass
+// L1 (ld.global.nc.L1::no_allocate).  Rows outside the caller's O buffer are skipped and
+// reported (MOE_STATUS_BAD_ID), never read.
 #include <cuda_bf16.h>
 
 #include "moe_common.cuh"
@@ -15,6 +17,15 @@ namespace moe {
 namespace {
 
 constexpr int kCombineThreads = 256;
+constexpr int kGroups = 2;  // 8-column groups per lane per iteration
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
 
 __device__ __forceinline__ void bf16x8_fma(const uint4 v, float g, float* acc) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -49,15 +60,29 @@ combine_kernel(const uint4* __restrict__ o, const int32_t* __restrict__ tok_row,
         }
       }
     }
-    for (int c = lane; c < d8; c += 32) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int c0 = lane; c0 < d8; c0 += 32 * kGroups) {
+      uint4 v[kGroups][kMaxK];
 #pragma unroll
-      for (int j = 0; j < kMaxK; ++j) {
-        if (j < k && rows[j] >= 0) bf16x8_fma(__ldg(o + (long long)rows[j] * d8 + c), g[j], acc);
+      for (int u = 0; u < kGroups; ++u) {
+        const int c = c0 + 32 * u;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+          v[u][j] = (j < k && rows[j] >= 0 && c < d8)
+                        ? ld_stream(o + (long long)rows[j] * d8 + c)
+                        : make_uint4(0, 0, 0, 0);
       }
-      float4* dst = y + (t * d8 + c) * 2;
-      dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+#pragma unroll
+      for (int u = 0; u < kGroups; ++u) {
+        const int c = c0 + 32 * u;
+        if (c >= d8) break;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+          if (j < k && rows[j] >= 0) bf16x8_fma(v[u][j], g[j], acc);
+        float4* dst = y + (t * d8 + c) * 2;
+        dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
     }
   }
   if (bad) set_status(status, MOE_STATUS_BAD_ID);

@@ -11,12 +11,19 @@
 // The array is a file-scope __device__ variable of MOE_NOALLOC_SCRATCH_BYTES (64 MiB).
 // Every GPU on which the library's device code is loaded reserves it until the process
 // exits.  Host code cannot use the variable's name as a device address, so the first
-// call on each device (with that device current) looks the address up once with
-// cudaGetSymbolAddress and caches it; that first call should therefore come before any
-// stream capture.  All calls share the one array: its contents are whatever the last
-// call left, and calls whose kernels overlap on the GPU (for example on two streams)
-// race on it.  The only part that must start at zero, the tile-scheduler counters, is
-// zeroed by every call; FC1 writes every row of A that FC2 reads for an output row.
+// call on each device (with that device current) looks the address up with
+// cudaGetSymbolAddress and caches it together with the CUDA context it belongs to; that
+// first call should therefore come before any stream capture.  A later call under another
+// context of the same device (after cudaDeviceReset, the module is loaded anew and the
+// array may move) looks the address up again instead of using a stale one.  All calls
+// share the one array: its contents are whatever the last call left, and calls whose
+// kernels overlap on the GPU (for example on two streams) race on it.  Every call zeroes
+// the parts that must start at zero: the tile-scheduler counters and, for the one-launch
+// FFN, its per-tile-half readiness counters; FC1 writes every row of A that FC2 reads for
+// an output row.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "moe_common.cuh"
@@ -28,17 +35,41 @@ static __device__ __align__(256) uint8_t g_ffn_scratch[MOE_NOALLOC_SCRATCH_BYTES
 
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 
-// Device address of the array on the current device (looked up once per device).
+// The driver's cuCtxGetCurrent, found once through the runtime (no link-time dependency on
+// the driver library).
+PFN_cuCtxGetCurrent_v4000 ctx_get_current() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  return fn;
+}
+
+// Device address of the array on the current device, looked up once per device and
+// context (again after the context changed, e.g. after cudaDeviceReset).
 int scratch_on_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  auto get_ctx = ctx_get_current();
+  if (!get_ctx) return MOE_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!ctx || !g_scratch_ptr[dev] || g_scratch_ctx[dev] != ctx) {
+    // the lookup also brings up the device's primary context when none is current yet
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_ffn_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+    if (!ctx && (get_ctx(&ctx) != CUDA_SUCCESS || !ctx)) return MOE_ERR_CUDA;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return MOE_OK;

@@ -885,6 +885,16 @@ cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUten
 
 }  // namespace
 
+// Whether a mode without a launch-count flag runs FC1 and FC2 as one launch: tiny layers
+// only (one launch saves a launch and overlaps FC1's tail with FC2's start; from a few items
+// per SM on, two launches with FC1 on whole 256-row tiles are faster, about 10 % on the
+// 4096-token layer with 14 FC1 half-tile items per SM)
+bool ffn_auto_one_launch(const moe_cfg& c, int mode) {
+  if (mode & (kOneLaunchExcludes | MOE_FFN_ONE_LAUNCH | MOE_FFN_TEST_WAIT_TIMEOUT)) return false;
+  const long long fc1_items = (long long)c.T * c.k / BM * (c.f / (BN / 2));
+  return fc1_items <= 2LL * num_sms();
+}
+
 cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
                        const uint16_t* w2, const int32_t* tiles, const int32_t* plan_info,
                        const int32_t* row_token, const float* row_gate, int mode,
@@ -893,7 +903,12 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   const bool pair = (mode & MOE_FFN_SM_PAIR) != 0;
   const long long r_max = max_rows(c);
   cudaError_t err;
-  if (!write_o && c.T > 0) {
+  // y is zeroed for the fused combine: by the whole-tile FC1 kernel beside its work when it
+  // runs (two launches), else by a memset first
+  const bool one_launch_forced = (mode & (MOE_FFN_ONE_LAUNCH | MOE_FFN_TEST_WAIT_TIMEOUT)) != 0;
+  const bool zero_in_fc1 = !write_o && c.T > 0 && r_max > 0 && fc1_wide_supported(mode) &&
+                           !one_launch_forced && !ffn_auto_one_launch(c, mode);
+  if (!write_o && c.T > 0 && !zero_in_fc1) {
     err = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)c.T * c.d, st);
     if (err != cudaSuccess) return err;
   }
@@ -965,14 +980,7 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   a2.write_o = write_o;
 
   const bool test_timeout = (mode & MOE_FFN_TEST_WAIT_TIMEOUT) != 0;
-  bool one_launch = (mode & (MOE_FFN_ONE_LAUNCH | MOE_FFN_TEST_WAIT_TIMEOUT)) != 0;
-  if (!one_launch && !(mode & kOneLaunchExcludes)) {
-    // tiny layers: one launch saves a launch and overlaps FC1's tail with FC2's start.  From
-    // a few items per SM on, two launches with FC1 on whole 256-row tiles are faster (about
-    // 10 % on the 4096-token layer with 14 FC1 half-tile items per SM)
-    const long long fc1_items = (long long)c.T * c.k / BM * (c.f / (BN / 2));
-    one_launch = fc1_items <= 2LL * num_sms();
-  }
+  const bool one_launch = one_launch_forced || ffn_auto_one_launch(c, mode);
   if (one_launch) {
     // FC1 items, then FC2 items, in one persistent launch; FC2 waits per tile half
     int32_t* ready = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(a_scratch) +
@@ -994,7 +1002,7 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
   }
   if (fc1_wide_supported(mode))
     err = launch_fc1_wide(c, xp, w1, tiles, plan_info, a_scratch, sched, status, a1.strict != 0,
-                          slot_rec, st);
+                          slot_rec, zero_in_fc1 ? static_cast<float*>(out) : nullptr, st);
   else if (gather)
     err = pair ? launch_one<1, true, true>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a1, st)
                : launch_one<1, false, true>(tm_xp, tm_w1, tm_xp64, tm_a, tm_w2, a1, st);

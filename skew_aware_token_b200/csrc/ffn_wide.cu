@@ -33,7 +33,7 @@
 // the next item's MMAs here, and the tile-half FC2 (double-buffered accumulators) is as fast
 // or faster on the layers measured.
 //
-// Roles (352 threads, one CTA per SM, persistent):
+// Roles (384 threads, one CTA per SM, persistent):
 //   warp 0      TMA producer: draws items from the global (or, strict slots, the slot's)
 //               counter, passes them through a ring in shared memory, and loads per K step
 //               the A rows [row0, row0 + 256) (the second 128-row box only when the tile
@@ -48,6 +48,9 @@
 //   warp 10     store warp (FC1, and FC2 with O rows): TMA stores of the staged boxes whose
 //               rows are in the tile (tile sizes are multiples of 64 rows), then frees the
 //               staging buffer once the copies have read it.  Idle in the fused combine.
+//   warp 11     FC1 only, when asked: zeroes the CTA's share of y (16-byte stores), which the
+//               following fused-combine FC2 adds into, while FC1 computes; without it the
+//               host writes y with a memset before FC1 (470 MB at T = 16384, d = 7168).
 // Every wait is bounded (globaltimer); on expiry the kernel sets MOE_STATUS_TIMEOUT, the
 // other roles drop out, copies and MMAs in flight are waited for, TMEM is freed.
 #include "tc_util.cuh"
@@ -67,7 +70,8 @@ constexpr int W_HALF_A = HM * WK * 2;   // one 128-row box
 constexpr int W_STG_BYTES = 32768;      // 128 rows x 128 bf16 (one store round); FC2 fused: 8 x 4 KB
 constexpr int W_RING = 8;
 constexpr int W_EPI_WARPS = 8;          // two per TMEM lane quadrant
-constexpr int W_THREADS = 32 * (3 + W_EPI_WARPS);
+constexpr int W_THREADS = 32 * (4 + W_EPI_WARPS);
+constexpr int W_ZERO_WARP = 3 + W_EPI_WARPS;
 // full[ST], empty[ST], drain, tfull, tempty, staged, stgfree, ifull[RING], iempty[RING]
 constexpr int W_NBARS = 2 * W_ST + 5 + 2 * W_RING;
 constexpr int W_META = 512;
@@ -94,6 +98,8 @@ struct WideArgs {
   int brows_per_e;  // B rows per expert: FC1 2f, FC2 d
   int strict;
   int32_t* slot_rec;  // MOE_FFN_RECORD_SLOTS: per tile, bit (unit mod P) [+ 8 for FC2]
+  uint4* zero;        // FC1: y to zero for the fused combine (16-byte units), or null
+  long long zero_n16;
   unsigned long long timeout_ns;
 };
 
@@ -510,6 +516,14 @@ wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       if (!ok) break;
       ++acc_it;
     }
+  } else if (warp == W_ZERO_WARP) {
+    // ------------------------------------------------------------ y zeroing (warp 11)
+    if (a.zero) {
+      const uint4 z = make_uint4(0, 0, 0, 0);
+      for (long long i = (long long)blockIdx.x * 32 + lane; i < a.zero_n16;
+           i += (long long)gridDim.x * 32)
+        a.zero[i] = z;
+    }
   } else if (STORE_WARP) {
     // ------------------------------------------------------------ store warp (warp 10)
     if (lane == 0) {
@@ -605,7 +619,7 @@ bool fc2_wide_supported(int mode) {
 cudaError_t launch_fc1_wide(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
                             const int32_t* tiles, const int32_t* plan_info, uint16_t* a_out,
                             int32_t* sched, int32_t* status, bool strict, int32_t* slot_rec,
-                            cudaStream_t st) {
+                            float* y_zero, cudaStream_t st) {
   const long long r_max = max_rows(c);
   CUtensorMap tm_x, tm_w, tm_a;
   // Xp: 128-row boxes; W1: the n-tile's 128 G (or U) rows; A: 32-row store boxes
@@ -618,6 +632,10 @@ cudaError_t launch_fc1_wide(const moe_cfg& c, const uint16_t* xp, const uint16_t
   a.n_n = c.f / 128;
   a.n_group = a.n_n;
   a.brows_per_e = 2 * c.f;
+  if (y_zero) {  // T * d fp32, d % 256 == 0: whole 16-byte units
+    a.zero = reinterpret_cast<uint4*>(y_zero);
+    a.zero_n16 = (long long)c.T * c.d / 4;
+  }
   return launch_wide<EPI_SWIGLU>(tm_x, tm_w, tm_a, a, st);
 }
 

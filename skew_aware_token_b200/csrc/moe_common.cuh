@@ -119,10 +119,11 @@ cudaError_t launch_ffn(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
 // FC1 + SwiGLU on whole 256-row tiles (ffn_wide.cu): the two-launch FFN's FC1 unless the
 // mode asks for SM pairs, rows gathered from x, Z kept for the backward, or 128-row halves
 bool fc1_wide_supported(int mode);
+// y_zero: y (T x d fp32) for the kernel to zero beside FC1's work, or null
 cudaError_t launch_fc1_wide(const moe_cfg& c, const uint16_t* xp, const uint16_t* w1,
                             const int32_t* tiles, const int32_t* plan_info, uint16_t* a_out,
                             int32_t* sched, int32_t* status, bool strict, int32_t* slot_rec,
-                            cudaStream_t st);
+                            float* y_zero, cudaStream_t st);
 // FC2 on whole 256-row tiles: the two-launch FFN's FC2 with O rows (unless on SM pairs), and
 // with the fused combine when the mode asks for MOE_FFN_FC2_WHOLE
 bool fc2_wide_supported(int mode);

@@ -14,10 +14,22 @@ import torch
 from . import native as N
 
 
+# y larger than this (about twice L2) makes the fused combine's fp32 reductions DRAM-bound;
+# above it a fused-combine call runs FC2 with O rows plus the ordered combine instead (about
+# 4 % faster FFN on the DeepSeek-V3-shaped layer, y = 470 MB; slower on the 134 MB y of the
+# 16384-token Qwen3-shaped layers)
+O_ROWS_MIN_Y_BYTES = 256 << 20
+
+
 class MoeLayer:
     def __init__(self, wl, device="cuda", write_o: bool = False, guard: int = 0,
-                 gather_x: bool = False, train: bool = False):
+                 gather_x: bool = False, train: bool = False, o_rows: bool | None = None):
         """`guard` adds that many spare elements after every buffer (canary checks).
+        `write_o`: also hold the O buffer (bf16 [R_max, d]) for MOE_FFN_WRITE_O calls.
+        `o_rows`: how a call in the fused-combine mode runs the combine: True, FC2 writes O
+        rows and moe_combine adds each token's k rows in order; False, FC2 adds into y
+        itself; None (default), O rows when y (T x d fp32) is larger than
+        O_ROWS_MIN_Y_BYTES.
         `gather_x`: FC1 gathers its rows from x by row_token (MOE_FFN_GATHER_X) and the
         dispatched copy Xp is neither allocated nor written (saves R_max * d * 2 bytes; as
         fast while x stays resident in L2, slower once it does not); False (default)
@@ -69,7 +81,8 @@ class MoeLayer:
             self.dw1 = z(max(E * 2 * f * d, 4), dt=f32)
             self.dw2 = z(max(E * d * f, 4), dt=f32)
         self.y = z(max(T * d, 4), dt=f32)
-        self.o = z(max(R * d, 8), dt=torch.bfloat16) if write_o else None
+        self.o_rows = (T * d * 4 > O_ROWS_MIN_Y_BYTES) if o_rows is None else bool(o_rows)
+        self.o = z(max(R * d, 8), dt=torch.bfloat16) if (write_o or self.o_rows) else None
         self.device = dev
         self._side = torch.cuda.Stream(dev) if dev.type == "cuda" else None
 
@@ -97,6 +110,11 @@ class MoeLayer:
                                self.xp, self.row_token, self.row_gate, self.tok_row,
                                self.status, stream)
 
+    def ffn_mode(self, mode=N.MOE_FFN_FUSED_COMBINE) -> int:
+        """The mode a layer call runs the FFN in: with o_rows, MOE_FFN_WRITE_O is added to a
+        fused-combine mode (the layer then runs moe_combine after the FFN)."""
+        return mode | N.MOE_FFN_WRITE_O if self.o_rows else mode
+
     def ffn(self, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, stream=None, y=None, x=None):
         """The expert FFN; `x` (the token rows) is needed when the layer gathers them."""
         out = self.o if mode & N.MOE_FFN_WRITE_O else (self.y if y is None else y)
@@ -123,6 +141,7 @@ class MoeLayer:
                  stream=None, y=None):
         """Route, plan, dispatch, FFN (+ combine): returns y fp32 [T, d], by default a view
         of the layer's buffer (valid until the next call), or the caller's `y`."""
+        mode = self.ffn_mode(mode)
         self.pre_ffn(logits, x, variant_mask, stream)
         self.ffn(w1, w2, mode, stream, y, x)
         if mode & N.MOE_FFN_WRITE_O:

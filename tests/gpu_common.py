@@ -47,7 +47,8 @@ def expected_tiles(q, block_off, beta):
 
 def run_gpu(wl, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, variant_mask=0, layer=None):
     logits, x = host_inputs(wl)
-    layer = layer or MoeLayer(wl, "cuda", write_o=bool(mode & N.MOE_FFN_WRITE_O))
+    # the test's mode runs as given (no switch to O rows for a large y)
+    layer = layer or MoeLayer(wl, "cuda", write_o=bool(mode & N.MOE_FFN_WRITE_O), o_rows=False)
     layer.clear_status()
     layer(logits.cuda(), x.cuda(), w1, w2, mode=mode, variant_mask=variant_mask)
     torch.cuda.synchronize()

@@ -184,3 +184,15 @@ def test_one_launch_rejects_unsupported_combinations():
         mode = N.MOE_FFN_ONE_LAUNCH | other
         assert lib.moe_expert_ffn_noalloc(cfg, *[ok] * 7, mode, *[ok] * 2,
                                           None) == N.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(not NO_GPU, reason="fake pointers are only passed where no GPU exists")
+def test_noalloc_refuses_modes_its_fixed_array_cannot_serve():
+    """MOE_FFN_SAVE_Z (Z belongs in the caller's scratch) and MOE_FFN_RECORD_SLOTS (the
+    record could not be read back) are refused before any CUDA call."""
+    cfg = ctypes.byref(N.MoeCfg.of(WORKLOADS["tiny"]))
+    ok = 1 << 20
+    lib = N.lib()
+    for flag in (N.MOE_FFN_SAVE_Z, N.MOE_FFN_RECORD_SLOTS):
+        assert lib.moe_expert_ffn_noalloc(cfg, *[ok] * 7, flag, ok, ok, None) == \
+            N.MOE_ERR_INVALID_ARG

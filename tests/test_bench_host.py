@@ -80,11 +80,12 @@ def test_roofline_fraction_is_algorithmic_flops_over_time():
 
 
 def test_launch_count_per_step():
-    wl = WORKLOADS["dsv3_a1"]
-    assert bench.gpu_launches_per_step(wl, 0, 148) == 8
-    assert bench.gpu_launches_per_step(wl, N.MOE_FFN_WRITE_O, 148) == 9
-    assert bench.gpu_launches_per_step(wl, N.MOE_FFN_GATHER_X, 148) == 7
-    assert bench.gpu_launches_per_step(WORKLOADS["tiny"], 0, 148) == 7  # one FFN launch
+    wl = WORKLOADS["dsv3_a1"]  # 131072 pairs: the dispatch's count and prefix kernels run
+    assert bench.gpu_launches_per_step(wl, 0, 148) == 10
+    assert bench.gpu_launches_per_step(wl, N.MOE_FFN_WRITE_O, 148) == 11
+    assert bench.gpu_launches_per_step(wl, N.MOE_FFN_GATHER_X, 148) == 9
+    # 512 pairs (one dispatch chunk), one FFN launch
+    assert bench.gpu_launches_per_step(WORKLOADS["tiny"], 0, 148) == 7
 
 
 def test_oracle_sample_fits_its_memory_bound():
@@ -96,3 +97,27 @@ def test_oracle_sample_fits_its_memory_bound():
     assert len(experts) * 3 * wl.d * wl.f * 4 <= 4e9
     # the next doubling would not fit
     assert len(bench.sample_experts(wl, logits, 2 * n)) * 3 * wl.d * wl.f * 4 > 4e9
+
+
+def test_layer_runs_large_y_with_o_rows(monkeypatch):
+    """A fused-combine call of a layer whose y exceeds the threshold runs FC2 with O rows and
+    the ordered combine; explicit choices win; the O buffer exists whenever it is used."""
+    from skew_aware_token_b200 import layer as L
+    wl = WORKLOADS["tiny"]
+    y_bytes = wl.T * wl.d * 4
+    monkeypatch.setattr(L, "O_ROWS_MIN_Y_BYTES", y_bytes - 1)
+    big = L.MoeLayer(wl, "cpu")
+    assert big.o_rows and big.o is not None
+    assert big.ffn_mode(0) == N.MOE_FFN_WRITE_O
+    assert big.ffn_mode(N.MOE_FFN_STRICT_SLOTS) == N.MOE_FFN_STRICT_SLOTS | N.MOE_FFN_WRITE_O
+    monkeypatch.setattr(L, "O_ROWS_MIN_Y_BYTES", y_bytes)
+    small = L.MoeLayer(wl, "cpu")
+    assert not small.o_rows and small.o is None and small.ffn_mode(0) == 0
+    assert L.MoeLayer(wl, "cpu", o_rows=True).o_rows
+    assert not L.MoeLayer(wl, "cpu", o_rows=False, write_o=True).o_rows
+
+
+def test_o_rows_threshold_splits_the_workloads():
+    from skew_aware_token_b200 import layer as L
+    big = {n for n, wl in WORKLOADS.items() if wl.T * wl.d * 4 > L.O_ROWS_MIN_Y_BYTES}
+    assert big == {"dsv3_a1"}

@@ -2,16 +2,18 @@
 allocate device memory: a plugin or custom operator that its host framework hands only
 inputs and outputs, or a deployment that forbids cudaMalloc after start-up.
 
-Through the C ABI it must give what moe_expert_ffn gives (with the caller's scratch) on
-two calls in a row (the library's array keeps the previous call's contents), within the
-parity tolerance 1e-2 + 2e-2|ref|, and refuse a problem whose FC1 output does not fit its
-fixed array.  This file is collected last and runs the same alone or after the others."""
+Through the C ABI it must give what moe_expert_ffn gives (with the caller's scratch), and
+what the CPU oracle gives, on two calls in a row (the library's array keeps the previous
+call's contents), within the parity tolerance 1e-2 + 2e-2|ref|, and refuse a problem whose
+FC1 output does not fit its fixed array.  This file is collected last and runs the same
+alone or after the others."""
 import ctypes
 
 import numpy as np
 import pytest
 import torch
 
+from oracle import moe_oracle as O
 from skew_aware_token_b200 import native as N
 from skew_aware_token_b200 import synth
 from skew_aware_token_b200.layer import MoeLayer
@@ -45,6 +47,9 @@ def test_noalloc_matches_scratch_entry_point_twice(wl, mode):
     layer.ffn(w1, w2, mode)                         # caller-provided scratch
     torch.cuda.synchronize()
     ref = out.clone()
+    W1, W2 = w1.float().cpu().numpy(), w2.float().cpu().numpy()
+    oracle = O.moe_forward(synth.make_logits(wl).numpy(), synth.make_x(wl).float().numpy(),
+                           lambda e: (W1[e], W2[e]), k=wl.k, beta=wl.beta, P=wl.P, s=wl.s)
     for call in range(2):
         out.fill_(float("nan"))
         N.moe_expert_ffn_noalloc(layer.cfg, layer.xp, w1, w2, layer.tiles, layer.plan_info,
@@ -56,10 +61,13 @@ def test_noalloc_matches_scratch_entry_point_twice(wl, mode):
             rows = layer.row_token[:R] >= 0
             got = out[: R * wl.d].view(R, wl.d)[rows]
             want = ref[: R * wl.d].view(R, wl.d)[rows]
+            want_oracle = torch.from_numpy(oracle["O"][rows.cpu().numpy()])
         else:
             got = out[: wl.T * wl.d]
             want = ref[: wl.T * wl.d]
-        assert _within(got, want), f"call {call}"
+            want_oracle = torch.from_numpy(oracle["y"]).reshape(-1)
+        assert _within(got, want), f"call {call}: against moe_expert_ffn"
+        assert _within(got, want_oracle), f"call {call}: against the oracle"
 
 
 def test_noalloc_refuses_a_problem_larger_than_its_array():
