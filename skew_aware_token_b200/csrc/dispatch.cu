@@ -69,14 +69,20 @@ dispatch_count_kernel(const int32_t* __restrict__ ids, int N, int E, int C,
 }
 
 __global__ void dispatch_prefix_kernel(int32_t* __restrict__ table, int E, int C) {
+  constexpr int kBatch = 8;  // chunk counts loaded ahead of the running sum
   const int e = threadIdx.x;
   if (e >= E) return;
   int run = 0;
-  for (int c = 0; c < C; ++c) {
-    int32_t* p = table + (long long)c * kChunk + e;
-    const int v = *p;
-    *p = run;
-    run += v;
+  for (int c0 = 0; c0 < C; c0 += kBatch) {
+    int v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      v[u] = c0 + u < C ? table[(long long)(c0 + u) * kChunk + e] : 0;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (c0 + u < C) table[(long long)(c0 + u) * kChunk + e] = run;
+      run += v[u];
+    }
   }
 }
 
@@ -155,9 +161,10 @@ dispatch_rank_kernel(const int32_t* __restrict__ ids, const float* __restrict__ 
     __syncthreads();  // hist is rewritten by the next pass
   }
   if (c == C - 1) {
-    // every expert's total is now known: mark its padding rows
-    for (int e = 0; e < E; ++e) {
-      for (long long r = run[e] + threadIdx.x; r < cap[e]; r += blockDim.x) {
+    // every expert's total is now known: one thread per expert marks its padding rows
+    // (fewer than beta of them unless the counts and blocks disagree)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      for (long long r = run[e]; r < cap[e]; ++r) {
         row_token[base[e] + r] = -1;
         row_gate[base[e] + r] = 0.f;
       }

@@ -89,6 +89,12 @@ def _build_workloads() -> dict[str, Workload]:
         w.append(_sweep("all4", 1.0, beta, alpha=1.5))
     w.append(Workload("dsv3_a1", T=16384, d=7168, E=256, k=8, f=2048, beta=128, P=8, s=4,
                       alpha=1.0))
+    # the DeepSeek-V3-shaped layer with 32 experts (2.8 GB of weights): small enough for
+    # profilers that replay a kernel many times; at T = 2048 an expert averages 512 rows,
+    # as in the full layer
+    for T in (2048, 8192):
+        w.append(Workload(f"dsv3_e32_t{T}", T=T, d=7168, E=32, k=8, f=2048, beta=128, P=8,
+                          s=4, alpha=1.0))
     return {x.name: x for x in w}
 
 
