@@ -545,7 +545,7 @@ def run_stage_bandwidth(layer, wl, logits, x, w1, w2, dev, flush, peaks, reps=10
 
 
 FFN_SOURCES = ("skew_aware_token_b200/csrc/ffn_tcgen05.cu", "skew_aware_token_b200/csrc/ffn_wide.cu",
-               "skew_aware_token_b200/csrc/tc_util.cuh")
+               "skew_aware_token_b200/csrc/tc_util.cuh", "skew_aware_token_b200/csrc/combine.cu")
 
 
 def ffn_source_digest() -> str:

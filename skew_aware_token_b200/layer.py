@@ -14,11 +14,14 @@ import torch
 from . import native as N
 
 
-# y larger than this (about twice L2) makes the fused combine's fp32 reductions DRAM-bound;
-# above it a fused-combine call runs FC2 with O rows plus the ordered combine instead (about
-# 4 % faster FFN on the DeepSeek-V3-shaped layer, y = 470 MB; slower on the 134 MB y of the
-# 16384-token Qwen3-shaped layers)
-O_ROWS_MIN_Y_BYTES = 256 << 20
+# From this size of y on, a fused-combine call of the layer runs FC2 with O rows plus the
+# ordered combine instead: the fused combine's fp32 reductions compete with the operand
+# copies for L2 (and go to DRAM once y outgrows it), while O rows leave through TMA stores
+# and the combine reads them once.  Measured FFN times: DeepSeek-V3-shaped layer (470 MB y)
+# 2 % faster, 8192-token Qwen3-shaped layer (64 MiB y) 6 % faster, 16384-token layers
+# (134 MB y) within 0.5 %, 4096-token layer (32 MiB y) even.  The ordered combine also
+# makes y independent of the reduction order.
+O_ROWS_MIN_Y_BYTES = 64 << 20
 
 
 class MoeLayer:
@@ -28,7 +31,7 @@ class MoeLayer:
         `write_o`: also hold the O buffer (bf16 [R_max, d]) for MOE_FFN_WRITE_O calls.
         `o_rows`: how a call in the fused-combine mode runs the combine: True, FC2 writes O
         rows and moe_combine adds each token's k rows in order; False, FC2 adds into y
-        itself; None (default), O rows when y (T x d fp32) is larger than
+        itself; None (default), O rows when y (T x d fp32) holds at least
         O_ROWS_MIN_Y_BYTES.
         `gather_x`: FC1 gathers its rows from x by row_token (MOE_FFN_GATHER_X) and the
         dispatched copy Xp is neither allocated nor written (saves R_max * d * 2 bytes; as
@@ -81,7 +84,7 @@ class MoeLayer:
             self.dw1 = z(max(E * 2 * f * d, 4), dt=f32)
             self.dw2 = z(max(E * d * f, 4), dt=f32)
         self.y = z(max(T * d, 4), dt=f32)
-        self.o_rows = (T * d * 4 > O_ROWS_MIN_Y_BYTES) if o_rows is None else bool(o_rows)
+        self.o_rows = (T * d * 4 >= O_ROWS_MIN_Y_BYTES) if o_rows is None else bool(o_rows)
         self.o = z(max(R * d, 8), dt=torch.bfloat16) if (write_o or self.o_rows) else None
         self.device = dev
         self._side = torch.cuda.Stream(dev) if dev.type == "cuda" else None

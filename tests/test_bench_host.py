@@ -105,12 +105,12 @@ def test_layer_runs_large_y_with_o_rows(monkeypatch):
     from skew_aware_token_b200 import layer as L
     wl = WORKLOADS["tiny"]
     y_bytes = wl.T * wl.d * 4
-    monkeypatch.setattr(L, "O_ROWS_MIN_Y_BYTES", y_bytes - 1)
+    monkeypatch.setattr(L, "O_ROWS_MIN_Y_BYTES", y_bytes)
     big = L.MoeLayer(wl, "cpu")
     assert big.o_rows and big.o is not None
     assert big.ffn_mode(0) == N.MOE_FFN_WRITE_O
     assert big.ffn_mode(N.MOE_FFN_STRICT_SLOTS) == N.MOE_FFN_STRICT_SLOTS | N.MOE_FFN_WRITE_O
-    monkeypatch.setattr(L, "O_ROWS_MIN_Y_BYTES", y_bytes)
+    monkeypatch.setattr(L, "O_ROWS_MIN_Y_BYTES", y_bytes + 1)
     small = L.MoeLayer(wl, "cpu")
     assert not small.o_rows and small.o is None and small.ffn_mode(0) == 0
     assert L.MoeLayer(wl, "cpu", o_rows=True).o_rows
@@ -118,6 +118,8 @@ def test_layer_runs_large_y_with_o_rows(monkeypatch):
 
 
 def test_o_rows_threshold_splits_the_workloads():
+    """O rows from the 8192-token layers on (64 MiB of y), fused below."""
     from skew_aware_token_b200 import layer as L
-    big = {n for n, wl in WORKLOADS.items() if wl.T * wl.d * 4 > L.O_ROWS_MIN_Y_BYTES}
-    assert big == {"dsv3_a1"}
+    for name, wl in WORKLOADS.items():
+        big = wl.T * wl.d * 4 >= L.O_ROWS_MIN_Y_BYTES
+        assert big == (wl.T >= 8192), name
