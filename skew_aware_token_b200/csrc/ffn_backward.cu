@@ -1,4 +1,7 @@
-// Backward of the grouped SwiGLU expert FFN on the sm_100a tensor cores.
+// Backward of the grouped SwiGLU expert FFN on the sm_100a tensor cores: the dispatch of the
+// output gradient, and the four gradient products on 128-row tile halves.  Each product runs
+// on the whole-tile kernels of ffn_bwd_wide.cu instead where its shape allows (all four when
+// f is a multiple of 256); the kernels here remain for the other shapes.
 //
 // "MegaFlux" summary, Methodology 2, backward gradients, with this library's weight layouts
 // w1 [E, 2f, d] and w2 [E, d, f] (each of the pages' products is taken with that transpose):
@@ -82,13 +85,6 @@ struct BwdArgs {
   unsigned long long timeout_ns;
 };
 
-// Shared-memory descriptor of an MN-major tile copied by 64-element x 64-row boxes with the
-// 128-byte swizzle: start >> 4, leading offset 8192 >> 4 (between 64-element MN chunks),
-// stride offset 1024 >> 4 (between 8-row K groups), version 1, swizzle mode 2.
-__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(8192 >> 4) << 16) |
-         ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
-}
 
 struct BItem {
   bool run;    // work to do (a DGrad half with rows, or any WGrad item)
@@ -583,6 +579,8 @@ cudaError_t launch_ffn_backward(const moe_cfg& c, const uint16_t* xp, const uint
   base.beta = c.beta;
   base.timeout_ns = kWaitNs;
 
+  // Each product runs on whole 256-row tiles where its shape allows (ffn_bwd_wide.cu), else
+  // on the 128-row tile halves below.
   // dA = D w2 (N = f in tiles of 256, or 128, K = d) with the SwiGLU backward -> dZ
   BwdArgs g1 = base;
   g1.sched = sched + 0;
@@ -590,7 +588,10 @@ cudaError_t launch_ffn_backward(const moe_cfg& c, const uint16_t* xp, const uint
   g1.dz = dz;
   g1.n_k = c.d / kBK;
   g1.k_rows = c.d;
-  if (c.f % 256 == 0) {
+  if (bwd_wide_supported(c, BWD_DGRAD_A)) {
+    err = launch_bwd_wide(c, BWD_DGRAD_A, d_rows, w2, dz, tiles, plan_info, block_off,
+                          row_token, z_saved, sched + 0, status, st);
+  } else if (c.f % 256 == 0) {
     g1.n_n = c.f / 256;
     err = launch_bwd<DGRAD_A, 256>(m_d_k, m_w2, g1, st);
   } else {
@@ -605,7 +606,10 @@ cudaError_t launch_ffn_backward(const moe_cfg& c, const uint16_t* xp, const uint
   g2.n_k = 2 * c.f / kBK;
   g2.n_n = c.d / 256;
   g2.k_rows = 2 * c.f;
-  err = launch_bwd<DGRAD_X, 256>(m_dz_k, m_w1, g2, st);
+  err = bwd_wide_supported(c, BWD_DGRAD_X)
+            ? launch_bwd_wide(c, BWD_DGRAD_X, dz, w1, dx, tiles, plan_info, block_off,
+                              row_token, nullptr, sched + 1, status, st)
+            : launch_bwd<DGRAD_X, 256>(m_dz_k, m_w1, g2, st);
   if (err != cudaSuccess) return err;
   // dW2_e [d, f] = D^T A (M = d, N = f, K = the expert's rows)
   BwdArgs g3 = base;
@@ -613,7 +617,10 @@ cudaError_t launch_ffn_backward(const moe_cfg& c, const uint16_t* xp, const uint
   g3.dw = dw2;
   g3.n_m = c.d / kBM;
   g3.n_out = c.f;
-  if (c.f % 256 == 0) {
+  if (bwd_wide_supported(c, BWD_WGRAD_2)) {
+    err = launch_bwd_wide(c, BWD_WGRAD_2, d_rows, a_saved, dw2, tiles, plan_info, block_off,
+                          row_token, nullptr, sched + 2, status, st);
+  } else if (c.f % 256 == 0) {
     g3.n_n = c.f / 256;
     err = launch_bwd<WGRAD_2, 256>(m_d_mn, m_a_mn, g3, st);
   } else {
@@ -628,7 +635,10 @@ cudaError_t launch_ffn_backward(const moe_cfg& c, const uint16_t* xp, const uint
   g4.n_m = 2 * c.f / kBM;
   g4.n_n = c.d / 256;
   g4.n_out = c.d;
-  return launch_bwd<WGRAD_1, 256>(m_dz_mn, m_xp_mn, g4, st);
+  return bwd_wide_supported(c, BWD_WGRAD_1)
+             ? launch_bwd_wide(c, BWD_WGRAD_1, dz, xp, dw1, tiles, plan_info, block_off,
+                               row_token, nullptr, sched + 3, status, st)
+             : launch_bwd<WGRAD_1, 256>(m_dz_mn, m_xp_mn, g4, st);
 }
 
 }  // namespace moe

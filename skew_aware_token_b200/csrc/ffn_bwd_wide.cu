@@ -1,0 +1,770 @@
+// Backward of the grouped SwiGLU expert FFN on whole 256-row tiles (tcgen05 + TMEM, fed by
+// TMA): the four gradient products of moe_expert_ffn_backward with the forward whole-tile
+// kernels' structure.
+//
+// "MegaFlux" summary, Methodology 2, backward gradients, with the weight layouts w1 [E, 2f, d]
+// and w2 [E, d, f]:
+//   dA  = D w2_e; dZ = [dA U SiLU'(G), dA SiLU(G)]   kind DGRAD_A  (M = rows, N = f, K = d)
+//   dX  = dZ w1_e; dx[row_token] += dX              kind DGRAD_X  (M = rows, N = d, K = 2f)
+//   dW2_e = D^T A                                   kind WGRAD_2  (M = d, N = f, K = rows of e)
+//   dW1_e = dZ^T Xp                                 kind WGRAD_1  (M = 2f, N = d, K = rows of e)
+// An item is 256 rows of the output (two M = 128 MMAs that share each B stage: 64 bytes of
+// copies per tensor-core clock, where the 128-row tile-half kernels need 96) times 256
+// columns.  The two 128 x 256 fp32 accumulators fill the 512 TMEM columns; the epilogue frees
+// them half by half, and the next item's second-half MMAs may lag its first-half MMAs by up to
+// the three pipeline stages, as in the forward.
+//
+// Operands.  K-major A (D and dZ rows for the DGrad kinds): per 128-row half one box of 64 K
+// (128 bytes) x 128 rows, 128-byte swizzle.  MN-major operands (the weights as B of the DGrad
+// kinds; both operands of the WGrad kinds, whose K is the expert's token rows): boxes of 64
+// MN elements (128 bytes) x 64 K rows, 8 KB apart; their descriptors give 8 KB between the
+// 64-element MN chunks and 1 KB between 8-row K groups, a K step of 16 advances 2 KB.
+//
+// Epilogues.  The warps that read TMEM keep global stores out of their way (pending stores
+// hold up a warp's next TMEM load): results go through a 32 KB shared staging buffer, in
+// 32-row x 128-byte boxes with the 128-byte swizzle, and a store warp writes the boxes with
+// TMA stores.
+//   DGRAD_A  per round 64 columns of dA: the warp loads the matching G and U of its row
+//            (bf16, saved by the forward) before reading TMEM, computes dG and dU, rounds
+//            them to bf16, and stages one box of dG and one of dU; the store warp writes
+//            them to dZ's G and U column ranges.
+//   DGRAD_X  dx[token] += dX with 16-byte vector reductions, each warp transposing 32 x 32
+//            chunks through its own 4 KB slot (as the forward's fused combine, gate 1: the
+//            gate is already in D).
+//   WGRAD    dW fp32: per round 64 columns (two 32-column fp32 boxes per row group).  An idle
+//            expert's items issue no MMA and stage zeros.
+// Roles (352 threads, one CTA per SM, persistent): warp 0 TMA producer, warp 1 MMA issuer,
+// warps 2..9 epilogue (warp w reads TMEM lanes 32 (w % 4) .. +31, and half of each round's
+// columns), warp 10 store warp (idle for DGRAD_X).  Items come from a global counter in
+// increasing order through a ring in shared memory; every wait is bounded.
+#include "tc_util.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BW_M = 256;   // output rows per item
+constexpr int BW_H = 128;   // rows per MMA (TMEM lanes)
+constexpr int BW_K = 64;    // K per stage
+constexpr int BW_N = 256;   // MMA N
+constexpr int BW_ST = 3;    // pipeline stages (DGRAD_A: 2, for a second staging buffer)
+constexpr int BW_A_BYTES = BW_M * BW_K * 2;
+constexpr int BW_B_BYTES = BW_N * BW_K * 2;
+constexpr int BW_STAGE = BW_A_BYTES + BW_B_BYTES;
+constexpr int BW_HALF_A = BW_H * BW_K * 2;
+constexpr int BW_STG_BYTES = 32768;
+constexpr int BW_RING = 8;
+constexpr int BW_EPI_WARPS = 8;
+constexpr int BW_THREADS = 32 * (3 + BW_EPI_WARPS);
+constexpr int BW_STORE_WARP = 2 + BW_EPI_WARPS;
+constexpr int BW_NBARS = 2 * BW_ST + 8 + 2 * BW_RING;
+constexpr int BW_META = 512;
+constexpr int BW_SMEM = BW_ST * BW_STAGE + BW_STG_BYTES + BW_META + 1024;
+static_assert(2 * BW_STAGE + 2 * BW_STG_BYTES <= BW_ST * BW_STAGE + BW_STG_BYTES, "DGRAD_A smem");
+constexpr int BW_RPH = 4;  // store rounds of 64 columns per accumulator half
+static_assert(BW_NBARS * 8 + 4 * (2 + BW_RING) <= BW_META, "meta");
+static_assert(BW_SMEM <= 227 * 1024, "smem");
+
+template <int KIND>
+struct BwGeo {
+  static constexpr bool DGRAD = KIND == BWD_DGRAD_A || KIND == BWD_DGRAD_X;
+  static constexpr bool A_MN = !DGRAD;                // WGrad: both operands MN-major
+  static constexpr bool STORES = KIND != BWD_DGRAD_X;  // the store warp takes items
+  static constexpr int ST = KIND == BWD_DGRAD_A ? 2 : BW_ST;  // pipeline stages
+  static constexpr int NSTG = KIND == BWD_DGRAD_A ? 2 : 1;    // 32 KB staging buffers
+  // kind::f16: D fp32, A and B bf16, A / B major bits, N >> 3 at bit 17, M >> 4 at bit 24
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
+                                    ((A_MN ? 1u : 0u) << 15) | (1u << 16) |
+                                    ((uint32_t)(BW_N >> 3) << 17) |
+                                    ((uint32_t)(BW_H >> 4) << 24);
+};
+
+struct BwArgs {
+  int32_t* sched;            // this launch's work counter (zeroed by the host)
+  const int32_t* tiles;      // DGrad: planner tiles (e, row0, nrows, slot)
+  const int32_t* plan_info;  // DGrad: number of tiles
+  const int32_t* block_off;  // WGrad: the expert's rows
+  const int32_t* row_token;  // DGRAD_X
+  const uint16_t* z;         // DGRAD_A: saved Z = [G, U] bf16 [r_max, 2f]
+  float* dx;                 // DGRAD_X: dx fp32 [T, d], zeroed by the host
+  int32_t* status;
+  long long r_max;
+  int T, d, f, E, beta;
+  int n_k;     // DGrad: K steps of 64
+  int n_n;     // n-tiles of 256 columns
+  int n_m;     // WGrad: m-tiles of 256 rows per expert
+  int k_rows;  // DGrad: first B row of expert e is e * k_rows (d for w2, 2f for w1)
+  int m_rows;  // WGrad: rows of one expert's gradient (d for dW2, 2f for dW1)
+  unsigned long long timeout_ns;
+};
+
+struct BwItem {
+  bool ok;    // a well-formed item
+  bool zero;  // WGrad item of an idle expert: no K, a zero output tile
+  bool two;   // two 128-row halves (always for WGrad)
+  int e, row0, nrows, nk, m0, n0;
+};
+
+template <int KIND>
+__device__ __forceinline__ BwItem bw_item(const BwArgs& a, int L) {
+  BwItem it;
+  if constexpr (BwGeo<KIND>::DGRAD) {
+    // (planner tile, n-tile), the n-tiles of a tile together
+    const int m = L / a.n_n;
+    it.n0 = (L - m * a.n_n) * BW_N;
+    const int4 v = __ldg(reinterpret_cast<const int4*>(a.tiles) + m);
+    it.e = v.x;
+    it.row0 = v.y;
+    it.nrows = v.z;
+    // tiles hold whole 64-row blocks; a 32-row store box is then all in the tile or all out
+    it.ok = v.x >= 0 && v.x < a.E && v.y >= 0 && v.z > 0 && v.z <= BW_M && (v.z & 31) == 0 &&
+            (long long)v.y + v.z <= a.r_max;
+    it.two = v.z > BW_H;
+    it.nk = a.n_k;
+    it.m0 = 0;
+    it.zero = false;
+  } else {
+    // (expert, m-tile, n-tile), an expert's items together
+    const int per_e = a.n_m * a.n_n;
+    it.e = L / per_e;
+    const int r = L - it.e * per_e;
+    const int mt = r / a.n_n;
+    it.m0 = mt * BW_M;
+    it.n0 = (r - mt * a.n_n) * BW_N;
+    const int b0 = __ldg(a.block_off + it.e), b1 = __ldg(a.block_off + it.e + 1);
+    it.row0 = a.beta * b0;
+    it.nrows = a.beta * (b1 - b0);
+    it.ok = b0 >= 0 && b1 >= b0 && (long long)a.beta * b1 <= a.r_max;
+    it.nk = it.ok ? it.nrows / BW_K : 0;
+    it.zero = it.nk == 0;
+    it.two = true;
+  }
+  return it;
+}
+
+// 16-byte chunk c of row r of a 128-byte-row box, 128-byte swizzle
+__device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t v) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(BW_THREADS, 1)
+bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmZ,
+               const BwArgs a) {
+  using G = BwGeo<KIND>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  constexpr int ST = G::ST;
+  uint8_t* stg = smem + ST * BW_STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + G::NSTG * BW_STG_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + BW_NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + BW_ST + s); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * BW_ST);
+  const uint32_t tfull_bar = smem_u32(bars + 2 * BW_ST + 1);
+  // tfree[h]: the epilogue has read accumulator half h (TMEM columns [256 h, +256))
+  auto tfree_bar = [&](int h) { return smem_u32(bars + 2 * BW_ST + 2 + h); };
+  const uint32_t staged_bar = smem_u32(bars + 2 * BW_ST + 4);
+  const uint32_t stgfree_bar = smem_u32(bars + 2 * BW_ST + 5);
+  // DGRAD_A, staging buffer b: zfull[b] its G and U copies have landed, dstaged[b] the
+  // epilogue has written its results
+  auto zfull_bar = [&](int b) { return b ? smem_u32(bars + 2 * BW_ST + 6) : stgfree_bar; };
+  auto dstaged_bar = [&](int b) { return b ? smem_u32(bars + 2 * BW_ST + 7) : staged_bar; };
+  auto ifull_bar = [&](int i) { return smem_u32(bars + 2 * BW_ST + 8 + i); };
+  auto iempty_bar = [&](int i) { return smem_u32(bars + 2 * BW_ST + 8 + BW_RING + i); };
+  auto sA = [&](int s) { return smem_u32(smem + s * BW_STAGE); };
+  auto sB = [&](int s) { return smem_u32(smem + s * BW_STAGE + BW_A_BYTES); };
+
+  long long total;
+  if constexpr (G::DGRAD)
+    total = (long long)max(a.plan_info[MOE_PI_NTILES], 0) * a.n_n;
+  else
+    total = (long long)a.E * a.n_m * a.n_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(drain_bar, 1);
+    mbar_init(tfull_bar, 1);
+    mbar_init(tfree_bar(0), BW_EPI_WARPS);
+    mbar_init(tfree_bar(1), BW_EPI_WARPS);
+    mbar_init(staged_bar, BW_EPI_WARPS);
+    mbar_init(stgfree_bar, 1);
+    mbar_init(dstaged_bar(1), BW_EPI_WARPS);
+    mbar_init(zfull_bar(1), 1);
+    for (int i = 0; i < BW_RING; ++i) {
+      mbar_init(ifull_bar(i), 1);
+      // MMA thread, epilogue warps (and the store thread)
+      mbar_init(iempty_bar(i), 1 + BW_EPI_WARPS + (G::STORES ? 1 : 0));
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    if (G::STORES) prefetch_tmap(&tmO);
+    if (KIND == BWD_DGRAD_A) prefetch_tmap(&tmZ);
+  }
+  if (warp == 1) tmem_alloc<false, 512>(smem_u32(tmem_slot));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // consumers: the item of ring position `it`, -1 when the work is done, -2 when the wait
+  // gave up
+  auto take_item = [&](int it) -> int {
+    const int slot = it % BW_RING;
+    if (!mbar_wait(ifull_bar(slot), (uint32_t)(it / BW_RING) & 1u, abort_flag, a.status,
+                   a.timeout_ns, true))
+      return -2;
+    return ring[slot];
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, pending = 0, pend_parity = 0;
+      bool bad = false;
+      for (int it = 0;; ++it) {
+        const int slot = it % BW_RING;
+        if (!mbar_wait(iempty_bar(slot), ((uint32_t)(it / BW_RING) & 1u) ^ 1u, abort_flag,
+                       a.status, a.timeout_ns, true))
+          break;
+        const long long v = atomicAdd(a.sched, 1);
+        const int L = v < total ? (int)v : -1;
+        ring[slot] = L;
+        mbar_arrive(ifull_bar(slot));
+        if (L < 0) break;
+        const BwItem w = bw_item<KIND>(a, L);
+        if (!w.ok) {
+          bad = true;
+          continue;
+        }
+        if (w.zero) continue;
+        if constexpr (KIND == BWD_DGRAD_A) {
+          // the epilogue reads the item's G and U columns (256 rows x 256 each): bring them
+          // into L2 while the item's MMAs run
+          for (int r0 = 0; r0 < w.nrows; r0 += 32)
+            for (int c = 0; c < BW_N / 64; ++c) {
+              tma_prefetch_l2_2d(&tmZ, w.n0 + 64 * c, w.row0 + r0);
+              tma_prefetch_l2_2d(&tmZ, a.f + w.n0 + 64 * c, w.row0 + r0);
+            }
+        }
+        const uint32_t tx = G::DGRAD ? (w.two ? 2 : 1) * BW_HALF_A + BW_B_BYTES : BW_STAGE;
+        bool stop = false;
+        for (int kb = 0; kb < w.nk; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status, a.timeout_ns,
+                         true)) {
+            stop = true;
+            break;
+          }
+          mbar_expect_tx(full_bar(stage), tx);
+          // B: 256 MN-major columns of the K rows (DGrad: the expert's weight rows; WGrad:
+          // its token rows)
+          const int krow = G::DGRAD ? w.e * a.k_rows + kb * BW_K : w.row0 + kb * BW_K;
+#pragma unroll
+          for (int j = 0; j < BW_N / 64; ++j)
+            tma_load_2d(sB(stage) + j * 8192, &tmB, full_bar(stage), w.n0 + 64 * j, krow);
+          if constexpr (G::A_MN) {
+#pragma unroll
+            for (int j = 0; j < BW_M / 64; ++j)
+              tma_load_2d(sA(stage) + j * 8192, &tmA, full_bar(stage), w.m0 + 64 * j, krow);
+          } else {
+            tma_load_2d(sA(stage), &tmA, full_bar(stage), kb * BW_K, w.row0);
+            if (w.two)
+              tma_load_2d(sA(stage) + BW_HALF_A, &tmA, full_bar(stage), kb * BW_K,
+                          w.row0 + BW_H);
+          }
+          pending |= 1u << stage;
+          pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == ST) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (stop) break;
+      }
+      if (bad) set_status(a.status, MOE_STATUS_PLAN);
+      if (*abort_flag) {
+        // let the copies already armed land before shared memory goes away
+        for (int s = 0; s < ST; ++s)
+          if (pending >> s & 1u)
+            mbar_wait(full_bar(s), pend_parity >> s & 1u, abort_flag, a.status, a.timeout_ns,
+                      false);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc_it = 0;
+      bool issued = false;
+      auto a_desc = [&](uint32_t base, int h, int kk) {
+        return G::A_MN ? sw128_mn_desc(base + h * BW_HALF_A + kk * 2048)
+                       : sw128_desc(base + h * BW_HALF_A + kk * 32);
+      };
+      for (int it = 0;; ++it) {
+        const int L = take_item(it);
+        if (L == -2) break;
+        mbar_arrive(iempty_bar(it % BW_RING));
+        if (L < 0) break;
+        const BwItem w = bw_item<KIND>(a, L);
+        if (!w.ok || w.zero) continue;
+        const bool two = w.two;
+        const uint32_t par = ((uint32_t)acc_it & 1u) ^ 1u;  // the previous item's phase
+        // the previous item's first accumulator half has been read out
+        if (!mbar_wait(tfree_bar(0), par, abort_flag, a.status, a.timeout_ns, true)) break;
+        tc_fence_after();
+        // second-half MMAs may lag the first half's by up to ST stages while the
+        // epilogue still reads the previous item's second half
+        bool m1_ready = false, stop = false;
+        int pend_stage = 0, pend_kb = 0, npend = 0;
+        auto issue_m1 = [&](int st, int kb) {
+          const uint32_t a0 = sA(st), b0 = sB(st);
+#pragma unroll
+          for (int kk = 0; kk < BW_K / 16; ++kk)
+            umma_bf16<false>(tmem_base + BW_N, a_desc(a0, 1, kk), sw128_mn_desc(b0 + kk * 2048),
+                             G::IDESC, (kb | kk) != 0);
+          umma_commit_all<false>(empty_bar(st));
+        };
+        for (int kb = 0; kb < w.nk; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, a.status, a.timeout_ns, true)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = sA(stage), b0 = sB(stage);
+#pragma unroll
+          for (int kk = 0; kk < BW_K / 16; ++kk)
+            umma_bf16<false>(tmem_base, a_desc(a0, 0, kk), sw128_mn_desc(b0 + kk * 2048),
+                             G::IDESC, (kb | kk) != 0);
+          issued = true;
+          if (!two) {
+            umma_commit_all<false>(empty_bar(stage));
+          } else {
+            if (!m1_ready && mbar_try_wait(tfree_bar(1), par)) {
+              m1_ready = true;
+              tc_fence_after();
+            }
+            if (!m1_ready) {
+              if (npend == 0) {
+                pend_stage = stage;
+                pend_kb = kb;
+              }
+              ++npend;
+              if (npend == ST || kb == w.nk - 1) {
+                if (!mbar_wait(tfree_bar(1), par, abort_flag, a.status, a.timeout_ns, true)) {
+                  stop = true;
+                  break;
+                }
+                m1_ready = true;
+                tc_fence_after();
+                for (int i = 0; i < npend; ++i)
+                  issue_m1((pend_stage + i) % ST, pend_kb + i);
+                npend = 0;
+              }
+            } else {
+              for (int i = 0; i < npend; ++i) issue_m1((pend_stage + i) % ST, pend_kb + i);
+              npend = 0;
+              issue_m1(stage, kb);
+            }
+          }
+          if (++stage == ST) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (stop) break;
+        if (!two && !mbar_wait(tfree_bar(1), par, abort_flag, a.status, a.timeout_ns, true))
+          break;  // keep one phase of each half's barrier per item
+        umma_commit_all<false>(tfull_bar);
+        ++acc_it;
+      }
+      if (issued) {
+        umma_commit_local<false>(drain_bar);
+        mbar_wait(drain_bar, 0, abort_flag, a.status, a.timeout_ns, false);
+      }
+    }
+  } else if (warp < 2 + BW_EPI_WARPS) {
+    // ------------------------------------------------------------ epilogue (warps 2..9)
+    const int quarter = warp & 3;    // TMEM lanes 32 quarter .. +31 = rows of each half
+    const int ch = (warp - 2) >> 2;  // which 32 of a round's 64 columns
+    int acc_it = 0, staged_n = 0;
+    for (int it = 0;; ++it) {
+      const int L = take_item(it);
+      if (!__all_sync(0xffffffffu, L != -2)) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(iempty_bar(it % BW_RING));
+      if (L < 0) break;
+      const BwItem w = bw_item<KIND>(a, L);
+      if (!w.ok) continue;
+      const int halves = w.two ? 2 : 1;
+      if (!w.zero) {
+        const bool got = wait_inl(tfull_bar, (uint32_t)acc_it & 1u, abort_flag, a.status,
+                                  a.timeout_ns);
+        if (!__all_sync(0xffffffffu, got)) break;
+        tc_fence_after();
+      }
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      bool ok = true;
+      if constexpr (KIND == BWD_DGRAD_X) {
+        // dx[token] += dX over columns [n0 + 128 ch, +128) for this warp's 32 rows of each
+        // half.  Each 32 x 32 chunk is staged in this warp's 4 KB slot (row r's 16-byte
+        // group j at position j ^ (r & 7)); then lanes 8q..8q+7 of a vector reduction take
+        // one 128-byte row segment.
+        float* slot_f = reinterpret_cast<float*>(stg + (warp - 2) * 4096);
+#pragma unroll 1
+        for (int h = 0; h < halves; ++h) {
+          const int rit = BW_H * h + 32 * quarter + lane;  // row inside the tile
+          const long long row = (long long)w.row0 + rit;
+          int tok = -1;
+          if (rit < w.nrows && row < a.r_max) {
+            tok = __ldg(a.row_token + row);
+            if (tok >= a.T) tok = -1;
+          }
+          float* ybase = a.dx + w.n0 + 128 * ch + 4 * (lane & 7);
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            tmem_ld32(taddr + h * BW_N + 128 * ch + 32 * c, v);
+            tmem_wait_ld();
+            if (c == 3) {
+              // accumulator half h has been read (a single-half item also frees the second)
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) {
+                mbar_arrive(tfree_bar(h));
+                if (halves == 1) mbar_arrive(tfree_bar(1));
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<float4*>(slot_f + 32 * lane + 4 * (j ^ (lane & 7))) =
+                  make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                              __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int r = 4 * i + (lane >> 3);
+              const int tk = __shfl_sync(0xffffffffu, tok, r);
+              if (tk >= 0) {
+                const float4 x = *reinterpret_cast<const float4*>(
+                    slot_f + 32 * r + 4 * ((lane & 7) ^ (r & 7)));
+                red_add_v4(ybase + (long long)tk * a.d + 32 * c, x);
+              }
+            }
+            __syncwarp();
+          }
+        }
+      } else if constexpr (!G::DGRAD) {
+        // WGrad: the warp reads all 128 of its columns of a half (64 r + 32 ch .. +32 for the
+        // rounds r = 0..3) into registers and frees the half, so that the next item's MMAs
+        // restart after the TMEM reads alone; the four store rounds (32 fp32 columns each into
+        // box (quarter, ch)) then go out of registers while those MMAs run.  An idle expert's
+        // item stages zeros.
+        uint8_t* box = stg + quarter * 8192 + ch * 4096;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v[4][32];
+          if (!w.zero) {
+#pragma unroll
+            for (int r = 0; r < BW_RPH; ++r) tmem_ld32(taddr + BW_N * h + 64 * r + 32 * ch, v[r]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tfree_bar(h));
+          } else {
+#pragma unroll
+            for (int r = 0; r < BW_RPH; ++r)
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[r][i] = 0u;
+          }
+#pragma unroll
+          for (int r = 0; r < BW_RPH; ++r) {
+            // the staging buffer is free once the store warp's copies have read the last round
+            const bool fr = wait_inl(stgfree_bar, ((uint32_t)staged_n & 1u) ^ 1u, abort_flag,
+                                     a.status, a.timeout_ns);
+            if (!__all_sync(0xffffffffu, fr)) {
+              ok = false;
+              break;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              *reinterpret_cast<uint4*>(box + swz(lane, i)) =
+                  make_uint4(v[r][4 * i], v[r][4 * i + 1], v[r][4 * i + 2], v[r][4 * i + 3]);
+            fence_proxy_async();  // make the staging writes visible to the TMA engine
+            __syncwarp();
+            if (lane == 0) mbar_arrive(staged_bar);
+            ++staged_n;
+          }
+          if (!ok) break;
+        }
+      } else {
+        // DGRAD_A: per round the store warp has copied the G and U boxes of the round's 64
+        // columns into one of the two staging buffers (the same 32-row x 128-byte boxes the
+        // results leave in; rounds alternate between the buffers, so that one round's copies
+        // in and out overlap the next round's arithmetic); this warp reads its 32 columns of
+        // G and U for row `lane`, computes dG and dU and writes them over G and U in place.
+#pragma unroll 1
+        for (int hr = 0; hr < halves * BW_RPH; ++hr) {
+          const int h = hr / BW_RPH, rnd = hr % BW_RPH;
+          const int b = staged_n & 1;
+          uint8_t* gbox = stg + b * BW_STG_BYTES + quarter * 4096;
+          uint8_t* ubox = gbox + 16384;
+          // G and U of this round have landed (use staged_n / 2 of buffer b)
+          const bool fr = wait_inl(zfull_bar(b), (uint32_t)(staged_n >> 1) & 1u, abort_flag,
+                                   a.status, a.timeout_ns);
+          if (!__all_sync(0xffffffffu, fr)) {
+            ok = false;
+            break;
+          }
+          uint32_t v[32];
+          tmem_ld32(taddr + BW_N * h + 64 * rnd + 32 * ch, v);
+          tmem_wait_ld();
+          if (rnd == BW_RPH - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(tfree_bar(h));
+              if (halves == 1) mbar_arrive(tfree_bar(1));
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t off = swz(lane, 4 * ch + i);
+            const uint4 gz = *reinterpret_cast<const uint4*>(gbox + off);
+            const uint4 uz = *reinterpret_cast<const uint4*>(ubox + off);
+            const uint32_t gw[4] = {gz.x, gz.y, gz.z, gz.w};
+            const uint32_t uw[4] = {uz.x, uz.y, uz.z, uz.w};
+            uint32_t dg[4], du[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 g = bf2_to_f2(gw[j]), u = bf2_to_f2(uw[j]);
+              // sigma = 1 / (1 + e^-g); t = dA sigma; dU = t g; dG = t u (1 + g (1 - sigma))
+              const float s0 = __fdividef(1.0f, 1.0f + __expf(-g.x));
+              const float s1 = __fdividef(1.0f, 1.0f + __expf(-g.y));
+              const float t0 = __uint_as_float(v[8 * i + 2 * j]) * s0;
+              const float t1 = __uint_as_float(v[8 * i + 2 * j + 1]) * s1;
+              dg[j] = pack_bf16(t0 * u.x * fmaf(g.x, 1.0f - s0, 1.0f),
+                                t1 * u.y * fmaf(g.y, 1.0f - s1, 1.0f));
+              du[j] = pack_bf16(t0 * g.x, t1 * g.y);
+            }
+            *reinterpret_cast<uint4*>(gbox + off) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+            *reinterpret_cast<uint4*>(ubox + off) = make_uint4(du[0], du[1], du[2], du[3]);
+          }
+          fence_proxy_async();  // make the staging writes visible to the TMA engine
+          __syncwarp();
+          if (lane == 0) mbar_arrive(dstaged_bar(b));
+          ++staged_n;
+        }
+      }
+      if (!ok) break;
+      if (!w.zero) ++acc_it;
+    }
+  } else if (G::STORES && warp == BW_STORE_WARP) {
+    // ------------------------------------------------------------ store warp (warp 10)
+    if (lane == 0) {
+      if constexpr (KIND == BWD_DGRAD_A) {
+        // Per round: the G and U boxes of the round's 64 columns in, two rounds ahead (round
+        // n uses buffer n % 2), then, once the epilogue has written dG and dU over them, the
+        // boxes out to dZ's G and U column ranges.
+        int n = 0;                // rounds so far (the epilogue counts the same)
+        int zarm0 = -1, zarm1 = -1;  // per buffer: the use whose copies are armed, not consumed
+        auto load_round = [&](const BwItem& w, int r, int nn) {
+          const int b = nn & 1, h = r / BW_RPH;
+          const int rows = min(w.nrows - BW_H * h, BW_H);
+          const int x = w.n0 + 64 * (r % BW_RPH);
+          uint8_t* buf = stg + b * BW_STG_BYTES;
+          mbar_expect_tx(zfull_bar(b), (uint32_t)(rows / 32) * 8192u);
+          for (int q = 0; 32 * q < rows; ++q) {
+            const int y = w.row0 + BW_H * h + 32 * q;
+            tma_load_2d(smem_u32(buf + q * 4096), &tmZ, zfull_bar(b), x, y);
+            tma_load_2d(smem_u32(buf + 16384 + q * 4096), &tmZ, zfull_bar(b), a.f + x, y);
+          }
+          (b ? zarm1 : zarm0) = nn >> 1;
+        };
+        bool stop = false;
+        for (int it = 0; !stop; ++it) {
+          const int L = take_item(it);
+          if (L == -2) break;
+          mbar_arrive(iempty_bar(it % BW_RING));
+          if (L < 0) break;
+          const BwItem w = bw_item<KIND>(a, L);
+          if (!w.ok) continue;
+          const int R = (w.two ? 2 : 1) * BW_RPH;
+          // both buffers are free: every earlier round's stores have been read
+          load_round(w, 0, n);
+          load_round(w, 1, n + 1);
+          for (int r = 0; r < R; ++r) {
+            const int nn = n + r, b = nn & 1, h = r / BW_RPH;
+            if (!mbar_wait(dstaged_bar(b), (uint32_t)(nn >> 1) & 1u, abort_flag, a.status,
+                           a.timeout_ns, true)) {
+              stop = true;
+              break;
+            }
+            (b ? zarm1 : zarm0) = -1;
+            const int rows = min(w.nrows - BW_H * h, BW_H);
+            const int x = w.n0 + 64 * (r % BW_RPH);
+            uint8_t* buf = stg + b * BW_STG_BYTES;
+            for (int q = 0; 32 * q < rows; ++q) {
+              const int y = w.row0 + BW_H * h + 32 * q;
+              tma_store_2d(&tmO, smem_u32(buf + q * 4096), x, y);
+              tma_store_2d(&tmO, smem_u32(buf + 16384 + q * 4096), a.f + x, y);
+            }
+            bulk_commit();
+            bulk_wait_read();  // the copies have read buffer b
+            if (r + 2 < R) load_round(w, r + 2, nn + 2);
+          }
+          n += R;
+        }
+        // copies still landing in the staging buffers, then the output, before the CTA's
+        // shared memory goes away
+        if (zarm0 >= 0)
+          mbar_wait(zfull_bar(0), (uint32_t)zarm0 & 1u, abort_flag, a.status, a.timeout_ns, false);
+        if (zarm1 >= 0)
+          mbar_wait(zfull_bar(1), (uint32_t)zarm1 & 1u, abort_flag, a.status, a.timeout_ns, false);
+        bulk_wait_all();
+      } else {
+        // WGrad: one staging buffer; per round the epilogue's fp32 boxes out, then the
+        // buffer is free for the next round
+        int staged_n = 0;
+        for (int it = 0;; ++it) {
+          const int L = take_item(it);
+          if (L == -2) break;
+          mbar_arrive(iempty_bar(it % BW_RING));
+          if (L < 0) break;
+          const BwItem w = bw_item<KIND>(a, L);
+          if (!w.ok) continue;
+          bool stop = false;
+          for (int hr = 0; hr < 2 * BW_RPH; ++hr) {
+            const int h = hr / BW_RPH, rnd = hr % BW_RPH;
+            if (!mbar_wait(staged_bar, (uint32_t)staged_n & 1u, abort_flag, a.status,
+                           a.timeout_ns, true)) {
+              stop = true;
+              break;
+            }
+            const int y0 = w.e * a.m_rows + w.m0 + BW_H * h;
+            const int x = w.n0 + 64 * rnd;
+            for (int q = 0; q < 4; ++q)
+              for (int c = 0; c < 2; ++c)
+                tma_store_2d(&tmO, smem_u32(stg + q * 8192 + c * 4096), x + 32 * c,
+                             y0 + 32 * q);
+            bulk_commit();
+            bulk_wait_read();  // the copies have read the staging buffer
+            mbar_arrive(stgfree_bar);
+            ++staged_n;
+          }
+          if (stop) break;
+        }
+        bulk_wait_all();  // the output is written before the CTA's shared memory goes away
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<false, 512>(tmem_base);
+  }
+}
+
+template <int KIND>
+cudaError_t launch_kind(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+                        const CUtensorMap& tz, const BwArgs& a, cudaStream_t st) {
+  static OncePerDevice attr_once;
+  cudaError_t err = once_per_device(attr_once, [&](int&) {
+    return cudaFuncSetAttribute(bw_wide_kernel<KIND>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, BW_SMEM);
+  });
+  if (err != cudaSuccess) return err;
+  bw_wide_kernel<KIND><<<num_sms(), BW_THREADS, BW_SMEM, st>>>(ta, tb, to, tz, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool bwd_wide_supported(const moe_cfg& c, int kind) {
+  // N of dA and of dW2 is f: whole 256-column n-tiles; the other kinds' N and M are d and
+  // 2f, multiples of 256 for every layer the FFN accepts
+  if (kind == BWD_DGRAD_A || kind == BWD_WGRAD_2) return c.f % 256 == 0;
+  return kind == BWD_DGRAD_X || kind == BWD_WGRAD_1;
+}
+
+cudaError_t launch_bwd_wide(const moe_cfg& c, int kind, const uint16_t* a_src,
+                            const uint16_t* b_src, void* out, const int32_t* tiles,
+                            const int32_t* plan_info, const int32_t* block_off,
+                            const int32_t* row_token, const uint16_t* z, int32_t* sched,
+                            int32_t* status, cudaStream_t st) {
+  if (!bwd_wide_supported(c, kind)) return cudaErrorInvalidValue;
+  const long long r_max = max_rows(c);
+  BwArgs a{};
+  a.sched = sched;
+  a.tiles = tiles;
+  a.plan_info = plan_info;
+  a.block_off = block_off;
+  a.row_token = row_token;
+  a.z = z;
+  a.status = status;
+  a.r_max = r_max;
+  a.T = c.T;
+  a.d = c.d;
+  a.f = c.f;
+  a.E = c.E;
+  a.beta = c.beta;
+  a.timeout_ns = 2000000000ull;
+  CUtensorMap ta, tb, to, tz;
+  switch (kind) {
+    case BWD_DGRAD_A:  // A = D rows (K = d), B = w2 (K rows e d + k, N = f), out = dZ
+      if (!encode_2d(&ta, a_src, c.d, r_max, BW_H) ||
+          !encode_2d(&tb, b_src, c.f, (uint64_t)c.E * c.d, BW_K) ||
+          !encode_2d(&to, out, 2 * c.f, r_max, 32) ||
+          !encode_2d(&tz, z, 2 * c.f, r_max, 32))
+        return cudaErrorInvalidValue;
+      a.n_k = c.d / BW_K;
+      a.n_n = c.f / BW_N;
+      a.k_rows = c.d;
+      return launch_kind<BWD_DGRAD_A>(ta, tb, to, tz, a, st);
+    case BWD_DGRAD_X:  // A = dZ rows (K = 2f), B = w1 (K rows e 2f + k, N = d), out = dx
+      if (!encode_2d(&ta, a_src, 2 * c.f, r_max, BW_H) ||
+          !encode_2d(&tb, b_src, c.d, (uint64_t)c.E * 2 * c.f, BW_K))
+        return cudaErrorInvalidValue;
+      a.dx = static_cast<float*>(out);
+      a.n_k = 2 * c.f / BW_K;
+      a.n_n = c.d / BW_N;
+      a.k_rows = 2 * c.f;
+      return launch_kind<BWD_DGRAD_X>(ta, tb, ta, ta, a, st);
+    case BWD_WGRAD_2:  // A = D (M = d), B = A rows (N = f), K = the expert's rows
+      if (!encode_2d(&ta, a_src, c.d, r_max, BW_K) ||
+          !encode_2d(&tb, b_src, c.f, r_max, BW_K) ||
+          !encode_2d_f32(&to, out, c.f, (uint64_t)c.E * c.d, 32))
+        return cudaErrorInvalidValue;
+      a.n_m = c.d / BW_M;
+      a.n_n = c.f / BW_N;
+      a.m_rows = c.d;
+      return launch_kind<BWD_WGRAD_2>(ta, tb, to, to, a, st);
+    default:  // BWD_WGRAD_1: A = dZ (M = 2f), B = Xp rows (N = d), K = the expert's rows
+      if (!encode_2d(&ta, a_src, 2 * c.f, r_max, BW_K) ||
+          !encode_2d(&tb, b_src, c.d, r_max, BW_K) ||
+          !encode_2d_f32(&to, out, c.d, (uint64_t)c.E * 2 * c.f, 32))
+        return cudaErrorInvalidValue;
+      a.n_m = 2 * c.f / BW_M;
+      a.n_n = c.d / BW_N;
+      a.m_rows = 2 * c.f;
+      return launch_kind<BWD_WGRAD_1>(ta, tb, to, to, a, st);
+  }
+}
+
+}  // namespace moe

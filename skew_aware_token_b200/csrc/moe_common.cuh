@@ -148,6 +148,16 @@ cudaError_t launch_ffn_backward(const moe_cfg& c, const uint16_t* xp, const uint
                                 const int32_t* row_token, const uint16_t* d_rows,
                                 const uint16_t* saved, uint16_t* bwd_scratch, float* dx,
                                 float* dw1, float* dw2, int32_t* status, cudaStream_t st);
+// The four gradient products on whole 256-row tiles (ffn_bwd_wide.cu); kinds as below.
+// a_src / b_src: the product's A and B operands, out: dZ (DGRAD_A), dx (DGRAD_X, zeroed by
+// the caller), dW2 or dW1 (fp32).
+enum BwdKind { BWD_DGRAD_A = 1, BWD_DGRAD_X = 2, BWD_WGRAD_2 = 3, BWD_WGRAD_1 = 4 };
+bool bwd_wide_supported(const moe_cfg& c, int kind);
+cudaError_t launch_bwd_wide(const moe_cfg& c, int kind, const uint16_t* a_src,
+                            const uint16_t* b_src, void* out, const int32_t* tiles,
+                            const int32_t* plan_info, const int32_t* block_off,
+                            const int32_t* row_token, const uint16_t* z, int32_t* sched,
+                            int32_t* status, cudaStream_t st);
 
 int num_sms();
 

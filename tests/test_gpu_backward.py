@@ -31,6 +31,8 @@ CASES = [
     Workload("hot_all", T=515, d=256, E=16, k=4, f=128, beta=64, P=8, s=2, hot_p=1.0,
              hot_mode="all4"),
     Workload("idle_experts", T=24, d=256, E=32, k=1, f=256, beta=64, P=4, s=1, alpha=2.0),
+    # every product on whole 256-row tiles, several n- and m-tiles, skewed experts
+    Workload("wide_skew", T=2048, d=1024, E=16, k=4, f=512, beta=128, P=4, s=2, alpha=1.0),
 ]
 
 
