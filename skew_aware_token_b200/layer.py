@@ -17,11 +17,12 @@ from . import native as N
 # From this size of y on, a fused-combine call of the layer runs FC2 with O rows plus the
 # ordered combine instead: the fused combine's fp32 reductions compete with the operand
 # copies for L2 (and go to DRAM once y outgrows it), while O rows leave through TMA stores
-# and the combine reads them once.  Measured FFN times: DeepSeek-V3-shaped layer (470 MB y)
-# 2 % faster, 8192-token Qwen3-shaped layer (64 MiB y) 6 % faster, 16384-token layers
-# (134 MB y) within 0.5 %, 4096-token layer (32 MiB y) even.  The ordered combine also
-# makes y independent of the reduction order.
-O_ROWS_MIN_Y_BYTES = 64 << 20
+# (the epilogue frees each accumulator half before staging them) and the combine reads them
+# once.  Measured FFN + combine times against the fused combine: DeepSeek-V3-shaped layer with
+# 32 experts (59 MB y) 3 % faster, 4096-token layers (32 MiB y) 1-4 % faster, and the larger
+# layers as fast or faster; the 256-token layer stays fused.  The ordered combine also makes
+# y independent of the reduction order.
+O_ROWS_MIN_Y_BYTES = 32 << 20
 
 
 class MoeLayer:
@@ -115,8 +116,11 @@ class MoeLayer:
 
     def ffn_mode(self, mode=N.MOE_FFN_FUSED_COMBINE) -> int:
         """The mode a layer call runs the FFN in: with o_rows, MOE_FFN_WRITE_O is added to a
-        fused-combine mode (the layer then runs moe_combine after the FFN)."""
-        return mode | N.MOE_FFN_WRITE_O if self.o_rows else mode
+        fused-combine mode (the layer then runs moe_combine after the FFN), except to one
+        that asks for the one-launch FFN, which fuses the combine by design."""
+        if self.o_rows and not mode & N.MOE_FFN_ONE_LAUNCH:
+            return mode | N.MOE_FFN_WRITE_O
+        return mode
 
     def ffn(self, w1, w2, mode=N.MOE_FFN_FUSED_COMBINE, stream=None, y=None, x=None):
         """The expert FFN; `x` (the token rows) is needed when the layer gathers them."""

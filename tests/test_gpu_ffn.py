@@ -65,7 +65,8 @@ def test_ffn_every_element(wl, gather_x):
     """Both A sources of FC1: rows gathered from x by row_token, and the dispatched Xp."""
     w1, w2 = synth.make_weights(wl, "cuda")
     ref = _oracle_full(wl, w1, w2)
-    layer = MoeLayer(wl, "cuda", write_o=True, gather_x=gather_x)
+    # o_rows=False: each mode runs as written (the layer's own choice would add O rows)
+    layer = MoeLayer(wl, "cuda", write_o=True, gather_x=gather_x, o_rows=False)
     for mode in MODES:
         if gather_x and mode & (N.MOE_FFN_ONE_LAUNCH | N.MOE_FFN_TWO_LAUNCHES |
                                 N.MOE_FFN_FC1_M128 | N.MOE_FFN_FC2_WHOLE):

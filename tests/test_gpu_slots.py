@@ -33,7 +33,9 @@ CONFIGS = {
 def _run(wl, mode, layer=None):
     w1, w2 = synth.make_weights(wl, "cuda")
     logits, x = synth.make_logits(wl).cuda(), synth.make_x(wl).cuda()
-    layer = layer or MoeLayer(wl, "cuda", write_o=True)
+    # o_rows=False: each configuration runs as written (the layer's own choice would add O
+    # rows to the fused-combine ones)
+    layer = layer or MoeLayer(wl, "cuda", write_o=True, o_rows=False)
     layer.clear_status()
     layer(logits, x, w1, w2, mode=mode | N.MOE_FFN_RECORD_SLOTS)
     torch.cuda.synchronize()
