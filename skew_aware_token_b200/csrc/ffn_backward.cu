@@ -1,15 +1,15 @@
 // Backward of the grouped SwiGLU expert FFN on the sm_100a tensor cores: the dispatch of the
-// output gradient, and the four gradient products on 128-row tile halves.  Each product runs
-// on the whole-tile kernels of ffn_bwd_wide.cu instead where its shape allows (all four when
-// f is a multiple of 256); the kernels here remain for the other shapes.
+// output gradient, the launch sequence of the four gradient products, and the tile-half
+// kernels for the two products whose N is f (dA and dW2) when f is not a multiple of 256.
+// Every other product runs on the whole-tile kernels of ffn_bwd_wide.cu.
 //
 // "MegaFlux" summary, Methodology 2, backward gradients, with this library's weight layouts
 // w1 [E, 2f, d] and w2 [E, d, f] (each of the pages' products is taken with that transpose):
 //   D   = row_gate * dy[row_token]                 moe_dispatch_grad (bf16, zero padding)
 //   dA  = D w2_e; dZ = [dA U SiLU'(G), dA SiLU(G)]  kind DGRAD_A: GEMM + SwiGLU backward
-//   dX  = dZ w1_e; dx[row_token] += dX              kind DGRAD_X: GEMM + scatter-add
+//   dX  = dZ w1_e; dx[row_token] += dX              kind DGRAD_X (whole tiles only)
 //   dW2_e = D^T A                                   kind WGRAD_2: per expert, K = its rows
-//   dW1_e = dZ^T Xp                                 kind WGRAD_1: per expert, K = its rows
+//   dW1_e = dZ^T Xp                                 kind WGRAD_1 (whole tiles only)
 // Backward item 3 requantizes D and dZ: both are stored bf16 and enter the products so.
 //
 // Operand layouts.  K-major operands (D and dZ as A of the DGrad kinds) are copied as in
@@ -59,8 +59,7 @@ struct BGeo {
                                     ((A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16) |
                                     ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 };
-static_assert(BGeo<DGRAD_A, 256>::SMEM <= 227 * 1024 && BGeo<DGRAD_X, 256>::SMEM <= 227 * 1024 &&
-                  BGeo<WGRAD_2, 256>::SMEM <= 227 * 1024 && BGeo<WGRAD_1, 256>::SMEM <= 227 * 1024,
+static_assert(BGeo<DGRAD_A, 128>::SMEM <= 227 * 1024 && BGeo<WGRAD_2, 128>::SMEM <= 227 * 1024,
               "smem");
 static_assert(BGeo<DGRAD_A, 128>::NBARS * 8 + 4 * (2 + kRing) + 4 * 128 <= kMetaBytes, "meta");
 
@@ -72,7 +71,6 @@ struct BwdArgs {
   const int32_t* row_token;
   const uint16_t* z;  // DGRAD_A: saved Z = [G, U] bf16 [r_max, 2f]
   uint16_t* dz;       // DGRAD_A: dZ bf16 [r_max, 2f]
-  float* dx;          // DGRAD_X: dx fp32 [T, d]
   float* dw;          // WGRAD: dW2 [E, d, f] or dW1 [E, 2f, d]
   int32_t* status;
   long long r_max;
@@ -138,7 +136,6 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + G::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
-  int* s_tok = reinterpret_cast<int*>(tmem_slot + 2 + kRing);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
@@ -294,7 +291,6 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int quarter = warp & 3;
-    const int rit = quarter * 32 + lane;  // accumulator row = TMEM lane
     const int ew = warp - 2;
     int acc_it = 0;
     for (int it = 0;; ++it) {
@@ -388,40 +384,6 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 make_uint2(pack_bf16(dg[0], dg[1]), pack_bf16(dg[2], dg[3]));
             *reinterpret_cast<uint2*>(dzrow + a.f + col) =
                 make_uint2(pack_bf16(du[0], du[1]), pack_bf16(du[2], du[3]));
-          }
-          __syncwarp();
-        }
-      } else if (KIND == DGRAD_X) {
-        // dx[token] += dX, staged per 32 x 32 chunk so that one vector reduction of 8 lanes
-        // covers a 128-byte segment of one row
-        const long long row = (long long)w.row0 + rit;
-        const bool valid = rit < w.nrows && row < a.r_max;
-        int tok = valid ? __ldg(a.row_token + row) : -1;
-        if (tok >= a.T) tok = -1;
-        s_tok[ew * 32 + lane] = tok;
-        float* my_row = stg + (ew * 32 + lane) * kStgStride;
-        float* y = a.dx + w.n0 + 4 * (lane & 7);
-        __syncwarp();
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(taddr + c * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<float4*>(my_row + 4 * j) =
-                make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                            __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-          __syncwarp();
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int r = 4 * i + (lane >> 3);
-            const int tk = s_tok[ew * 32 + r];
-            if (tk >= 0) {
-              const float4 x = *reinterpret_cast<const float4*>(
-                  stg + (ew * 32 + r) * kStgStride + 4 * (lane & 7));
-              red_add_v4(y + (long long)tk * a.d + c * 32, x);
-            }
           }
           __syncwarp();
         }
@@ -554,15 +516,11 @@ cudaError_t launch_ffn_backward(const moe_cfg& c, const uint16_t* xp, const uint
       reinterpret_cast<const uint8_t*>(saved) + ffn_scratch_bytes(c));
 
   // K-major A operands: boxes of 128 rows; MN-major operands: boxes of 64 rows
-  CUtensorMap m_d_k, m_dz_k, m_w2, m_w1, m_d_mn, m_a_mn, m_dz_mn, m_xp_mn;
+  CUtensorMap m_d_k, m_w2, m_d_mn, m_a_mn;
   if (!encode_2d(&m_d_k, d_rows, c.d, r_max, kBM) ||
-      !encode_2d(&m_dz_k, dz, 2 * c.f, r_max, kBM) ||
       !encode_2d(&m_w2, w2, c.f, (uint64_t)c.E * c.d, kBK) ||
-      !encode_2d(&m_w1, w1, c.d, (uint64_t)c.E * 2 * c.f, kBK) ||
       !encode_2d(&m_d_mn, d_rows, c.d, r_max, kBK) ||
-      !encode_2d(&m_a_mn, a_saved, c.f, r_max, kBK) ||
-      !encode_2d(&m_dz_mn, dz, 2 * c.f, r_max, kBK) ||
-      !encode_2d(&m_xp_mn, xp, c.d, r_max, kBK))
+      !encode_2d(&m_a_mn, a_saved, c.f, r_max, kBK))
     return cudaErrorInvalidValue;
 
   BwdArgs base{};
@@ -579,66 +537,44 @@ cudaError_t launch_ffn_backward(const moe_cfg& c, const uint16_t* xp, const uint
   base.beta = c.beta;
   base.timeout_ns = kWaitNs;
 
-  // Each product runs on whole 256-row tiles where its shape allows (ffn_bwd_wide.cu), else
-  // on the 128-row tile halves below.
-  // dA = D w2 (N = f in tiles of 256, or 128, K = d) with the SwiGLU backward -> dZ
-  BwdArgs g1 = base;
-  g1.sched = sched + 0;
-  g1.z = z_saved;
-  g1.dz = dz;
-  g1.n_k = c.d / kBK;
-  g1.k_rows = c.d;
+  // Each product runs on whole 256-row tiles (ffn_bwd_wide.cu) where its shape allows: dX and
+  // dW1 always, dA and dW2 when f is a multiple of 256; else on 128-row tile halves (N = 128).
+  // dA = D w2 (N = f, K = d) with the SwiGLU backward -> dZ
   if (bwd_wide_supported(c, BWD_DGRAD_A)) {
     err = launch_bwd_wide(c, BWD_DGRAD_A, d_rows, w2, dz, tiles, plan_info, block_off,
                           row_token, z_saved, sched + 0, status, st);
-  } else if (c.f % 256 == 0) {
-    g1.n_n = c.f / 256;
-    err = launch_bwd<DGRAD_A, 256>(m_d_k, m_w2, g1, st);
   } else {
+    BwdArgs g1 = base;
+    g1.sched = sched + 0;
+    g1.z = z_saved;
+    g1.dz = dz;
+    g1.n_k = c.d / kBK;
+    g1.k_rows = c.d;
     g1.n_n = c.f / 128;
     err = launch_bwd<DGRAD_A, 128>(m_d_k, m_w2, g1, st);
   }
   if (err != cudaSuccess) return err;
-  // dX = dZ w1 (N = d in tiles of 256, K = 2f), scattered into dx
-  BwdArgs g2 = base;
-  g2.sched = sched + 1;
-  g2.dx = dx;
-  g2.n_k = 2 * c.f / kBK;
-  g2.n_n = c.d / 256;
-  g2.k_rows = 2 * c.f;
-  err = bwd_wide_supported(c, BWD_DGRAD_X)
-            ? launch_bwd_wide(c, BWD_DGRAD_X, dz, w1, dx, tiles, plan_info, block_off,
-                              row_token, nullptr, sched + 1, status, st)
-            : launch_bwd<DGRAD_X, 256>(m_dz_k, m_w1, g2, st);
+  // dX = dZ w1 (N = d, K = 2f), reduced into dx
+  err = launch_bwd_wide(c, BWD_DGRAD_X, dz, w1, dx, tiles, plan_info, block_off, row_token,
+                        nullptr, sched + 1, status, st);
   if (err != cudaSuccess) return err;
   // dW2_e [d, f] = D^T A (M = d, N = f, K = the expert's rows)
-  BwdArgs g3 = base;
-  g3.sched = sched + 2;
-  g3.dw = dw2;
-  g3.n_m = c.d / kBM;
-  g3.n_out = c.f;
   if (bwd_wide_supported(c, BWD_WGRAD_2)) {
     err = launch_bwd_wide(c, BWD_WGRAD_2, d_rows, a_saved, dw2, tiles, plan_info, block_off,
                           row_token, nullptr, sched + 2, status, st);
-  } else if (c.f % 256 == 0) {
-    g3.n_n = c.f / 256;
-    err = launch_bwd<WGRAD_2, 256>(m_d_mn, m_a_mn, g3, st);
   } else {
+    BwdArgs g3 = base;
+    g3.sched = sched + 2;
+    g3.dw = dw2;
+    g3.n_m = c.d / kBM;
+    g3.n_out = c.f;
     g3.n_n = c.f / 128;
     err = launch_bwd<WGRAD_2, 128>(m_d_mn, m_a_mn, g3, st);
   }
   if (err != cudaSuccess) return err;
   // dW1_e [2f, d] = dZ^T Xp (M = 2f, N = d, K = the expert's rows)
-  BwdArgs g4 = base;
-  g4.sched = sched + 3;
-  g4.dw = dw1;
-  g4.n_m = 2 * c.f / kBM;
-  g4.n_n = c.d / 256;
-  g4.n_out = c.d;
-  return bwd_wide_supported(c, BWD_WGRAD_1)
-             ? launch_bwd_wide(c, BWD_WGRAD_1, dz, xp, dw1, tiles, plan_info, block_off,
-                               row_token, nullptr, sched + 3, status, st)
-             : launch_bwd<WGRAD_1, 256>(m_dz_mn, m_xp_mn, g4, st);
+  return launch_bwd_wide(c, BWD_WGRAD_1, dz, xp, dw1, tiles, plan_info, block_off, row_token,
+                         nullptr, sched + 3, status, st);
 }
 
 }  // namespace moe
