@@ -21,18 +21,22 @@
 // 64-element MN chunks and 1 KB between 8-row K groups, a K step of 16 advances 2 KB.
 //
 // Epilogues.  The warps that read TMEM keep global stores out of their way (pending stores
-// hold up a warp's next TMEM load): results go through a 32 KB shared staging buffer, in
-// 32-row x 128-byte boxes with the 128-byte swizzle, and a store warp writes the boxes with
-// TMA stores.
-//   DGRAD_A  per round 64 columns of dA: the warp loads the matching G and U of its row
-//            (bf16, saved by the forward) before reading TMEM, computes dG and dU, rounds
-//            them to bf16, and stages one box of dG and one of dU; the store warp writes
-//            them to dZ's G and U column ranges.
+// hold up a warp's next TMEM load): results go through 32 KB of shared staging, and a store
+// warp writes them with TMA stores.
+//   DGRAD_A  rounds of 32 dA columns alternate between two 16 KB staging buffers.  The store
+//            warp copies the round's G and U (bf16, saved by the forward; 32-row x 64-byte
+//            boxes, the producer having prefetched the item's G and U into L2) into a buffer
+//            two rounds ahead; the epilogue warps read dA from TMEM, compute dG and dU, round
+//            them to bf16 and write them over G and U; the store warp writes the boxes to
+//            dZ's G and U column ranges.  One round's copies in and out overlap the next
+//            round's arithmetic.
 //   DGRAD_X  dx[token] += dX with 16-byte vector reductions, each warp transposing 32 x 32
 //            chunks through its own 4 KB slot (as the forward's fused combine, gate 1: the
 //            gate is already in D).
-//   WGRAD    dW fp32: per round 64 columns (two 32-column fp32 boxes per row group).  An idle
-//            expert's items issue no MMA and stage zeros.
+//   WGRAD    dW fp32: each epilogue warp reads its 128 columns of a half into registers and
+//            frees the half, then stages them in rounds of 64 columns (32-row x 128-byte
+//            fp32 boxes, 128-byte swizzle).  An idle expert's items issue no MMA and stage
+//            zeros.
 // Roles (352 threads, one CTA per SM, persistent): warp 0 TMA producer, warp 1 MMA issuer,
 // warps 2..9 epilogue (warp w reads TMEM lanes 32 (w % 4) .. +31, and half of each round's
 // columns), warp 10 store warp (idle for DGRAD_X).  Items come from a global counter in
@@ -46,7 +50,7 @@ constexpr int BW_M = 256;   // output rows per item
 constexpr int BW_H = 128;   // rows per MMA (TMEM lanes)
 constexpr int BW_K = 64;    // K per stage
 constexpr int BW_N = 256;   // MMA N
-constexpr int BW_ST = 3;    // pipeline stages (DGRAD_A: 2, for a second staging buffer)
+constexpr int BW_ST = 3;    // pipeline stages
 constexpr int BW_A_BYTES = BW_M * BW_K * 2;
 constexpr int BW_B_BYTES = BW_N * BW_K * 2;
 constexpr int BW_STAGE = BW_A_BYTES + BW_B_BYTES;
@@ -59,8 +63,11 @@ constexpr int BW_STORE_WARP = 2 + BW_EPI_WARPS;
 constexpr int BW_NBARS = 2 * BW_ST + 8 + 2 * BW_RING;
 constexpr int BW_META = 512;
 constexpr int BW_SMEM = BW_ST * BW_STAGE + BW_STG_BYTES + BW_META + 1024;
-static_assert(2 * BW_STAGE + 2 * BW_STG_BYTES <= BW_ST * BW_STAGE + BW_STG_BYTES, "DGRAD_A smem");
-constexpr int BW_RPH = 4;  // store rounds of 64 columns per accumulator half
+constexpr int BW_RPH = 4;  // WGrad: store rounds of 64 columns per accumulator half
+// DGRAD_A: rounds of 32 columns (8 per half) through two 16 KB staging buffers, each holding
+// the round's G and U boxes (32 rows x 64 bytes per TMEM lane quadrant, no swizzle)
+constexpr int BWA_RPH = 8;
+constexpr int BWA_BUF = 16384;
 static_assert(BW_NBARS * 8 + 4 * (2 + BW_RING) <= BW_META, "meta");
 static_assert(BW_SMEM <= 227 * 1024, "smem");
 
@@ -69,8 +76,7 @@ struct BwGeo {
   static constexpr bool DGRAD = KIND == BWD_DGRAD_A || KIND == BWD_DGRAD_X;
   static constexpr bool A_MN = !DGRAD;                // WGrad: both operands MN-major
   static constexpr bool STORES = KIND != BWD_DGRAD_X;  // the store warp takes items
-  static constexpr int ST = KIND == BWD_DGRAD_A ? 2 : BW_ST;  // pipeline stages
-  static constexpr int NSTG = KIND == BWD_DGRAD_A ? 2 : 1;    // 32 KB staging buffers
+  static constexpr int ST = BW_ST;  // pipeline stages
   // kind::f16: D fp32, A and B bf16, A / B major bits, N >> 3 at bit 17, M >> 4 at bit 24
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
                                     ((A_MN ? 1u : 0u) << 15) | (1u << 16) |
@@ -159,7 +165,7 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                                              ~uintptr_t(1023));
   constexpr int ST = G::ST;
   uint8_t* stg = smem + ST * BW_STAGE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + G::NSTG * BW_STG_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + BW_STG_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + BW_NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -256,9 +262,9 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           // the epilogue reads the item's G and U columns (256 rows x 256 each): bring them
           // into L2 while the item's MMAs run
           for (int r0 = 0; r0 < w.nrows; r0 += 32)
-            for (int c = 0; c < BW_N / 64; ++c) {
-              tma_prefetch_l2_2d(&tmZ, w.n0 + 64 * c, w.row0 + r0);
-              tma_prefetch_l2_2d(&tmZ, a.f + w.n0 + 64 * c, w.row0 + r0);
+            for (int c = 0; c < BW_N / 32; ++c) {
+              tma_prefetch_l2_2d(&tmZ, w.n0 + 32 * c, w.row0 + r0);
+              tma_prefetch_l2_2d(&tmZ, a.f + w.n0 + 32 * c, w.row0 + r0);
             }
         }
         const uint32_t tx = G::DGRAD ? (w.two ? 2 : 1) * BW_HALF_A + BW_B_BYTES : BW_STAGE;
@@ -512,17 +518,17 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (!ok) break;
         }
       } else {
-        // DGRAD_A: per round the store warp has copied the G and U boxes of the round's 64
-        // columns into one of the two staging buffers (the same 32-row x 128-byte boxes the
-        // results leave in; rounds alternate between the buffers, so that one round's copies
-        // in and out overlap the next round's arithmetic); this warp reads its 32 columns of
-        // G and U for row `lane`, computes dG and dU and writes them over G and U in place.
+        // DGRAD_A: per round the store warp has copied the G and U boxes of the round's 32
+        // columns into one of the two staging buffers (rounds alternate between them, so that
+        // one round's copies in and out overlap the next round's arithmetic); this warp reads
+        // its 16 columns of G and U for row `lane` (two 16-byte chunks of the row's 64 bytes),
+        // computes dG and dU and writes them over G and U in place.
 #pragma unroll 1
-        for (int hr = 0; hr < halves * BW_RPH; ++hr) {
-          const int h = hr / BW_RPH, rnd = hr % BW_RPH;
+        for (int hr = 0; hr < halves * BWA_RPH; ++hr) {
+          const int h = hr / BWA_RPH, rnd = hr % BWA_RPH;
           const int b = staged_n & 1;
-          uint8_t* gbox = stg + b * BW_STG_BYTES + quarter * 4096;
-          uint8_t* ubox = gbox + 16384;
+          uint8_t* grow = stg + b * BWA_BUF + quarter * 2048 + lane * 64 + ch * 32;
+          uint8_t* urow = grow + BWA_BUF / 2;
           // G and U of this round have landed (use staged_n / 2 of buffer b)
           const bool fr = wait_inl(zfull_bar(b), (uint32_t)(staged_n >> 1) & 1u, abort_flag,
                                    a.status, a.timeout_ns);
@@ -530,10 +536,10 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             ok = false;
             break;
           }
-          uint32_t v[32];
-          tmem_ld32(taddr + BW_N * h + 64 * rnd + 32 * ch, v);
+          uint32_t v[16];
+          tmem_ld16(taddr + BW_N * h + 32 * rnd + 16 * ch, v);
           tmem_wait_ld();
-          if (rnd == BW_RPH - 1) {
+          if (rnd == BWA_RPH - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -542,10 +548,9 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
           }
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t off = swz(lane, 4 * ch + i);
-            const uint4 gz = *reinterpret_cast<const uint4*>(gbox + off);
-            const uint4 uz = *reinterpret_cast<const uint4*>(ubox + off);
+          for (int i = 0; i < 2; ++i) {
+            const uint4 gz = *reinterpret_cast<const uint4*>(grow + 16 * i);
+            const uint4 uz = *reinterpret_cast<const uint4*>(urow + 16 * i);
             const uint32_t gw[4] = {gz.x, gz.y, gz.z, gz.w};
             const uint32_t uw[4] = {uz.x, uz.y, uz.z, uz.w};
             uint32_t dg[4], du[4];
@@ -561,8 +566,8 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                                 t1 * u.y * fmaf(g.y, 1.0f - s1, 1.0f));
               du[j] = pack_bf16(t0 * g.x, t1 * g.y);
             }
-            *reinterpret_cast<uint4*>(gbox + off) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
-            *reinterpret_cast<uint4*>(ubox + off) = make_uint4(du[0], du[1], du[2], du[3]);
+            *reinterpret_cast<uint4*>(grow + 16 * i) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+            *reinterpret_cast<uint4*>(urow + 16 * i) = make_uint4(du[0], du[1], du[2], du[3]);
           }
           fence_proxy_async();  // make the staging writes visible to the TMA engine
           __syncwarp();
@@ -577,21 +582,21 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // ------------------------------------------------------------ store warp (warp 10)
     if (lane == 0) {
       if constexpr (KIND == BWD_DGRAD_A) {
-        // Per round: the G and U boxes of the round's 64 columns in, two rounds ahead (round
+        // Per round: the G and U boxes of the round's 32 columns in, two rounds ahead (round
         // n uses buffer n % 2), then, once the epilogue has written dG and dU over them, the
         // boxes out to dZ's G and U column ranges.
-        int n = 0;                // rounds so far (the epilogue counts the same)
+        int n = 0;                   // rounds so far (the epilogue counts the same)
         int zarm0 = -1, zarm1 = -1;  // per buffer: the use whose copies are armed, not consumed
         auto load_round = [&](const BwItem& w, int r, int nn) {
-          const int b = nn & 1, h = r / BW_RPH;
+          const int b = nn & 1, h = r / BWA_RPH;
           const int rows = min(w.nrows - BW_H * h, BW_H);
-          const int x = w.n0 + 64 * (r % BW_RPH);
-          uint8_t* buf = stg + b * BW_STG_BYTES;
-          mbar_expect_tx(zfull_bar(b), (uint32_t)(rows / 32) * 8192u);
+          const int x = w.n0 + 32 * (r % BWA_RPH);
+          uint8_t* buf = stg + b * BWA_BUF;
+          mbar_expect_tx(zfull_bar(b), (uint32_t)(rows / 32) * 4096u);
           for (int q = 0; 32 * q < rows; ++q) {
             const int y = w.row0 + BW_H * h + 32 * q;
-            tma_load_2d(smem_u32(buf + q * 4096), &tmZ, zfull_bar(b), x, y);
-            tma_load_2d(smem_u32(buf + 16384 + q * 4096), &tmZ, zfull_bar(b), a.f + x, y);
+            tma_load_2d(smem_u32(buf + q * 2048), &tmZ, zfull_bar(b), x, y);
+            tma_load_2d(smem_u32(buf + BWA_BUF / 2 + q * 2048), &tmZ, zfull_bar(b), a.f + x, y);
           }
           (b ? zarm1 : zarm0) = nn >> 1;
         };
@@ -603,12 +608,12 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (L < 0) break;
           const BwItem w = bw_item<KIND>(a, L);
           if (!w.ok) continue;
-          const int R = (w.two ? 2 : 1) * BW_RPH;
+          const int R = (w.two ? 2 : 1) * BWA_RPH;
           // both buffers are free: every earlier round's stores have been read
           load_round(w, 0, n);
           load_round(w, 1, n + 1);
           for (int r = 0; r < R; ++r) {
-            const int nn = n + r, b = nn & 1, h = r / BW_RPH;
+            const int nn = n + r, b = nn & 1, h = r / BWA_RPH;
             if (!mbar_wait(dstaged_bar(b), (uint32_t)(nn >> 1) & 1u, abort_flag, a.status,
                            a.timeout_ns, true)) {
               stop = true;
@@ -616,12 +621,12 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
             (b ? zarm1 : zarm0) = -1;
             const int rows = min(w.nrows - BW_H * h, BW_H);
-            const int x = w.n0 + 64 * (r % BW_RPH);
-            uint8_t* buf = stg + b * BW_STG_BYTES;
+            const int x = w.n0 + 32 * (r % BWA_RPH);
+            uint8_t* buf = stg + b * BWA_BUF;
             for (int q = 0; 32 * q < rows; ++q) {
               const int y = w.row0 + BW_H * h + 32 * q;
-              tma_store_2d(&tmO, smem_u32(buf + q * 4096), x, y);
-              tma_store_2d(&tmO, smem_u32(buf + 16384 + q * 4096), a.f + x, y);
+              tma_store_2d(&tmO, smem_u32(buf + q * 2048), x, y);
+              tma_store_2d(&tmO, smem_u32(buf + BWA_BUF / 2 + q * 2048), a.f + x, y);
             }
             bulk_commit();
             bulk_wait_read();  // the copies have read buffer b
@@ -730,8 +735,8 @@ cudaError_t launch_bwd_wide(const moe_cfg& c, int kind, const uint16_t* a_src,
     case BWD_DGRAD_A:  // A = D rows (K = d), B = w2 (K rows e d + k, N = f), out = dZ
       if (!encode_2d(&ta, a_src, c.d, r_max, BW_H) ||
           !encode_2d(&tb, b_src, c.f, (uint64_t)c.E * c.d, BW_K) ||
-          !encode_2d(&to, out, 2 * c.f, r_max, 32) ||
-          !encode_2d(&tz, z, 2 * c.f, r_max, 32))
+          !encode_2d_plain(&to, out, 2 * c.f, r_max, 32, 32) ||
+          !encode_2d_plain(&tz, z, 2 * c.f, r_max, 32, 32))
         return cudaErrorInvalidValue;
       a.n_k = c.d / BW_K;
       a.n_n = c.f / BW_N;
