@@ -1,33 +1,27 @@
 // Backward of the grouped SwiGLU expert FFN on the sm_100a tensor cores: the dispatch of the
-// output gradient, the launch sequence of the four gradient products, and the tile-half
-// kernels for the two products whose N is f (dA and dW2) when f is not a multiple of 256.
-// Every other product runs on the whole-tile kernels of ffn_bwd_wide.cu.
+// output gradient, the launch sequence of the four gradient products, and a weight-gradient
+// kernel on 128-row tiles for dW2 when f is not a multiple of 256.  The products themselves
+// run on the whole-tile kernels of ffn_bwd_wide.cu.
 //
 // "MegaFlux" summary, Methodology 2, backward gradients, with this library's weight layouts
 // w1 [E, 2f, d] and w2 [E, d, f] (each of the pages' products is taken with that transpose):
 //   D   = row_gate * dy[row_token]                 moe_dispatch_grad (bf16, zero padding)
-//   dA  = D w2_e; dZ = [dA U SiLU'(G), dA SiLU(G)]  kind DGRAD_A: GEMM + SwiGLU backward
-//   dX  = dZ w1_e; dx[row_token] += dX              kind DGRAD_X (whole tiles only)
-//   dW2_e = D^T A                                   kind WGRAD_2: per expert, K = its rows
-//   dW1_e = dZ^T Xp                                 kind WGRAD_1 (whole tiles only)
+//   dA  = D w2_e; dZ = [dA U SiLU'(G), dA SiLU(G)]  GEMM + SwiGLU backward
+//   dX  = dZ w1_e; dx[row_token] += dX              GEMM + reduction into dx
+//   dW2_e = D^T A                                   per expert, K = its rows
+//   dW1_e = dZ^T Xp                                 per expert, K = its rows
 // Backward item 3 requantizes D and dZ: both are stored bf16 and enter the products so.
 //
-// Operand layouts.  K-major operands (D and dZ as A of the DGrad kinds) are copied as in
-// the forward: boxes of 64 K (128 bytes) x 128 rows, 128-byte swizzle.  MN-major operands
-// (the weights as B of the DGrad kinds, and both operands of the WGrad kinds, whose K is
-// the token rows) are copied in boxes of 64 MN elements (128 bytes) x 64 K rows, box j of
-// a stage 8 KB after box j-1; their MMA descriptors describe the MN-major swizzled layout:
-// leading offset 8 KB (between 64-element MN chunks), stride offset 1 KB (between 8-row K
-// groups), and a K step of 16 advances 2 KB.  The instruction descriptor marks such an
-// operand MN-major (bit 15 for A, bit 16 for B).
-//
-// Roles (192 threads, one CTA per SM, persistent), scheduling and bounded waits are those
-// of the forward kernels: warp 0 issues the TMA copies, one thread of warp 1 the MMAs into
-// two TMEM accumulators, warps 2..5 drain them; work items come from a global counter in
-// increasing order through a ring in shared memory.  DGrad items are (128-row half of a
-// planner tile, n-tile), so each expert's weights stream about once; WGrad items are
-// (expert, m-tile, n-tile) with the expert's padded rows as K (an idle expert's items just
-// write zeros).
+// The 128-row weight-gradient kernel: items (expert, m-tile of 128 dW2 rows, n-tile of 128
+// columns) with the expert's padded rows as K (an idle expert's items just write zeros).
+// Both operands are MN-major, copied in boxes of 64 MN elements (128 bytes) x 64 K rows, box
+// j of a stage 8 KB after box j-1; their MMA descriptors describe the MN-major swizzled
+// layout: leading offset 8 KB (between 64-element MN chunks), stride offset 1 KB (between
+// 8-row K groups), and a K step of 16 advances 2 KB; the instruction descriptor marks both
+// operands MN-major (bits 15 and 16).  Roles (192 threads, one CTA per SM, persistent): warp
+// 0 issues the TMA copies, one thread of warp 1 the MMAs into two TMEM accumulators, warps
+// 2..5 drain them; work items come from a global counter in increasing order through a ring
+// in shared memory; every wait is bounded.
 #include "tc_util.cuh"
 
 namespace moe {
@@ -40,12 +34,8 @@ constexpr int kStgStride = 36;
 constexpr int kMetaBytes = 2048;
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
-enum Kind { DGRAD_A = 1, DGRAD_X = 2, WGRAD_2 = 3, WGRAD_1 = 4 };
-
-template <int KIND, int BN>
+template <int BN>
 struct BGeo {
-  static constexpr bool A_MN = KIND == WGRAD_2 || KIND == WGRAD_1;  // A read MN-major
-  static constexpr bool B_MN = true;                                // B always MN-major
   static constexpr int A_BYTES = kBM * kBK * 2;
   static constexpr int B_BYTES = BN * kBK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -56,78 +46,54 @@ struct BGeo {
   static constexpr int SMEM = STAGES * STAGE_BYTES + STG + kMetaBytes + 1024;
   // kind::f16: D fp32, A and B bf16, A / B major bits, N >> 3 at bit 17, M >> 4 at bit 24
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
-                                    ((A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16) |
+                                    (1u << 15) | (1u << 16) |
                                     ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 };
-static_assert(BGeo<DGRAD_A, 128>::SMEM <= 227 * 1024 && BGeo<WGRAD_2, 128>::SMEM <= 227 * 1024,
-              "smem");
-static_assert(BGeo<DGRAD_A, 128>::NBARS * 8 + 4 * (2 + kRing) + 4 * 128 <= kMetaBytes, "meta");
+static_assert(BGeo<128>::SMEM <= 227 * 1024, "smem");
+static_assert(BGeo<128>::NBARS * 8 + 4 * (2 + kRing) <= kMetaBytes, "meta");
 
 struct BwdArgs {
   int32_t* sched;  // this launch's work counter (zeroed by the launcher)
-  const int32_t* tiles;
-  const int32_t* plan_info;
   const int32_t* block_off;
-  const int32_t* row_token;
-  const uint16_t* z;  // DGRAD_A: saved Z = [G, U] bf16 [r_max, 2f]
-  uint16_t* dz;       // DGRAD_A: dZ bf16 [r_max, 2f]
-  float* dw;          // WGRAD: dW2 [E, d, f] or dW1 [E, 2f, d]
+  float* dw;  // dW2 [E, d, f]
   int32_t* status;
   long long r_max;
-  int T, d, f, E, beta;
-  int n_k;        // DGrad: K steps of 64
-  int n_n;        // n-tiles (N / BN)
-  int n_m;        // WGrad: m-tiles per expert (M / 128)
-  int n_out;      // WGrad: row length of dW (N); DGrad: unused
-  int k_rows;     // DGrad: first B row of expert e is e * k_rows (d for w2, 2f for w1)
+  int E, beta;
+  int n_n;    // n-tiles (N / BN)
+  int n_m;    // m-tiles per expert (M / 128)
+  int n_out;  // row length of dW (N)
   unsigned long long timeout_ns;
 };
 
 
 struct BItem {
-  bool run;    // work to do (a DGrad half with rows, or any WGrad item)
-  bool zero;   // WGrad item of an idle expert: no K, the output tile is zero
+  bool zero;   // item of an idle expert: no K, the output tile is zero
   bool ok;     // a well-formed tile
   int e, row0, nrows, nk, m0, n0;
 };
 
-template <int KIND, int BN>
+template <int BN>
 __device__ __forceinline__ BItem decode_item(const BwdArgs& a, int L) {
   BItem it;
   const int n = L % a.n_n;
   const int t = L / a.n_n;
   it.n0 = n * BN;
-  if (KIND == DGRAD_A || KIND == DGRAD_X) {
-    const int m = t >> 1, half = t & 1;
-    const int4 v = __ldg(reinterpret_cast<const int4*>(a.tiles) + m);
-    it.e = v.x;
-    it.ok = v.x >= 0 && v.x < a.E && v.y >= 0 && (long long)v.y < a.r_max && v.z > 0 &&
-            v.z <= 2 * kBM;
-    it.row0 = v.y + kBM * half;
-    it.nrows = min(v.z - kBM * half, kBM);
-    it.run = it.ok && it.nrows > 0;
-    it.zero = false;
-    it.nk = a.n_k;
-    it.m0 = 0;
-  } else {
-    it.e = t / a.n_m;
-    it.m0 = (t % a.n_m) * kBM;
-    const int b0 = __ldg(a.block_off + it.e), b1 = __ldg(a.block_off + it.e + 1);
-    it.row0 = a.beta * b0;
-    it.nrows = a.beta * (b1 - b0);
-    it.ok = b0 >= 0 && b1 >= b0 && (long long)a.beta * b1 <= a.r_max;
-    it.nk = it.ok ? it.nrows / kBK : 0;
-    it.run = true;
-    it.zero = it.nk == 0;
-  }
+  it.e = t / a.n_m;
+  it.m0 = (t % a.n_m) * kBM;
+  const int b0 = __ldg(a.block_off + it.e), b1 = __ldg(a.block_off + it.e + 1);
+  it.row0 = a.beta * b0;
+  it.nrows = a.beta * (b1 - b0);
+  it.ok = b0 >= 0 && b1 >= b0 && (long long)a.beta * b1 <= a.r_max;
+  it.nk = it.ok ? it.nrows / kBK : 0;
+  it.zero = it.nk == 0;
   return it;
 }
 
-template <int KIND, int BN>
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const BwdArgs a) {
-  using G = BGeo<KIND, BN>;
+  using G = BGeo<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -148,11 +114,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
   auto sA = [&](int s) { return smem_u32(smem + s * G::STAGE_BYTES); };
   auto sB = [&](int s) { return smem_u32(smem + s * G::STAGE_BYTES + G::A_BYTES); };
 
-  long long total;
-  if (KIND == DGRAD_A || KIND == DGRAD_X)
-    total = (long long)max(a.plan_info[MOE_PI_NTILES], 0) * 2 * a.n_n;
-  else
-    total = (long long)a.E * a.n_m * a.n_n;
+  const long long total = (long long)a.E * a.n_m * a.n_n;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < G::STAGES; ++s) {
@@ -196,9 +158,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         ring[slot] = L;
         mbar_arrive(ifull_bar(slot));
         if (L < 0) break;
-        const BItem w = decode_item<KIND, BN>(a, L);
+        const BItem w = decode_item<BN>(a, L);
         if (!w.ok) bad = true;
-        if (!w.run || w.zero) continue;
+        if (w.zero) continue;
         bool stop = false;
         for (int kb = 0; kb < w.nk; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status, a.timeout_ns,
@@ -207,18 +169,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             break;
           }
           mbar_expect_tx(full_bar(stage), G::STAGE_BYTES);
-          const int krow = KIND == DGRAD_A || KIND == DGRAD_X ? w.e * a.k_rows + kb * kBK
-                                                              : w.row0 + kb * kBK;
+          const int krow = w.row0 + kb * kBK;
 #pragma unroll
           for (int j = 0; j < BN / 64; ++j)
             tma_load_2d(sB(stage) + j * 8192, &tmB, full_bar(stage), w.n0 + 64 * j, krow);
-          if (G::A_MN) {
 #pragma unroll
-            for (int j = 0; j < kBM / 64; ++j)
-              tma_load_2d(sA(stage) + j * 8192, &tmA, full_bar(stage), w.m0 + 64 * j, krow);
-          } else {
-            tma_load_2d(sA(stage), &tmA, full_bar(stage), kb * kBK, w.row0);
-          }
+          for (int j = 0; j < kBM / 64; ++j)
+            tma_load_2d(sA(stage) + j * 8192, &tmA, full_bar(stage), w.m0 + 64 * j, krow);
           pending |= 1u << stage;
           pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == G::STAGES) {
@@ -250,8 +207,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         const int L = ring[slot];
         mbar_arrive(iempty_bar(slot));
         if (L < 0) break;
-        const BItem w = decode_item<KIND, BN>(a, L);
-        if (!w.run || w.zero) continue;
+        const BItem w = decode_item<BN>(a, L);
+        if (w.zero) continue;
         const int buf = acc_it & 1;
         const uint32_t use = (uint32_t)(acc_it >> 1) & 1u;
         if (!mbar_wait(tempty_bar(buf), use ^ 1u, abort_flag, a.status, a.timeout_ns, true))
@@ -268,7 +225,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
           const uint32_t a0 = sA(stage), b0 = sB(stage);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = G::A_MN ? sw128_mn_desc(a0 + kk * 2048) : sw128_desc(a0 + kk * 32);
+            const uint64_t ad = sw128_mn_desc(a0 + kk * 2048);
             const uint64_t bd = sw128_mn_desc(b0 + kk * 2048);
             umma_bf16<false>(d_tmem, ad, bd, G::IDESC, (kb | kk) != 0);
           }
@@ -303,18 +260,15 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       __syncwarp();
       if (lane == 0) mbar_arrive(iempty_bar(slot));
       if (L < 0) break;
-      const BItem w = decode_item<KIND, BN>(a, L);
-      if (!w.run) continue;
-      if (KIND == WGRAD_2 || KIND == WGRAD_1) {
-        if (w.zero) {  // idle expert: its gradient is zero (the warp's 32 rows, coalesced)
-          float* out0 =
-              a.dw + ((long long)w.e * a.n_m * kBM + w.m0 + quarter * 32) * a.n_out + w.n0;
-          const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int r = 0; r < 32; ++r)
-            for (int i = lane; i < BN / 4; i += 32)
-              reinterpret_cast<float4*>(out0 + (long long)r * a.n_out)[i] = z4;
-          continue;
-        }
+      const BItem w = decode_item<BN>(a, L);
+      if (w.zero) {  // idle expert: its gradient is zero (the warp's 32 rows, coalesced)
+        float* out0 =
+            a.dw + ((long long)w.e * a.n_m * kBM + w.m0 + quarter * 32) * a.n_out + w.n0;
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < 32; ++r)
+          for (int i = lane; i < BN / 4; i += 32)
+            reinterpret_cast<float4*>(out0 + (long long)r * a.n_out)[i] = z4;
+        continue;
       }
       const int buf = acc_it & 1;
       const uint32_t use = (uint32_t)(acc_it >> 1) & 1u;
@@ -323,71 +277,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-      if (KIND == DGRAD_A) {
-        // dZ = [dA * U * SiLU'(G), dA * SiLU(G)] for the n-tile's BN columns of G and U.
-        // Each 32 x 32 chunk of dA goes through shared memory; then lanes 8q..8q+7 take
-        // four columns each of one row, so a warp's loads of G and U and stores of dG and
-        // dU each cover four whole 64-byte row segments.
-        float* my_row = stg + (ew * 32 + lane) * kStgStride;
-        const int rq = lane >> 3, cq = 4 * (lane & 7);
-        bool rvalid[8];
-        long long rrow[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = quarter * 32 + 4 * i + rq;
-          rrow[i] = (long long)w.row0 + r;
-          rvalid[i] = r < w.nrows && rrow[i] < a.r_max;
-        }
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(taddr + c * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<float4*>(my_row + 4 * j) =
-                make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                            __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-          __syncwarp();
-          const int col = w.n0 + 32 * c + cq;
-          // all sixteen loads of the chunk in flight at once (rows outside the tile read the
-          // tile's first row and store nothing)
-          uint2 gzs[8], uzs[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint16_t* zrow = a.z + (rvalid[i] ? rrow[i] : (long long)w.row0) * 2 * a.f;
-            gzs[i] = __ldg(reinterpret_cast<const uint2*>(zrow + col));
-            uzs[i] = __ldg(reinterpret_cast<const uint2*>(zrow + a.f + col));
-          }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if (!rvalid[i]) continue;
-            const float4 da = *reinterpret_cast<const float4*>(
-                stg + (ew * 32 + 4 * i + rq) * kStgStride + cq);
-            const uint2 gz = gzs[i], uz = uzs[i];
-            const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gz.x));
-            const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gz.y));
-            const float2 u01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uz.x));
-            const float2 u23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uz.y));
-            const float gs[4] = {g01.x, g01.y, g23.x, g23.y};
-            const float us[4] = {u01.x, u01.y, u23.x, u23.y};
-            const float ds[4] = {da.x, da.y, da.z, da.w};
-            float dg[4], du[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float sg = 1.0f / (1.0f + __expf(-gs[q]));
-              dg[q] = ds[q] * us[q] * (sg * (1.0f + gs[q] * (1.0f - sg)));
-              du[q] = ds[q] * gs[q] * sg;
-            }
-            uint16_t* dzrow = a.dz + rrow[i] * 2 * a.f;
-            *reinterpret_cast<uint2*>(dzrow + col) =
-                make_uint2(pack_bf16(dg[0], dg[1]), pack_bf16(dg[2], dg[3]));
-            *reinterpret_cast<uint2*>(dzrow + a.f + col) =
-                make_uint2(pack_bf16(du[0], du[1]), pack_bf16(du[2], du[3]));
-          }
-          __syncwarp();
-        }
-      } else {
+      {
         // WGrad: rows m0 + 32 quarter .. of expert e's gradient, BN fp32 columns; each
         // 32 x 32 chunk goes through shared memory so that one store instruction writes
         // four whole 128-byte row segments
@@ -462,17 +352,17 @@ dispatch_grad_kernel(const float4* __restrict__ dy, const int32_t* __restrict__ 
   if (bad) set_status(status, MOE_STATUS_BAD_ID);
 }
 
-template <int KIND, int BN>
+template <int BN>
 cudaError_t launch_bwd(const CUtensorMap& ta, const CUtensorMap& tb, const BwdArgs& args,
                        cudaStream_t st) {
-  auto kern = bwd_kernel<KIND, BN>;
+  auto kern = bwd_kernel<BN>;
   static OncePerDevice attr_once;
   cudaError_t err = once_per_device(attr_once, [&](int&) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                BGeo<KIND, BN>::SMEM);
+                                BGeo<BN>::SMEM);
   });
   if (err != cudaSuccess) return err;
-  kern<<<num_sms(), kThreads, BGeo<KIND, BN>::SMEM, st>>>(ta, tb, args);
+  kern<<<num_sms(), kThreads, BGeo<BN>::SMEM, st>>>(ta, tb, args);
   return cudaGetLastError();
 }
 
@@ -515,61 +405,38 @@ cudaError_t launch_ffn_backward(const moe_cfg& c, const uint16_t* xp, const uint
   const uint16_t* z_saved = reinterpret_cast<const uint16_t*>(
       reinterpret_cast<const uint8_t*>(saved) + ffn_scratch_bytes(c));
 
-  // K-major A operands: boxes of 128 rows; MN-major operands: boxes of 64 rows
-  CUtensorMap m_d_k, m_w2, m_d_mn, m_a_mn;
-  if (!encode_2d(&m_d_k, d_rows, c.d, r_max, kBM) ||
-      !encode_2d(&m_w2, w2, c.f, (uint64_t)c.E * c.d, kBK) ||
-      !encode_2d(&m_d_mn, d_rows, c.d, r_max, kBK) ||
-      !encode_2d(&m_a_mn, a_saved, c.f, r_max, kBK))
-    return cudaErrorInvalidValue;
-
-  BwdArgs base{};
-  base.tiles = tiles;
-  base.plan_info = plan_info;
-  base.block_off = block_off;
-  base.row_token = row_token;
-  base.status = status;
-  base.r_max = r_max;
-  base.T = c.T;
-  base.d = c.d;
-  base.f = c.f;
-  base.E = c.E;
-  base.beta = c.beta;
-  base.timeout_ns = kWaitNs;
-
-  // Each product runs on whole 256-row tiles (ffn_bwd_wide.cu) where its shape allows: dX and
-  // dW1 always, dA and dW2 when f is a multiple of 256; else on 128-row tile halves (N = 128).
   // dA = D w2 (N = f, K = d) with the SwiGLU backward -> dZ
-  if (bwd_wide_supported(c, BWD_DGRAD_A)) {
-    err = launch_bwd_wide(c, BWD_DGRAD_A, d_rows, w2, dz, tiles, plan_info, block_off,
-                          row_token, z_saved, sched + 0, status, st);
-  } else {
-    BwdArgs g1 = base;
-    g1.sched = sched + 0;
-    g1.z = z_saved;
-    g1.dz = dz;
-    g1.n_k = c.d / kBK;
-    g1.k_rows = c.d;
-    g1.n_n = c.f / 128;
-    err = launch_bwd<DGRAD_A, 128>(m_d_k, m_w2, g1, st);
-  }
+  err = launch_bwd_wide(c, BWD_DGRAD_A, d_rows, w2, dz, tiles, plan_info, block_off, row_token,
+                        z_saved, sched + 0, status, st);
   if (err != cudaSuccess) return err;
   // dX = dZ w1 (N = d, K = 2f), reduced into dx
   err = launch_bwd_wide(c, BWD_DGRAD_X, dz, w1, dx, tiles, plan_info, block_off, row_token,
                         nullptr, sched + 1, status, st);
   if (err != cudaSuccess) return err;
-  // dW2_e [d, f] = D^T A (M = d, N = f, K = the expert's rows)
+  // dW2_e [d, f] = D^T A (M = d, N = f, K = the expert's rows): whole tiles when f is a
+  // multiple of 256, else the 128-row kernel above (n-tiles of 128)
   if (bwd_wide_supported(c, BWD_WGRAD_2)) {
     err = launch_bwd_wide(c, BWD_WGRAD_2, d_rows, a_saved, dw2, tiles, plan_info, block_off,
                           row_token, nullptr, sched + 2, status, st);
   } else {
-    BwdArgs g3 = base;
+    // MN-major operands: boxes of 64 rows
+    CUtensorMap m_d_mn, m_a_mn;
+    if (!encode_2d(&m_d_mn, d_rows, c.d, r_max, kBK) ||
+        !encode_2d(&m_a_mn, a_saved, c.f, r_max, kBK))
+      return cudaErrorInvalidValue;
+    BwdArgs g3{};
     g3.sched = sched + 2;
+    g3.block_off = block_off;
     g3.dw = dw2;
+    g3.status = status;
+    g3.r_max = r_max;
+    g3.E = c.E;
+    g3.beta = c.beta;
     g3.n_m = c.d / kBM;
     g3.n_out = c.f;
     g3.n_n = c.f / 128;
-    err = launch_bwd<WGRAD_2, 128>(m_d_mn, m_a_mn, g3, st);
+    g3.timeout_ns = kWaitNs;
+    err = launch_bwd<128>(m_d_mn, m_a_mn, g3, st);
   }
   if (err != cudaSuccess) return err;
   // dW1_e [2f, d] = dZ^T Xp (M = 2f, N = d, K = the expert's rows)

@@ -9,10 +9,13 @@
 //   dW2_e = D^T A                                   kind WGRAD_2  (M = d, N = f, K = rows of e)
 //   dW1_e = dZ^T Xp                                 kind WGRAD_1  (M = 2f, N = d, K = rows of e)
 // An item is 256 rows of the output (two M = 128 MMAs that share each B stage: 64 bytes of
-// copies per tensor-core clock, where the 128-row tile-half kernels need 96) times 256
+// copies per tensor-core clock for 256 columns, where 128-row tiles need 96) times 256
 // columns.  The two 128 x 256 fp32 accumulators fill the 512 TMEM columns; the epilogue frees
 // them half by half, and the next item's second-half MMAs may lag its first-half MMAs by up to
-// the three pipeline stages, as in the forward.
+// the three pipeline stages, as in the forward.  DGRAD_A, whose epilogue takes about as long
+// as its MMAs, uses items of 128 columns instead: two accumulators of 2 x 128 columns, so that
+// an item's epilogue overlaps the next item's MMAs entirely (96 B of copies per clock, in four
+// 48 KB stages).
 //
 // Operands.  K-major A (D and dZ rows for the DGrad kinds): per 128-row half one box of 64 K
 // (128 bytes) x 128 rows, 128-byte swizzle.  MN-major operands (the weights as B of the DGrad
@@ -60,13 +63,14 @@ constexpr int BW_RING = 8;
 constexpr int BW_EPI_WARPS = 8;
 constexpr int BW_THREADS = 32 * (3 + BW_EPI_WARPS);
 constexpr int BW_STORE_WARP = 2 + BW_EPI_WARPS;
-constexpr int BW_NBARS = 2 * BW_ST + 8 + 2 * BW_RING;
+constexpr int BW_ST_MAX = 4;  // barrier slots for the pipeline stages
+constexpr int BW_NBARS = 2 * BW_ST_MAX + 9 + 2 * BW_RING;
 constexpr int BW_META = 512;
 constexpr int BW_SMEM = BW_ST * BW_STAGE + BW_STG_BYTES + BW_META + 1024;
 constexpr int BW_RPH = 4;  // WGrad: store rounds of 64 columns per accumulator half
-// DGRAD_A: rounds of 32 columns (8 per half) through two 16 KB staging buffers, each holding
+// DGRAD_A: rounds of 32 columns (4 per half) through two 16 KB staging buffers, each holding
 // the round's G and U boxes (32 rows x 64 bytes per TMEM lane quadrant, no swizzle)
-constexpr int BWA_RPH = 8;
+constexpr int BWA_RPH = 4;
 constexpr int BWA_BUF = 16384;
 static_assert(BW_NBARS * 8 + 4 * (2 + BW_RING) <= BW_META, "meta");
 static_assert(BW_SMEM <= 227 * 1024, "smem");
@@ -76,11 +80,19 @@ struct BwGeo {
   static constexpr bool DGRAD = KIND == BWD_DGRAD_A || KIND == BWD_DGRAD_X;
   static constexpr bool A_MN = !DGRAD;                // WGrad: both operands MN-major
   static constexpr bool STORES = KIND != BWD_DGRAD_X;  // the store warp takes items
-  static constexpr int ST = BW_ST;  // pipeline stages
+  // DGRAD_A: items of 128 dA columns with two accumulators (of 2 x 128 TMEM columns each),
+  // so that an item's epilogue, the heavy part of this product, overlaps the next item's
+  // MMAs entirely; its copies are 48 KB per K step (96 B per tensor-core clock, above the
+  // 64 of the 256-column item, a price the epilogue-bound product can pay), in 4 stages
+  static constexpr bool DBUF = KIND == BWD_DGRAD_A;
+  static constexpr int N = DBUF ? 128 : BW_N;  // MMA N = output columns per item
+  static constexpr int B_BYTES = N * BW_K * 2;
+  static constexpr int STAGE = BW_A_BYTES + B_BYTES;
+  static constexpr int ST = DBUF ? 4 : BW_ST;  // pipeline stages
   // kind::f16: D fp32, A and B bf16, A / B major bits, N >> 3 at bit 17, M >> 4 at bit 24
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
                                     ((A_MN ? 1u : 0u) << 15) | (1u << 16) |
-                                    ((uint32_t)(BW_N >> 3) << 17) |
+                                    ((uint32_t)((DBUF ? 128 : BW_N) >> 3) << 17) |
                                     ((uint32_t)(BW_H >> 4) << 24);
 };
 
@@ -116,7 +128,7 @@ __device__ __forceinline__ BwItem bw_item(const BwArgs& a, int L) {
   if constexpr (BwGeo<KIND>::DGRAD) {
     // (planner tile, n-tile), the n-tiles of a tile together
     const int m = L / a.n_n;
-    it.n0 = (L - m * a.n_n) * BW_N;
+    it.n0 = (L - m * a.n_n) * BwGeo<KIND>::N;
     const int4 v = __ldg(reinterpret_cast<const int4*>(a.tiles) + m);
     it.e = v.x;
     it.row0 = v.y;
@@ -135,7 +147,7 @@ __device__ __forceinline__ BwItem bw_item(const BwArgs& a, int L) {
     const int r = L - it.e * per_e;
     const int mt = r / a.n_n;
     it.m0 = mt * BW_M;
-    it.n0 = (r - mt * a.n_n) * BW_N;
+    it.n0 = (r - mt * a.n_n) * BwGeo<KIND>::N;
     const int b0 = __ldg(a.block_off + it.e), b1 = __ldg(a.block_off + it.e + 1);
     it.row0 = a.beta * b0;
     it.nrows = a.beta * (b1 - b0);
@@ -164,29 +176,34 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   constexpr int ST = G::ST;
-  uint8_t* stg = smem + ST * BW_STAGE;
+  static_assert(G::ST * G::STAGE <= BW_ST * BW_STAGE && G::ST <= BW_ST_MAX, "stages");
+  uint8_t* stg = smem + BW_ST * BW_STAGE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(stg + BW_STG_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + BW_NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int B0 = 2 * BW_ST_MAX;
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
-  auto empty_bar = [&](int s) { return smem_u32(bars + BW_ST + s); };
-  const uint32_t drain_bar = smem_u32(bars + 2 * BW_ST);
-  const uint32_t tfull_bar = smem_u32(bars + 2 * BW_ST + 1);
-  // tfree[h]: the epilogue has read accumulator half h (TMEM columns [256 h, +256))
-  auto tfree_bar = [&](int h) { return smem_u32(bars + 2 * BW_ST + 2 + h); };
-  const uint32_t staged_bar = smem_u32(bars + 2 * BW_ST + 4);
-  const uint32_t stgfree_bar = smem_u32(bars + 2 * BW_ST + 5);
+  auto empty_bar = [&](int s) { return smem_u32(bars + BW_ST_MAX + s); };
+  const uint32_t drain_bar = smem_u32(bars + B0);
+  // tfull[b]: accumulator b complete (one accumulator, b = 0, except for DGRAD_A)
+  auto tfull_b = [&](int b) { return smem_u32(bars + (b ? B0 + 8 : B0 + 1)); };
+  const uint32_t tfull_bar = tfull_b(0);
+  // tfree[h]: the epilogue has read accumulator half h (TMEM columns [256 h, +256)); for
+  // DGRAD_A, tfree[b]: it has read accumulator b (columns [256 b, +256))
+  auto tfree_bar = [&](int h) { return smem_u32(bars + B0 + 2 + h); };
+  const uint32_t staged_bar = smem_u32(bars + B0 + 4);
+  const uint32_t stgfree_bar = smem_u32(bars + B0 + 5);
   // DGRAD_A, staging buffer b: zfull[b] its G and U copies have landed, dstaged[b] the
   // epilogue has written its results
-  auto zfull_bar = [&](int b) { return b ? smem_u32(bars + 2 * BW_ST + 6) : stgfree_bar; };
-  auto dstaged_bar = [&](int b) { return b ? smem_u32(bars + 2 * BW_ST + 7) : staged_bar; };
-  auto ifull_bar = [&](int i) { return smem_u32(bars + 2 * BW_ST + 8 + i); };
-  auto iempty_bar = [&](int i) { return smem_u32(bars + 2 * BW_ST + 8 + BW_RING + i); };
-  auto sA = [&](int s) { return smem_u32(smem + s * BW_STAGE); };
-  auto sB = [&](int s) { return smem_u32(smem + s * BW_STAGE + BW_A_BYTES); };
+  auto zfull_bar = [&](int b) { return b ? smem_u32(bars + B0 + 6) : stgfree_bar; };
+  auto dstaged_bar = [&](int b) { return b ? smem_u32(bars + B0 + 7) : staged_bar; };
+  auto ifull_bar = [&](int i) { return smem_u32(bars + B0 + 9 + i); };
+  auto iempty_bar = [&](int i) { return smem_u32(bars + B0 + 9 + BW_RING + i); };
+  auto sA = [&](int s) { return smem_u32(smem + s * G::STAGE); };
+  auto sB = [&](int s) { return smem_u32(smem + s * G::STAGE + BW_A_BYTES); };
 
   long long total;
   if constexpr (G::DGRAD)
@@ -200,7 +217,8 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       mbar_init(empty_bar(s), 1);
     }
     mbar_init(drain_bar, 1);
-    mbar_init(tfull_bar, 1);
+    mbar_init(tfull_b(0), 1);
+    mbar_init(tfull_b(1), 1);
     mbar_init(tfree_bar(0), BW_EPI_WARPS);
     mbar_init(tfree_bar(1), BW_EPI_WARPS);
     mbar_init(staged_bar, BW_EPI_WARPS);
@@ -262,12 +280,12 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           // the epilogue reads the item's G and U columns (256 rows x 256 each): bring them
           // into L2 while the item's MMAs run
           for (int r0 = 0; r0 < w.nrows; r0 += 32)
-            for (int c = 0; c < BW_N / 32; ++c) {
+            for (int c = 0; c < G::N / 32; ++c) {
               tma_prefetch_l2_2d(&tmZ, w.n0 + 32 * c, w.row0 + r0);
               tma_prefetch_l2_2d(&tmZ, a.f + w.n0 + 32 * c, w.row0 + r0);
             }
         }
-        const uint32_t tx = G::DGRAD ? (w.two ? 2 : 1) * BW_HALF_A + BW_B_BYTES : BW_STAGE;
+        const uint32_t tx = G::DGRAD ? (w.two ? 2 : 1) * BW_HALF_A + G::B_BYTES : G::STAGE;
         bool stop = false;
         for (int kb = 0; kb < w.nk; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status, a.timeout_ns,
@@ -280,7 +298,7 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           // its token rows)
           const int krow = G::DGRAD ? w.e * a.k_rows + kb * BW_K : w.row0 + kb * BW_K;
 #pragma unroll
-          for (int j = 0; j < BW_N / 64; ++j)
+          for (int j = 0; j < G::N / 64; ++j)
             tma_load_2d(sB(stage) + j * 8192, &tmB, full_bar(stage), w.n0 + 64 * j, krow);
           if constexpr (G::A_MN) {
 #pragma unroll
@@ -329,6 +347,43 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const BwItem w = bw_item<KIND>(a, L);
         if (!w.ok || w.zero) continue;
         const bool two = w.two;
+        if constexpr (G::DBUF) {
+          // accumulator b = acc_it % 2 (TMEM columns [256 b, +256): rows 0..127 at +0, rows
+          // 128..255 at +128), free once the epilogue has read its previous item
+          const int b = acc_it & 1;
+          if (!mbar_wait(tfree_bar(b), ((uint32_t)(acc_it >> 1) & 1u) ^ 1u, abort_flag,
+                         a.status, a.timeout_ns, true))
+            break;
+          tc_fence_after();
+          const uint32_t d0 = tmem_base + 256 * b;
+          bool stop = false;
+          for (int kb = 0; kb < w.nk; ++kb) {
+            if (!mbar_wait(full_bar(stage), phase, abort_flag, a.status, a.timeout_ns, true)) {
+              stop = true;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = sA(stage), b0 = sB(stage);
+#pragma unroll
+            for (int kk = 0; kk < BW_K / 16; ++kk) {
+              umma_bf16<false>(d0, a_desc(a0, 0, kk), sw128_mn_desc(b0 + kk * 2048), G::IDESC,
+                               (kb | kk) != 0);
+              if (two)
+                umma_bf16<false>(d0 + G::N, a_desc(a0, 1, kk), sw128_mn_desc(b0 + kk * 2048),
+                                 G::IDESC, (kb | kk) != 0);
+            }
+            issued = true;
+            umma_commit_all<false>(empty_bar(stage));
+            if (++stage == ST) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (stop) break;
+          umma_commit_all<false>(tfull_b(b));
+          ++acc_it;
+          continue;
+        }
         const uint32_t par = ((uint32_t)acc_it & 1u) ^ 1u;  // the previous item's phase
         // the previous item's first accumulator half has been read out
         if (!mbar_wait(tfree_bar(0), par, abort_flag, a.status, a.timeout_ns, true)) break;
@@ -341,7 +396,7 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const uint32_t a0 = sA(st), b0 = sB(st);
 #pragma unroll
           for (int kk = 0; kk < BW_K / 16; ++kk)
-            umma_bf16<false>(tmem_base + BW_N, a_desc(a0, 1, kk), sw128_mn_desc(b0 + kk * 2048),
+            umma_bf16<false>(tmem_base + G::N, a_desc(a0, 1, kk), sw128_mn_desc(b0 + kk * 2048),
                              G::IDESC, (kb | kk) != 0);
           umma_commit_all<false>(empty_bar(st));
         };
@@ -417,13 +472,16 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const BwItem w = bw_item<KIND>(a, L);
       if (!w.ok) continue;
       const int halves = w.two ? 2 : 1;
+      // DGRAD_A: accumulator acc_it % 2, its (acc_it / 2)-th use; otherwise the one
+      // accumulator, one phase per item
+      const int abuf = G::DBUF ? (acc_it & 1) : 0;
+      const uint32_t apar = G::DBUF ? (uint32_t)(acc_it >> 1) & 1u : (uint32_t)acc_it & 1u;
       if (!w.zero) {
-        const bool got = wait_inl(tfull_bar, (uint32_t)acc_it & 1u, abort_flag, a.status,
-                                  a.timeout_ns);
+        const bool got = wait_inl(tfull_b(abuf), apar, abort_flag, a.status, a.timeout_ns);
         if (!__all_sync(0xffffffffu, got)) break;
         tc_fence_after();
       }
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + 256 * abuf;
       bool ok = true;
       if constexpr (KIND == BWD_DGRAD_X) {
         // dx[token] += dX over columns [n0 + 128 ch, +128) for this warp's 32 rows of each
@@ -537,15 +595,13 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             break;
           }
           uint32_t v[16];
-          tmem_ld16(taddr + BW_N * h + 32 * rnd + 16 * ch, v);
+          tmem_ld16(taddr + G::N * h + 32 * rnd + 16 * ch, v);
           tmem_wait_ld();
-          if (rnd == BWA_RPH - 1) {
+          if (hr == halves * BWA_RPH - 1) {
+            // the item's accumulator has been read: the MMAs of the item after next may use it
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-              mbar_arrive(tfree_bar(h));
-              if (halves == 1) mbar_arrive(tfree_bar(1));
-            }
+            if (lane == 0) mbar_arrive(tfree_bar(abuf));
           }
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
@@ -702,10 +758,10 @@ cudaError_t launch_kind(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
 }  // namespace
 
 bool bwd_wide_supported(const moe_cfg& c, int kind) {
-  // N of dA and of dW2 is f: whole 256-column n-tiles; the other kinds' N and M are d and
-  // 2f, multiples of 256 for every layer the FFN accepts
-  if (kind == BWD_DGRAD_A || kind == BWD_WGRAD_2) return c.f % 256 == 0;
-  return kind == BWD_DGRAD_X || kind == BWD_WGRAD_1;
+  // N of dW2 is f: whole 256-column n-tiles; dA's items are 128 columns wide, and the other
+  // kinds' N and M are d and 2f, multiples of 256 for every layer the FFN accepts
+  if (kind == BWD_WGRAD_2) return c.f % 256 == 0;
+  return kind == BWD_DGRAD_A || kind == BWD_DGRAD_X || kind == BWD_WGRAD_1;
 }
 
 cudaError_t launch_bwd_wide(const moe_cfg& c, int kind, const uint16_t* a_src,
@@ -739,7 +795,7 @@ cudaError_t launch_bwd_wide(const moe_cfg& c, int kind, const uint16_t* a_src,
           !encode_2d_plain(&tz, z, 2 * c.f, r_max, 32, 32))
         return cudaErrorInvalidValue;
       a.n_k = c.d / BW_K;
-      a.n_n = c.f / BW_N;
+      a.n_n = c.f / BwGeo<BWD_DGRAD_A>::N;
       a.k_rows = c.d;
       return launch_kind<BWD_DGRAD_A>(ta, tb, to, tz, a, st);
     case BWD_DGRAD_X:  // A = dZ rows (K = 2f), B = w1 (K rows e 2f + k, N = d), out = dx
