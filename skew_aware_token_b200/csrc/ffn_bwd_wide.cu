@@ -13,9 +13,9 @@
 // columns.  The two 128 x 256 fp32 accumulators fill the 512 TMEM columns; the epilogue frees
 // them half by half, and the next item's second-half MMAs may lag its first-half MMAs by up to
 // the three pipeline stages, as in the forward.  DGRAD_A, whose epilogue takes about as long
-// as its MMAs, uses items of 128 columns instead: two accumulators of 2 x 128 columns, so that
-// an item's epilogue overlaps the next item's MMAs entirely (96 B of copies per clock, in four
-// 48 KB stages).
+// as its MMAs, uses items of 128 columns instead, with two accumulators of 2 x 128 columns, so
+// that an item's epilogue overlaps the next item's MMAs entirely (96 B of copies per clock, in
+// four 48 KB stages); so does dW2 when f is not a multiple of 256.
 //
 // Operands.  K-major A (D and dZ rows for the DGrad kinds): per 128-row half one box of 64 K
 // (128 bytes) x 128 rows, 128-byte swizzle.  MN-major operands (the weights as B of the DGrad
@@ -36,10 +36,10 @@
 //   DGRAD_X  dx[token] += dX with 16-byte vector reductions, each warp transposing 32 x 32
 //            chunks through its own 4 KB slot (as the forward's fused combine, gate 1: the
 //            gate is already in D).
-//   WGRAD    dW fp32: each epilogue warp reads its 128 columns of a half into registers and
-//            frees the half, then stages them in rounds of 64 columns (32-row x 128-byte
-//            fp32 boxes, 128-byte swizzle).  An idle expert's items issue no MMA and stage
-//            zeros.
+//   WGRAD    dW fp32: each epilogue warp reads its columns of a half (128 of 256-column
+//            items) into registers and frees the half, then stages them in rounds of 64
+//            columns (32-row x 128-byte fp32 boxes, 128-byte swizzle).  An idle expert's items
+//            issue no MMA and stage zeros.
 // Roles (352 threads, one CTA per SM, persistent): warp 0 TMA producer, warp 1 MMA issuer,
 // warps 2..9 epilogue (warp w reads TMEM lanes 32 (w % 4) .. +31, and half of each round's
 // columns), warp 10 store warp (idle for DGRAD_X).  Items come from a global counter in
@@ -67,7 +67,8 @@ constexpr int BW_ST_MAX = 4;  // barrier slots for the pipeline stages
 constexpr int BW_NBARS = 2 * BW_ST_MAX + 9 + 2 * BW_RING;
 constexpr int BW_META = 512;
 constexpr int BW_SMEM = BW_ST * BW_STAGE + BW_STG_BYTES + BW_META + 1024;
-constexpr int BW_RPH = 4;  // WGrad: store rounds of 64 columns per accumulator half
+// dW2 on items of 128 columns (when f is not a multiple of 256): an internal kind
+constexpr int BW_WGRAD_2_N128 = 5;
 // DGRAD_A: rounds of 32 columns (4 per half) through two 16 KB staging buffers, each holding
 // the round's G and U boxes (32 rows x 64 bytes per TMEM lane quadrant, no swizzle)
 constexpr int BWA_RPH = 4;
@@ -80,11 +81,12 @@ struct BwGeo {
   static constexpr bool DGRAD = KIND == BWD_DGRAD_A || KIND == BWD_DGRAD_X;
   static constexpr bool A_MN = !DGRAD;                // WGrad: both operands MN-major
   static constexpr bool STORES = KIND != BWD_DGRAD_X;  // the store warp takes items
-  // DGRAD_A: items of 128 dA columns with two accumulators (of 2 x 128 TMEM columns each),
-  // so that an item's epilogue, the heavy part of this product, overlaps the next item's
-  // MMAs entirely; its copies are 48 KB per K step (96 B per tensor-core clock, above the
-  // 64 of the 256-column item, a price the epilogue-bound product can pay), in 4 stages
-  static constexpr bool DBUF = KIND == BWD_DGRAD_A;
+  // DGRAD_A: items of 128 columns with two accumulators (of 2 x 128 TMEM columns each), so
+  // that an item's epilogue, the heavy part of this product, overlaps the next item's MMAs
+  // entirely; its copies are 48 KB per K step (96 B per tensor-core clock, above the 64 of
+  // the 256-column item, a price the epilogue-bound product can pay), in 4 stages.  dW2 takes
+  // the same shape when f is not a multiple of 256.
+  static constexpr bool DBUF = KIND == BWD_DGRAD_A || KIND == BW_WGRAD_2_N128;
   static constexpr int N = DBUF ? 128 : BW_N;  // MMA N = output columns per item
   static constexpr int B_BYTES = N * BW_K * 2;
   static constexpr int STAGE = BW_A_BYTES + B_BYTES;
@@ -533,30 +535,34 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
         }
       } else if constexpr (!G::DGRAD) {
-        // WGrad: the warp reads all 128 of its columns of a half (64 r + 32 ch .. +32 for the
-        // rounds r = 0..3) into registers and frees the half, so that the next item's MMAs
-        // restart after the TMEM reads alone; the four store rounds (32 fp32 columns each into
-        // box (quarter, ch)) then go out of registers while those MMAs run.  An idle expert's
-        // item stages zeros.
+        // WGrad: the warp reads all its columns of a half (64 r + 32 ch .. +32 for the rounds
+        // r < RW) into registers, then stages them in RW rounds (32 fp32 columns each into box
+        // (quarter, ch)).  256-column items free each half after its reads, so that the next
+        // item's MMAs restart after the TMEM reads alone; 128-column items free the
+        // accumulator, for the item after next, after the second half's reads.  An idle
+        // expert's item stages zeros.
+        constexpr int RW = G::N / 64;  // store rounds of 64 columns per half
         uint8_t* box = stg + quarter * 8192 + ch * 4096;
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
-          uint32_t v[4][32];
+          uint32_t v[RW][32];
           if (!w.zero) {
 #pragma unroll
-            for (int r = 0; r < BW_RPH; ++r) tmem_ld32(taddr + BW_N * h + 64 * r + 32 * ch, v[r]);
+            for (int r = 0; r < RW; ++r) tmem_ld32(taddr + G::N * h + 64 * r + 32 * ch, v[r]);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tfree_bar(h));
+            if (!G::DBUF || h == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(tfree_bar(G::DBUF ? abuf : h));
+            }
           } else {
 #pragma unroll
-            for (int r = 0; r < BW_RPH; ++r)
+            for (int r = 0; r < RW; ++r)
 #pragma unroll
               for (int i = 0; i < 32; ++i) v[r][i] = 0u;
           }
 #pragma unroll
-          for (int r = 0; r < BW_RPH; ++r) {
+          for (int r = 0; r < RW; ++r) {
             // the staging buffer is free once the store warp's copies have read the last round
             const bool fr = wait_inl(stgfree_bar, ((uint32_t)staged_n & 1u) ^ 1u, abort_flag,
                                      a.status, a.timeout_ns);
@@ -700,6 +706,7 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       } else {
         // WGrad: one staging buffer; per round the epilogue's fp32 boxes out, then the
         // buffer is free for the next round
+        constexpr int RW = G::N / 64;  // store rounds of 64 columns per half
         int staged_n = 0;
         for (int it = 0;; ++it) {
           const int L = take_item(it);
@@ -709,8 +716,8 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const BwItem w = bw_item<KIND>(a, L);
           if (!w.ok) continue;
           bool stop = false;
-          for (int hr = 0; hr < 2 * BW_RPH; ++hr) {
-            const int h = hr / BW_RPH, rnd = hr % BW_RPH;
+          for (int hr = 0; hr < 2 * RW; ++hr) {
+            const int h = hr / RW, rnd = hr % RW;
             if (!mbar_wait(staged_bar, (uint32_t)staged_n & 1u, abort_flag, a.status,
                            a.timeout_ns, true)) {
               stop = true;
@@ -758,10 +765,10 @@ cudaError_t launch_kind(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
 }  // namespace
 
 bool bwd_wide_supported(const moe_cfg& c, int kind) {
-  // N of dW2 is f: whole 256-column n-tiles; dA's items are 128 columns wide, and the other
-  // kinds' N and M are d and 2f, multiples of 256 for every layer the FFN accepts
-  if (kind == BWD_WGRAD_2) return c.f % 256 == 0;
-  return kind == BWD_DGRAD_A || kind == BWD_DGRAD_X || kind == BWD_WGRAD_1;
+  // N and M are d, f or 2f: multiples of 128 (d of 256) for every layer the FFN accepts, and
+  // items 128 or 256 columns wide
+  (void)c;
+  return kind >= BWD_DGRAD_A && kind <= BWD_WGRAD_1;
 }
 
 cudaError_t launch_bwd_wide(const moe_cfg& c, int kind, const uint16_t* a_src,
@@ -813,16 +820,20 @@ cudaError_t launch_bwd_wide(const moe_cfg& c, int kind, const uint16_t* a_src,
           !encode_2d_f32(&to, out, c.f, (uint64_t)c.E * c.d, 32))
         return cudaErrorInvalidValue;
       a.n_m = c.d / BW_M;
-      a.n_n = c.f / BW_N;
       a.m_rows = c.d;
-      return launch_kind<BWD_WGRAD_2>(ta, tb, to, to, a, st);
+      if (c.f % 256 == 0) {
+        a.n_n = c.f / BwGeo<BWD_WGRAD_2>::N;
+        return launch_kind<BWD_WGRAD_2>(ta, tb, to, to, a, st);
+      }
+      a.n_n = c.f / BwGeo<BW_WGRAD_2_N128>::N;
+      return launch_kind<BW_WGRAD_2_N128>(ta, tb, to, to, a, st);
     default:  // BWD_WGRAD_1: A = dZ (M = 2f), B = Xp rows (N = d), K = the expert's rows
       if (!encode_2d(&ta, a_src, 2 * c.f, r_max, BW_K) ||
           !encode_2d(&tb, b_src, c.d, r_max, BW_K) ||
           !encode_2d_f32(&to, out, c.d, (uint64_t)c.E * 2 * c.f, 32))
         return cudaErrorInvalidValue;
       a.n_m = 2 * c.f / BW_M;
-      a.n_n = c.d / BW_N;
+      a.n_n = c.d / BwGeo<BWD_WGRAD_1>::N;
       a.m_rows = 2 * c.f;
       return launch_kind<BWD_WGRAD_1>(ta, tb, to, to, a, st);
   }
