@@ -33,6 +33,8 @@ CASES = [
     Workload("idle_experts", T=24, d=256, E=32, k=1, f=256, beta=64, P=4, s=1, alpha=2.0),
     # every product on whole 256-row tiles, several n- and m-tiles, skewed experts
     Workload("wide_skew", T=2048, d=1024, E=16, k=4, f=512, beta=128, P=4, s=2, alpha=1.0),
+    # f not a multiple of 256: dW2 on 128-column items, several of them per expert
+    Workload("wide_skew_f384", T=1536, d=768, E=12, k=4, f=384, beta=64, P=4, s=2, alpha=1.0),
 ]
 
 
