@@ -356,7 +356,8 @@ def roofline(wl, ffn_ms, ffn_timed_s, peaks, peak_src, traffic=None):
             "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
             "peak_source": f"bf16 {kind} {peak_src} (FFN timed {ffn_timed_s:.3f} s in total; "
-                           f"burst below {SUSTAINED_AFTER_S:g} s)",
+                           f"the burst peak applies below {SUSTAINED_AFTER_S:g} s of FFN "
+                           f"time, the sustained one from there on)",
             "frac_of_burst": round(achieved / burst, 4),
             "frac_of_sustained": round(achieved / sustained, 4),
             "traffic": traffic, "flops_per_launch": wl.flops, "ms_per_launch": round(ffn_ms, 4)}
