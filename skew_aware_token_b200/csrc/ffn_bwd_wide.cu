@@ -94,7 +94,7 @@ struct BwGeo {
   // kind::f16: D fp32, A and B bf16, A / B major bits, N >> 3 at bit 17, M >> 4 at bit 24
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
                                     ((A_MN ? 1u : 0u) << 15) | (1u << 16) |
-                                    ((uint32_t)((DBUF ? 128 : BW_N) >> 3) << 17) |
+                                    ((uint32_t)(N >> 3) << 17) |
                                     ((uint32_t)(BW_H >> 4) << 24);
 };
 
@@ -110,7 +110,7 @@ struct BwArgs {
   long long r_max;
   int T, d, f, E, beta;
   int n_k;     // DGrad: K steps of 64
-  int n_n;     // n-tiles of 256 columns
+  int n_n;     // n-tiles (of the kind's N columns)
   int n_m;     // WGrad: m-tiles of 256 rows per expert
   int k_rows;  // DGrad: first B row of expert e is e * k_rows (d for w2, 2f for w1)
   int m_rows;  // WGrad: rows of one expert's gradient (d for dW2, 2f for dW1)
@@ -279,8 +279,8 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         if (w.zero) continue;
         if constexpr (KIND == BWD_DGRAD_A) {
-          // the epilogue reads the item's G and U columns (256 rows x 256 each): bring them
-          // into L2 while the item's MMAs run
+          // the epilogue reads the item's G and U columns (up to 256 rows x 128 of each):
+          // bring them into L2 while the item's MMAs run
           for (int r0 = 0; r0 < w.nrows; r0 += 32)
             for (int c = 0; c < G::N / 32; ++c) {
               tma_prefetch_l2_2d(&tmZ, w.n0 + 32 * c, w.row0 + r0);
@@ -296,8 +296,8 @@ bw_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             break;
           }
           mbar_expect_tx(full_bar(stage), tx);
-          // B: 256 MN-major columns of the K rows (DGrad: the expert's weight rows; WGrad:
-          // its token rows)
+          // B: the item's N columns, MN-major, of the K rows (DGrad: the expert's weight rows;
+          // WGrad: its token rows)
           const int krow = G::DGRAD ? w.e * a.k_rows + kb * BW_K : w.row0 + kb * BW_K;
 #pragma unroll
           for (int j = 0; j < G::N / 64; ++j)
