@@ -146,3 +146,21 @@ def test_backward_repeatable_and_forward_unchanged():
     layer.backward(dy.cuda(), w1, w2)
     torch.cuda.synchronize()
     assert torch.equal(layer.view("dw1"), dw1)  # no atomics in the weight gradients
+
+
+def test_backward_empty_input():
+    """A layer with no tokens: the weight gradients come out zero and the status stays
+    clean (one-element buffers stand in for the empty inputs)."""
+    wl = CASES[0].with_(T=0)
+    layer = MoeLayer(wl, "cuda", train=True)
+    layer.clear_status()
+    w1 = torch.zeros(wl.E, 2 * wl.f, wl.d, dtype=torch.bfloat16, device="cuda")
+    w2 = torch.zeros(wl.E, wl.d, wl.f, dtype=torch.bfloat16, device="cuda")
+    layer(torch.zeros(1, wl.E, device="cuda"),
+          torch.zeros(1, wl.d, dtype=torch.bfloat16, device="cuda"), w1, w2)
+    layer.dw1.fill_(float("nan"))
+    layer.dw2.fill_(float("nan"))
+    layer.backward(torch.zeros(1, wl.d, device="cuda"), w1, w2)
+    torch.cuda.synchronize()
+    assert layer.read_status() == 0
+    assert not layer.view("dw1").any() and not layer.view("dw2").any()
